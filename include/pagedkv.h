@@ -1,0 +1,247 @@
+/*
+ * pagedkv.h - C ABI of libpagedkv: PagedAttention's data-parallel decode path
+ * on NVIDIA B200 (sm_100a), plus the host block manager that feeds it.
+ *
+ * Sources (web pages on PagedAttention, cited by page title and section):
+ *   [Q] "What is PagedAttention?" (qubittool.com glossary), How It Works:
+ *       Map Logical to Physical Blocks; Share Without Mutating State.
+ *   [K] "PagedAttention" (kongchang.com knowledge page), Core Facts.
+ *   [G] "PagedAttention: Optimizing KV Cache in vLLM" (grasp.study lesson),
+ *       section 2 (The Solution), section 3 (Making it Work: The PagedAttention
+ *       Kernel), section 4 (Zero-Cost Sharing with Copy-on-Write).
+ *
+ * Conventions for every call below
+ * --------------------------------
+ * - All tensors are caller-owned. Device pointers must point to memory on the
+ *   current CUDA device; the library never frees or keeps them after return.
+ *   No kernel entry point allocates device memory.
+ * - Every kernel entry point enqueues work on `stream` (a cudaStream_t passed
+ *   as void*; NULL is the legacy default stream) and returns without
+ *   synchronising. A PA_OK return means the launch was accepted.
+ * - Layouts (row-major, contiguous, no padding):
+ *     k_pool, v_pool : [num_blocks][num_kv_heads][block_size][head_dim]
+ *                      One (physical block, KV head) tile is contiguous.
+ *     q, out         : [num_seqs][num_q_heads][head_dim]
+ *     block_tables   : int32 [num_seqs][max_blocks_per_seq]; entry [s][i] is the
+ *                      physical block of logical block i of sequence s [Q].
+ *                      Entries at or past ceil(ctx_s / block_size) are never read.
+ *     context_lens   : int32 [num_seqs], tokens held by each sequence.
+ *     slot_mapping   : int64 [num_tokens], slot = block * block_size + offset;
+ *                      a negative slot is padding and writes nothing.
+ * - Query head h reads KV head h / (num_q_heads / num_kv_heads): consecutive
+ *   query heads share one KV head (grouped-query attention, [K]).
+ * - dtype is PA_F32 (all of q, pools, out fp32) or PA_BF16 (all bf16);
+ *   arithmetic is fp32 in both cases. out has q's dtype.
+ * - Supported shapes: head_dim in {64, 128, 256} (256 for bf16 only),
+ *   block_size in {16, 32}; bf16 takes any group size 1..16, fp32 takes group
+ *   sizes 1, 2, 4, 8. num_blocks * num_kv_heads * block_size < 2^31.
+ *   Pointers to pools, q, out, k_new and v_new must be 16-byte aligned.
+ * - Errors: invalid arguments are rejected before anything is enqueued
+ *   (PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED, nothing changes). Kernels never
+ *   trap: an index found out of range on the device (a block id outside
+ *   [0, num_blocks), a context length outside [0, max_blocks_per_seq *
+ *   block_size], a slot past the pool) sets a PA_DEVERR_* bit in *dev_err (when
+ *   dev_err is non-NULL, atomically OR-ed, never cleared by the library) and
+ *   the offending access is skipped. The text of the last host-side error of
+ *   the calling thread is returned by pa_last_error_string().
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,     /* bad pointer, size, shape or alignment */
+  PA_ERR_NO_FREE_BLOCKS = 2,  /* block manager out of blocks; state unchanged */
+  PA_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
+  PA_ERR_UNSUPPORTED = 4      /* valid request outside the compiled shapes */
+} pa_status_t;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype_t;
+
+/* Bits OR-ed into the optional device error word. */
+#define PA_DEVERR_BLOCK_ID 0x1u     /* block table entry outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 0x2u  /* context length < 0 or > max_blocks_per_seq*block_size */
+#define PA_DEVERR_SLOT 0x4u         /* slot >= num_blocks * block_size */
+#define PA_DEVERR_COPY_PAIR 0x8u    /* copy pair index outside [0, num_blocks) */
+#define PA_DEVERR_TIMEOUT 0x10u     /* a pipeline wait hit its time limit; output invalid */
+
+/* Library version string, e.g. "pagedkv 0.1 sm_100a". */
+const char* pa_version(void);
+/* Text of the last error reported to the calling thread ("" if none). */
+const char* pa_last_error_string(void);
+/* Static name of a status code. */
+const char* pa_status_string(pa_status_t status);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode - single-query decode attention over the paged KV cache.
+ *
+ * For every sequence s and query head h:
+ *     out[s][h] = softmax(scale * K_s q[s][h]) V_s
+ * where K_s, V_s are the first context_lens[s] tokens of KV head
+ * h / (num_q_heads / num_kv_heads), gathered in logical order through
+ * block_tables[s]. The kernel walks the blocks in logical order with a
+ * running-max softmax, so the result equals attention over a contiguous copy
+ * of the sequence ([G] section 3; the table indirection is [Q], Map Logical to
+ * Physical Blocks). A sequence with context length 0 gets zeros.
+ *
+ * One CTA per (sequence, KV head) handles the whole context; for long or
+ * ragged contexts prefer pa_decode_split.
+ * ------------------------------------------------------------------------- */
+pa_status_t pa_decode(const void* q, const void* k_pool, const void* v_pool,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                      int block_size, int num_blocks, int max_blocks_per_seq,
+                      float scale, pa_dtype_t dtype, void* out, uint32_t* dev_err,
+                      void* stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_split - the same result as pa_decode, computed by cutting each
+ * context into partitions of partition_tokens tokens (a multiple of
+ * block_size). Each (sequence, KV head, partition) produces a running max, a
+ * running sum and an unnormalised accumulator; a log-sum-exp merge combines
+ * the partitions. Sequences that fit in one partition are written directly.
+ * The split is a scheduling device for long and ragged contexts; it does not
+ * appear on the pages, which only require that the blockwise walk reproduce
+ * the contiguous result ([G] section 3).
+ *
+ * workspace: caller-owned device memory of at least
+ *   pa_decode_split_workspace_size(...) bytes, 256-byte aligned. Its first 256
+ *   bytes are a control header that must be zero before the first call
+ *   (pa_decode_split_workspace_init does that); every completed call leaves the
+ *   header zero again, so one workspace serves any number of calls issued in
+ *   stream order. Calls that may overlap on the GPU need separate workspaces.
+ * num_seqs must be <= 4096 (PA_ERR_UNSUPPORTED above that).
+ * ------------------------------------------------------------------------- */
+size_t pa_decode_split_workspace_size(int num_seqs, int num_q_heads, int head_dim,
+                                      int block_size, int max_blocks_per_seq,
+                                      int partition_tokens);
+
+pa_status_t pa_decode_split_workspace_init(void* workspace, size_t workspace_bytes,
+                                           void* stream);
+
+pa_status_t pa_decode_split(const void* q, const void* k_pool, const void* v_pool,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            int num_seqs, int num_q_heads, int num_kv_heads,
+                            int head_dim, int block_size, int num_blocks,
+                            int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                            int partition_tokens, void* workspace,
+                            size_t workspace_bytes, void* out, uint32_t* dev_err,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_kv_append - decode-step write of new tokens' keys and values into their
+ * slots ([Q], Map Logical to Physical Blocks: decode appends into the partly
+ * filled tail block; [G] section 4 step 3: the write proceeds on the private
+ * block). k_new, v_new: [num_tokens][num_kv_heads][head_dim] in `dtype`.
+ * Token t goes to block slot/block_size, offset slot%block_size, every KV head.
+ * Bit-exact copy. Slots must be unique within a call (duplicates race).
+ * ------------------------------------------------------------------------- */
+pa_status_t pa_kv_append(const void* k_new, const void* v_new,
+                         const int64_t* slot_mapping, int num_tokens,
+                         int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype_t dtype, void* k_pool,
+                         void* v_pool, uint32_t* dev_err, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_copy_blocks - the data movement of copy-on-write: for each pair
+ * (src, dst) in src_dst_pairs (int64 [num_pairs][2], device memory), copy the
+ * whole physical block (block_bytes = num_kv_heads*block_size*head_dim*elt
+ * bytes, a multiple of 16) from src to dst in both pools ([G] section 4 step
+ * 3; [Q], Share Without Mutating State). Pairs must not chain (no dst is
+ * another pair's src) and dst ids must be unique.
+ * ------------------------------------------------------------------------- */
+pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pairs,
+                           int num_pairs, size_t block_bytes, int num_blocks,
+                           uint32_t* dev_err, void* stream);
+
+/* ===========================================================================
+ * Host block manager ([Q] How It Works; [G] sections 2 and 4).
+ *
+ * An opaque handle owned by the caller (pa_bm_destroy frees it). Not
+ * thread-safe: one thread at a time per handle. Sequence ids are any int64.
+ * Every call is all-or-nothing: on any error status nothing changes.
+ *
+ * Policy (the pages leave it open): free blocks form a FIFO queue seeded from
+ * initial_free_order (identity when NULL); allocation pops the front; a free
+ * call returns the blocks it reclaims to the back in ascending id order.
+ * ========================================================================= */
+typedef struct pa_bm* pa_bm_t;
+
+typedef struct {
+  int64_t num_blocks;
+  int64_t free_blocks;
+  int64_t used_blocks;      /* blocks with reference count > 0 */
+  int64_t shared_blocks;    /* blocks with reference count > 1 */
+  int64_t num_seqs;
+  int64_t logical_tokens;   /* sum of context lengths */
+  int64_t logical_slots;    /* sum of table lengths * block_size */
+  int64_t tail_waste_slots; /* logical_slots - logical_tokens */
+  int64_t cow_copies;       /* copy-on-write copies made so far */
+} pa_bm_stats_t;
+
+/* Create a manager for a pool of num_blocks blocks of block_size tokens; a
+ * sequence may hold at most max_blocks_per_seq blocks. initial_free_order, if
+ * given, is a permutation of 0..num_blocks-1 (host memory, copied). */
+pa_status_t pa_bm_create(int num_blocks, int block_size, int max_blocks_per_seq,
+                         const int32_t* initial_free_order, pa_bm_t* out);
+pa_status_t pa_bm_destroy(pa_bm_t bm);
+
+/* Prefill: a new sequence with num_tokens tokens takes ceil(num_tokens /
+ * block_size) blocks ([Q]). PA_ERR_NO_FREE_BLOCKS if the pool cannot supply
+ * them; PA_ERR_INVALID_ARG for an existing id or more than max_blocks_per_seq. */
+pa_status_t pa_bm_allocate(pa_bm_t bm, int64_t seq_id, int64_t num_tokens);
+
+/* Sharing: child gets the parent's table and context length; every block's
+ * reference count goes up by one; no data moves ([G] section 4 step 1). */
+pa_status_t pa_bm_fork(pa_bm_t bm, int64_t parent_id, int64_t child_id);
+
+/* Decode step for one sequence: reserve the slot of its next token. A full
+ * (or absent) tail takes a new block; a partly filled tail held by more than
+ * one sequence is copied first: a new block is taken, *cow_src/*cow_dst name
+ * the copy the caller must perform (pa_copy_blocks) before writing, only this
+ * sequence's table changes and the shared block's count drops by one ([G]
+ * section 4 steps 2-3). Otherwise *cow_src = *cow_dst = -1. */
+pa_status_t pa_bm_append_slot(pa_bm_t bm, int64_t seq_id, int64_t* slot,
+                              int64_t* cow_src, int64_t* cow_dst);
+
+/* The same for n distinct sequences in the given order, all or nothing.
+ * slots: int64 [n]. cow_pairs: int64 [n][2] receives the copies made, packed
+ * at the front; *num_cow (may be NULL) receives their count. */
+pa_status_t pa_bm_append_slots(pa_bm_t bm, const int64_t* seq_ids, int n,
+                               int64_t* slots, int64_t* cow_pairs, int* num_cow);
+
+/* *ok = 1 if pa_bm_append_slots(seq_ids, n) would succeed now, else 0. */
+pa_status_t pa_bm_can_append(pa_bm_t bm, const int64_t* seq_ids, int n, int* ok);
+
+/* Finish a sequence: counts drop by one; blocks reaching zero are reclaimed. */
+pa_status_t pa_bm_free(pa_bm_t bm, int64_t seq_id);
+
+/* Copy one sequence's block table into row[0..row_capacity); *n_blocks gets
+ * its length (PA_ERR_INVALID_ARG if row_capacity is too small). */
+pa_status_t pa_bm_block_table(pa_bm_t bm, int64_t seq_id, int32_t* row,
+                              int row_capacity, int* n_blocks);
+pa_status_t pa_bm_context_len(pa_bm_t bm, int64_t seq_id, int64_t* context_len);
+
+/* Export a batch: tables int32 [n][max_blocks_per_seq] (unused entries set to
+ * pad_value) and context_lens int32 [n], both host memory, ready to upload
+ * for pa_decode. */
+pa_status_t pa_bm_export(pa_bm_t bm, const int64_t* seq_ids, int n, int32_t* tables,
+                         int32_t* context_lens, int32_t pad_value);
+
+pa_status_t pa_bm_refcount(pa_bm_t bm, int block_id, int* refcount);
+/* Free queue front to back into out[0..capacity); *n gets its length. */
+pa_status_t pa_bm_free_queue(pa_bm_t bm, int32_t* out, int capacity, int* n);
+pa_status_t pa_bm_stats(pa_bm_t bm, pa_bm_stats_t* stats);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* PAGEDKV_H_ */

@@ -1,0 +1,390 @@
+// C-ABI entry points for paged decode attention: argument validation, kernel
+// selection, TMA descriptor encoding and launch (see include/pagedkv.h).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "decode_dispatch.h"
+#include "decode_kernel.cuh"
+#include "pa_internal.h"
+
+namespace pagedkv {
+namespace {
+
+constexpr size_t kWorkspaceHeader = 256;
+constexpr int kMaxSplitSeqs = 4096;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elt_bytes(pa_dtype_t dt) { return dt == PA_F32 ? 4 : 2; }
+
+// ---- cuTensorMapEncodeTiled through the runtime's driver entry point ----------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// A pool [num_blocks][num_kv_heads][block_size][head_dim] viewed as a 2-D
+// tensor of rows = num_blocks*num_kv_heads*block_size, cols = head_dim; one
+// box = block_size rows x 128 bytes, 128-byte swizzle.
+struct MapKey {
+  const void* base;
+  int rows;
+  int head_dim;
+  int block_size;
+  pa_dtype_t dtype;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && rows == o.rows && head_dim == o.head_dim &&
+           block_size == o.block_size && dtype == o.dtype;
+  }
+};
+
+struct MapCache {
+  static constexpr int kSlots = 8;
+  MapKey key[kSlots];
+  CUtensorMap map[kSlots];
+  int used = 0;
+  int next = 0;
+};
+
+pa_status_t pool_tensor_map(const void* base, int rows, int head_dim, int block_size,
+                            pa_dtype_t dtype, CUtensorMap* out) {
+  thread_local MapCache cache;
+  const MapKey k{base, rows, head_dim, block_size, dtype};
+  for (int i = 0; i < cache.used; ++i) {
+    if (cache.key[i] == k) {
+      *out = cache.map[i];
+      return PA_OK;
+    }
+  }
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const int eb = elt_bytes(dtype);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * eb};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(block_size)};
+  cuuint32_t estr[2] = {1, 1};
+  CUtensorMap m;
+  std::memset(&m, 0, sizeof(m));
+  CUresult r = fn(&m, dtype == PA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  const int slot = cache.used < MapCache::kSlots ? cache.used++ : (cache.next++ % MapCache::kSlots);
+  cache.key[slot] = k;
+  cache.map[slot] = m;
+  *out = m;
+  return PA_OK;
+}
+
+struct DecodeReq {
+  const void* q;
+  const void* k_pool;
+  const void* v_pool;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  int num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq;
+  float scale;
+  pa_dtype_t dtype;
+  void* out;
+  uint32_t* dev_err;
+  cudaStream_t stream;
+};
+
+pa_status_t validate_and_pick(const DecodeReq& r, DecodeInstance* inst) {
+  if (r.num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "num_seqs < 0");
+  if (r.q == nullptr || r.k_pool == nullptr || r.v_pool == nullptr || r.block_tables == nullptr ||
+      r.context_lens == nullptr || r.out == nullptr)
+    return fail(PA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (r.num_q_heads <= 0 || r.num_kv_heads <= 0 || r.num_q_heads % r.num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                r.num_q_heads, r.num_kv_heads);
+  if (r.num_blocks <= 0 || r.max_blocks_per_seq <= 0)
+    return fail(PA_ERR_INVALID_ARG, "num_blocks and max_blocks_per_seq must be positive");
+  if (r.dtype != PA_F32 && r.dtype != PA_BF16) return fail(PA_ERR_INVALID_ARG, "unknown dtype");
+  if (!std::isfinite(r.scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+  if (!aligned16(r.q) || !aligned16(r.k_pool) || !aligned16(r.v_pool) || !aligned16(r.out))
+    return fail(PA_ERR_INVALID_ARG, "q, pools and out must be 16-byte aligned");
+  const int64_t rows = static_cast<int64_t>(r.num_blocks) * r.num_kv_heads * r.block_size;
+  if (rows >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID_ARG, "num_blocks * num_kv_heads * block_size must be < 2^31");
+  if (static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID_ARG, "max_blocks_per_seq * block_size must be < 2^31");
+  const int group = r.num_q_heads / r.num_kv_heads;
+  bool found = false;
+  if (r.dtype == PA_F32) {
+    found = find_decode_f32(r.head_dim, r.block_size, group, inst);
+  } else if (group == 1) {
+    found = find_decode_bf16_simt(r.head_dim, r.block_size, group, inst);
+  } else if (group <= 16) {
+    found = find_decode_bf16_mma(r.head_dim, r.block_size, inst);
+  }
+  if (!found)
+    return fail(PA_ERR_UNSUPPORTED,
+                "no kernel for dtype=%s head_dim=%d block_size=%d group=%d",
+                r.dtype == PA_F32 ? "f32" : "bf16", r.head_dim, r.block_size, group);
+  return PA_OK;
+}
+
+// Optional host-side check of the device tables (PAGEDKV_VALIDATE=1): copies
+// block tables and context lengths to the host and checks every entry the
+// kernels will read. Synchronous; meant for tests and debugging.
+pa_status_t host_validate(const DecodeReq& r) {
+  static const bool enabled = [] {
+    const char* e = std::getenv("PAGEDKV_VALIDATE");
+    return e != nullptr && e[0] == '1';
+  }();
+  if (!enabled || r.num_seqs == 0) return PA_OK;
+  std::vector<int32_t> ctx(r.num_seqs);
+  std::vector<int32_t> bt(static_cast<size_t>(r.num_seqs) * r.max_blocks_per_seq);
+  if (cudaMemcpyAsync(ctx.data(), r.context_lens, ctx.size() * 4, cudaMemcpyDeviceToHost, r.stream) != cudaSuccess ||
+      cudaMemcpyAsync(bt.data(), r.block_tables, bt.size() * 4, cudaMemcpyDeviceToHost, r.stream) != cudaSuccess ||
+      cudaStreamSynchronize(r.stream) != cudaSuccess)
+    return fail(PA_ERR_CUDA, "PAGEDKV_VALIDATE copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+  for (int s = 0; s < r.num_seqs; ++s) {
+    if (ctx[s] < 0 || static_cast<int64_t>(ctx[s]) > static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size)
+      return fail(PA_ERR_INVALID_ARG, "context_lens[%d] = %d out of range", s, ctx[s]);
+    const int nb = (ctx[s] + r.block_size - 1) / r.block_size;
+    for (int i = 0; i < nb; ++i) {
+      const int32_t b = bt[static_cast<size_t>(s) * r.max_blocks_per_seq + i];
+      if (b < 0 || b >= r.num_blocks)
+        return fail(PA_ERR_INVALID_ARG, "block_tables[%d][%d] = %d out of range", s, i, b);
+    }
+  }
+  return PA_OK;
+}
+
+int l2_hint_default() {
+  static const int hint = [] {
+    const char* e = std::getenv("PAGEDKV_L2_HINT");
+    if (e == nullptr) return 1;
+    const int v = std::atoi(e);
+    return (v >= 0 && v <= 2) ? v : 1;
+  }();
+  return hint;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+};
+
+pa_status_t device_info(DeviceInfo* info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice failed");
+  static std::mutex mu;
+  static std::vector<int> sms;
+  std::lock_guard<std::mutex> lock(mu);
+  if (static_cast<int>(sms.size()) <= dev) sms.resize(dev + 1, 0);
+  if (sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return fail(PA_ERR_CUDA, "cudaDeviceGetAttribute failed");
+    sms[dev] = n;
+  }
+  info->sms = sms[dev];
+  return PA_OK;
+}
+
+// Raises the kernel's dynamic shared memory limit when needed (per device).
+pa_status_t prepare_kernel(const void* kernel, int smem) {
+  static std::mutex mu;
+  struct Entry {
+    int dev;
+    const void* k;
+    int smem;
+  };
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& e : done) {
+    if (e.dev == dev && e.k == kernel && e.smem >= smem) return PA_OK;
+  }
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess)
+    return fail(PA_ERR_CUDA, "cudaFuncSetAttribute(smem=%d): %s", smem, cudaGetErrorString(err));
+  done.push_back({dev, kernel, smem});
+  return PA_OK;
+}
+
+pa_status_t launch_error(const char* what) {
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+  return ok();
+}
+
+struct SplitLayout {
+  size_t m_off, l_off, acc_off, total;
+  int pmax;
+};
+
+SplitLayout split_layout(int num_seqs, int num_q_heads, int head_dim, int block_size,
+                         int max_blocks_per_seq, int partition_tokens) {
+  SplitLayout L{};
+  const int pb = partition_tokens / block_size;
+  L.pmax = (max_blocks_per_seq + pb - 1) / pb;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * L.pmax;
+  L.m_off = kWorkspaceHeader;
+  L.l_off = L.m_off + align256(rows * 4);
+  L.acc_off = L.l_off + align256(rows * 4);
+  L.total = L.acc_off + align256(rows * head_dim * 4);
+  return L;
+}
+
+pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, void* workspace,
+                       size_t workspace_bytes) {
+  DecodeInstance inst;
+  pa_status_t st = validate_and_pick(r, &inst);
+  if (st != PA_OK) return st;
+  if (r.num_seqs == 0) return ok();
+  st = host_validate(r);
+  if (st != PA_OK) return st;
+
+  DecodeArgs a{};
+  a.q = r.q;
+  a.out = r.out;
+  a.block_tables = r.block_tables;
+  a.context_lens = r.context_lens;
+  a.dev_err = r.dev_err;
+  a.num_seqs = r.num_seqs;
+  a.num_q_heads = r.num_q_heads;
+  a.num_kv_heads = r.num_kv_heads;
+  a.group = r.num_q_heads / r.num_kv_heads;
+  a.num_blocks = r.num_blocks;
+  a.max_blocks_per_seq = r.max_blocks_per_seq;
+  a.scale_log2 = r.scale * 1.4426950408889634f;
+  a.l2_hint = l2_hint_default();
+
+  int smem = inst.fixed_smem;
+  dim3 grid;
+  if (split) {
+    if (partition_tokens <= 0 || partition_tokens % r.block_size != 0)
+      return fail(PA_ERR_INVALID_ARG, "partition_tokens (%d) must be a positive multiple of block_size",
+                  partition_tokens);
+    if (r.num_seqs > kMaxSplitSeqs)
+      return fail(PA_ERR_UNSUPPORTED, "pa_decode_split takes at most %d sequences", kMaxSplitSeqs);
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+    const SplitLayout L = split_layout(r.num_seqs, r.num_q_heads, r.head_dim, r.block_size,
+                                       r.max_blocks_per_seq, partition_tokens);
+    if (workspace_bytes < L.total)
+      return fail(PA_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", workspace_bytes, L.total);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.counters = reinterpret_cast<uint32_t*>(ws);
+    a.part_m = reinterpret_cast<float*>(ws + L.m_off);
+    a.part_l = reinterpret_cast<float*>(ws + L.l_off);
+    a.part_acc = reinterpret_cast<float*>(ws + L.acc_off);
+    a.partition_blocks = partition_tokens / r.block_size;
+    a.max_partitions = L.pmax;
+    a.persistent = 1;
+    smem += (r.num_seqs + 1) * 4;
+    st = prepare_kernel(inst.kernel, smem);
+    if (st != PA_OK) return st;
+    DeviceInfo dinfo;
+    st = device_info(&dinfo);
+    if (st != PA_OK) return st;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, inst.kernel, inst.threads, smem) != cudaSuccess ||
+        occ <= 0)
+      return fail(PA_ERR_CUDA, "occupancy query failed for %s (smem %d)", inst.name, smem);
+    const int64_t max_items = static_cast<int64_t>(r.num_seqs) * r.num_kv_heads * L.pmax;
+    const int64_t ctas = std::min<int64_t>(max_items, static_cast<int64_t>(dinfo.sms) * occ);
+    grid = dim3(static_cast<unsigned>(ctas > 0 ? ctas : 1));
+  } else {
+    a.partition_blocks = r.max_blocks_per_seq;
+    a.max_partitions = 1;
+    a.persistent = 0;
+    st = prepare_kernel(inst.kernel, smem);
+    if (st != PA_OK) return st;
+    grid = dim3(static_cast<unsigned>(r.num_seqs * r.num_kv_heads));
+  }
+
+  const int rows = r.num_blocks * r.num_kv_heads * r.block_size;
+  CUtensorMap tmk, tmv;
+  st = pool_tensor_map(r.k_pool, rows, r.head_dim, r.block_size, r.dtype, &tmk);
+  if (st != PA_OK) return st;
+  st = pool_tensor_map(r.v_pool, rows, r.head_dim, r.block_size, r.dtype, &tmv);
+  if (st != PA_OK) return st;
+
+  void* args[] = {&tmk, &tmv, &a};
+  cudaError_t err = cudaLaunchKernel(inst.kernel, grid, dim3(inst.threads), args, smem, r.stream);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+  if (split && a.max_partitions > 1) {
+    int bs = r.block_size;
+    void* margs[] = {&a, &bs};
+    const int warps = r.num_seqs * r.num_q_heads;
+    err = cudaLaunchKernel(inst.merge, dim3((warps + 3) / 4), dim3(128), margs, 0, r.stream);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(err));
+  }
+  return launch_error("decode");
+}
+
+}  // namespace
+}  // namespace pagedkv
+
+using namespace pagedkv;
+
+extern "C" {
+
+pa_status_t pa_decode(const void* q, const void* k_pool, const void* v_pool,
+                      const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                      void* out, uint32_t* dev_err, void* stream) {
+  DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+              head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
+              static_cast<cudaStream_t>(stream)};
+  return run_decode(r, false, 0, nullptr, 0);
+}
+
+size_t pa_decode_split_workspace_size(int num_seqs, int num_q_heads, int head_dim, int block_size,
+                                      int max_blocks_per_seq, int partition_tokens) {
+  if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_blocks_per_seq <= 0 || partition_tokens <= 0 || partition_tokens % block_size != 0)
+    return 0;
+  return split_layout(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
+                      partition_tokens)
+      .total;
+}
+
+pa_status_t pa_decode_split_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (workspace == nullptr || workspace_bytes < kWorkspaceHeader)
+    return fail(PA_ERR_INVALID_ARG, "workspace must hold at least %zu bytes", kWorkspaceHeader);
+  cudaError_t err =
+      cudaMemsetAsync(workspace, 0, kWorkspaceHeader, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "workspace init: %s", cudaGetErrorString(err));
+  return ok();
+}
+
+pa_status_t pa_decode_split(const void* q, const void* k_pool, const void* v_pool,
+                            const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                            int partition_tokens, void* workspace, size_t workspace_bytes,
+                            void* out, uint32_t* dev_err, void* stream) {
+  DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+              head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
+              static_cast<cudaStream_t>(stream)};
+  return run_decode(r, true, partition_tokens, workspace, workspace_bytes);
+}
+
+}  // extern "C"

@@ -1,0 +1,24 @@
+// Registry of compiled decode-kernel instances (filled by decode_inst_*.cu).
+#pragma once
+
+#include <cstdint>
+
+#include "pagedkv.h"
+
+namespace pagedkv {
+
+struct DecodeInstance {
+  const void* kernel = nullptr;  // paged_decode_kernel<Cfg>
+  const void* merge = nullptr;   // lse_merge_kernel<T, D>
+  int threads = 0;
+  int fixed_smem = 0;            // dynamic smem bytes before the prefix array
+  int stages = 0;
+  const char* name = "";
+};
+
+// Each returns false when (head_dim, block_size, group) has no instance.
+bool find_decode_f32(int head_dim, int block_size, int group, DecodeInstance* out);
+bool find_decode_bf16_simt(int head_dim, int block_size, int group, DecodeInstance* out);
+bool find_decode_bf16_mma(int head_dim, int block_size, DecodeInstance* out);
+
+}  // namespace pagedkv

@@ -1,0 +1,701 @@
+// Paged decode attention kernels for sm_100a (templates; instantiated in
+// decode_inst_*.cu).
+//
+// What is computed: for each sequence s and query head h,
+//   out[s][h] = softmax(scale * K_s q) V_s over the first ctx_s tokens of the
+// KV head that h reads, gathered in logical order through the sequence's
+// block table ("What is PagedAttention?", How It Works / Map Logical to
+// Physical Blocks). Blocks are visited in logical order and combined with a
+// running (online) max/sum, which reproduces the contiguous-layout result
+// ("PagedAttention: Optimizing KV Cache in vLLM", section 3).
+//
+// How (B200 design; the pages describe no kernel, so all of this is ours):
+// * Work item = (sequence, KV head, partition of PB blocks). A CTA of W warps
+//   takes an item; warp w walks the item's blocks w, w+W, w+2W, ... Each warp
+//   owns an NS-stage ring in shared memory fed by its lane 0 with 2-D TMA
+//   loads (cp.async.bulk.tensor) of the (block, head) K and V tiles, each
+//   completing on an mbarrier. Block ids are prefetched 32 at a time into
+//   lane registers, one chunk ahead, so the dependent table load is off the
+//   critical path.
+// * Tiles land in 128-byte-swizzled layout: each 128-byte column chunk of a
+//   tile is one TMA box of block_size rows; unit (16 B) u of row r sits at
+//   u ^ (r % 8). Row-wise reads and 8x8 ldmatrix reads are bank-conflict free.
+// * MHA (and fp32) path: CUDA cores. Each lane owns head_dim/32 dims; per-token
+//   partial dot products are folded across lanes by a transposing butterfly
+//   (block_size values in log2(32) shuffle stages), one exp2 per token, p
+//   broadcast by shuffles for the p*V accumulate.
+// * GQA path (bf16, group 2..16): tensor cores via mma.sync m16n8k16. The
+//   group's query rows (padded to 16) are the A operand held in registers;
+//   S = Q K^T comes from ldmatrix'ed K tiles, P stays in registers as the A
+//   operand of O += P V with V fragments from ldmatrix.trans.
+// * After an item, the warps' (m, l, acc) are merged through shared memory;
+//   a sequence that fits one partition is written to `out`, otherwise the
+//   partition's (m, l, acc) go to the workspace for the merge kernel.
+// * Persistent mode (split decode): grid = SMs x occupancy; CTAs pull item
+//   tickets from a device counter. Every CTA builds the per-sequence partition
+//   prefix sum in shared memory to map a ticket to (s, p, kvh). The last CTA to
+//   finish resets the counters to zero for the next call.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+#include <type_traits>
+
+#include "device_common.cuh"
+
+namespace pagedkv {
+
+struct DecodeArgs {
+  const void* q;
+  void* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* part_m;      // [B][Hq][PMAX], log2-domain running max (scaled logits)
+  float* part_l;      // [B][Hq][PMAX], running sum of 2^(logit - m)
+  float* part_acc;    // [B][Hq][PMAX][D], unnormalised accumulators
+  uint32_t* counters; // [0] ticket, [1] finished CTAs (persistent mode)
+  uint32_t* dev_err;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int num_blocks;
+  int max_blocks_per_seq;
+  int partition_blocks;  // PB
+  int max_partitions;    // PMAX = ceil(max_blocks_per_seq / PB)
+  float scale_log2;      // scale * log2(e)
+  int persistent;        // 1: ticket loop + partials; 0: item = blockIdx.x, whole context
+  int l2_hint;           // L2 policy of the KV stream: 0 normal, 1 evict-first, 2 evict-last
+};
+
+template <typename T, int BS, int D>
+struct TileGeom {
+  static constexpr int kElt = static_cast<int>(sizeof(T));
+  static constexpr int kRowBytes = D * kElt;
+  static constexpr int kChunks = kRowBytes / 128;  // TMA boxes per tile
+  static constexpr int kBoxCols = 128 / kElt;      // elements per box row
+  static constexpr int kChunkBytes = BS * 128;
+  static constexpr int kTileBytes = BS * kRowBytes;
+  static_assert(kRowBytes % 128 == 0, "head_dim * element size must be a multiple of 128 bytes");
+  static_assert(BS % 16 == 0, "block_size must be a multiple of 16");
+  // Byte offset of byte `b` of row `row` inside a swizzled tile.
+  __device__ __forceinline__ static uint32_t offset(int row, int b) {
+    const int chunk = b >> 7;
+    const int within = b & 127;
+    return static_cast<uint32_t>(chunk * kChunkBytes + row * 128 +
+                                 ((((within >> 4) ^ (row & 7)) << 4) | (within & 15)));
+  }
+};
+
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+
+// G_ > 0: CUDA-core path with compile-time group; G_ == 0: tensor-core path,
+// runtime group 1..16 (bf16 only).
+template <typename T, int BS_, int D_, int G_>
+struct DecodeCfg {
+  using Elt = T;
+  static constexpr int BS = BS_;
+  static constexpr int D = D_;
+  static constexpr int G = G_;
+  static constexpr bool kMma = (G_ == 0);
+  static constexpr int W = 4;
+  static constexpr int kThreads = 32 * W;
+  using Geo = TileGeom<T, BS, D>;
+  static constexpr int kStageBytes = 2 * Geo::kTileBytes;
+  static constexpr int NS = cmin(4, cmax(2, 98304 / (W * kStageBytes)));
+  static constexpr int kRingBytes = W * NS * kStageBytes;
+  static constexpr int kRowsMax = kMma ? 16 : G;
+  static constexpr int kMergeBytes = W * kRowsMax * (D + 2) * 4;
+  static constexpr int kMainBytes = cmax(kRingBytes, kMergeBytes);
+  static constexpr int kBarBytes = W * NS * 8;
+  static constexpr int kMiscInts = 8;
+  // Dynamic shared memory = 1024 (alignment slack) + main + barriers + misc
+  // + (num_seqs + 1) ints of partition prefix in persistent mode.
+  static constexpr int kFixedSmem = 1024 + kMainBytes + kBarBytes + kMiscInts * 4;
+  static_assert(!kMma || sizeof(T) == 2, "tensor-core path is bf16 only");
+  static_assert(kMma || D % 32 == 0, "CUDA-core path needs head_dim % 32 == 0");
+};
+
+// Transposing butterfly: on entry every lane holds N partial sums (one per
+// token); on exit v[0] holds the full 32-lane sum for token (N == 16 ?
+// lane >> 1 : lane). Each stage halves the values a lane keeps while pairing
+// lanes across one bit.
+template <int N>
+__device__ __forceinline__ void transpose_reduce(float (&v)[N], int lane) {
+  static_assert(N == 16 || N == 32, "block_size 16 or 32");
+#pragma unroll
+  for (int half = N / 2, mask = 16; half >= 1; half >>= 1, mask >>= 1) {
+    const bool upper = (lane & mask) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+    }
+  }
+  if constexpr (N == 16) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+// ---------------------------------------------------------------------------
+// Per-warp state and per-block math: CUDA-core path.
+template <class Cfg>
+struct SimtWarp {
+  using T = typename Cfg::Elt;
+  static constexpr int G = Cfg::G;
+  static constexpr int D = Cfg::D;
+  static constexpr int BS = Cfg::BS;
+  static constexpr int VEC = D / 32;
+  using Geo = typename Cfg::Geo;
+
+  float qf[G][VEC];
+  float m[G];
+  float l[G];
+  float acc[G][VEC];
+
+  __device__ __forceinline__ void begin(const T* q_group, float scale_log2, int lane) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      load_vec_f32<T, VEC>(q_group + h * D + lane * VEC, qf[h]);
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) {
+        qf[h][j] *= scale_log2;
+        acc[h][j] = 0.f;
+      }
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+    }
+  }
+
+  __device__ __forceinline__ void block(const uint8_t* kt, uint8_t* vt, int nvalid, int lane) {
+    const int byte_off = lane * VEC * Geo::kElt;
+    const int my_token = (BS == 16) ? (lane >> 1) : lane;
+    const bool counts = (BS == 32) || ((lane & 1) == 0);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float v[BS];
+#pragma unroll
+      for (int t = 0; t < BS; ++t) {
+        float kf[VEC];
+        load_vec_f32<T, VEC>(reinterpret_cast<const T*>(kt + Geo::offset(t, byte_off)), kf);
+        float d = 0.f;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) d = fmaf(qf[h][j], kf[j], d);
+        v[t] = d;
+      }
+      transpose_reduce<BS>(v, lane);
+      const float s = (my_token < nvalid) ? v[0] : -INFINITY;
+      const float m_new = fmaxf(m[h], warp_max(s));
+      const float alpha = fast_exp2(m[h] - m_new);
+      const float p = fast_exp2(s - m_new);
+      l[h] = l[h] * alpha + (counts ? p : 0.f);
+      m[h] = m_new;
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) acc[h][j] *= alpha;
+#pragma unroll
+      for (int t = 0; t < BS; ++t) {
+        if (t < nvalid) {  // warp-uniform; rows past the context may hold anything
+          const float pt = __shfl_sync(0xffffffffu, p, (BS == 16) ? 2 * t : t);
+          float vf[VEC];
+          load_vec_f32<T, VEC>(reinterpret_cast<const T*>(vt + Geo::offset(t, byte_off)), vf);
+#pragma unroll
+          for (int j = 0; j < VEC; ++j) acc[h][j] = fmaf(pt, vf[j], acc[h][j]);
+        }
+      }
+    }
+  }
+
+  // Writes this warp's state (rows 0..G-1) into the merge area.
+  __device__ __forceinline__ void publish(float* sm_m, float* sm_l, float* sm_acc, int lane) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float lt = warp_sum(l[h]);
+      if (lane == 0) {
+        sm_m[h] = m[h];
+        sm_l[h] = lt;
+      }
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) sm_acc[h * D + lane * VEC + j] = acc[h][j];
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Per-warp state and per-block math: tensor-core path (bf16, group <= 16).
+template <class Cfg>
+struct MmaWarp {
+  static constexpr int D = Cfg::D;
+  static constexpr int BS = Cfg::BS;
+  static constexpr int KS = D / 16;   // k-steps of S = Q K^T
+  static constexpr int NT = BS / 8;   // 8-token n-tiles of S
+  static constexpr int ND = D / 8;    // 8-dim n-tiles of O
+  using Geo = typename Cfg::Geo;
+
+  uint32_t qa[KS][4];
+  float o[ND][4];
+  float m[2];
+  float l[2];
+  float scale_log2;
+
+  __device__ __forceinline__ void begin(const __nv_bfloat16* q_group, int group, float scale,
+                                        int lane) {
+    const int g = lane >> 2;
+    const int t4 = lane & 3;
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(q_group);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int c0 = ks * 16 + 2 * t4;
+      qa[ks][0] = (g < group) ? q32[(g * D + c0) >> 1] : 0u;
+      qa[ks][1] = (g + 8 < group) ? q32[((g + 8) * D + c0) >> 1] : 0u;
+      qa[ks][2] = (g < group) ? q32[(g * D + c0 + 8) >> 1] : 0u;
+      qa[ks][3] = (g + 8 < group) ? q32[((g + 8) * D + c0 + 8) >> 1] : 0u;
+    }
+#pragma unroll
+    for (int n = 0; n < ND; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+    scale_log2 = scale;
+  }
+
+  __device__ __forceinline__ void block(const uint8_t* kt, uint8_t* vt, int nvalid, int lane) {
+    const int t4 = lane & 3;
+    const int mj = lane >> 3;  // which 8x8 matrix this lane addresses
+    const int mr = lane & 7;   // which row of it
+    const uint32_t kbase = smem_addr(kt);
+    const uint32_t vbase = smem_addr(vt);
+
+    float s[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+      for (int sub = 0; sub < BS / 16; ++sub) {
+        const int tok = sub * 16 + (mj >> 1) * 8 + mr;
+        const int dim = ks * 16 + (mj & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(kbase + Geo::offset(tok, dim * 2), b0, b1, b2, b3);
+        mma_bf16_16816(s[2 * sub], qa[ks], b0, b1);
+        mma_bf16_16816(s[2 * sub + 1], qa[ks], b2, b3);
+      }
+    }
+    // Scale, mask tokens past the context, online softmax per query row.
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = n * 8 + 2 * t4 + (e & 1);
+        s[n][e] = (tok < nvalid) ? s[n][e] * scale_log2 : -INFINITY;
+      }
+      mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][1]));
+      mx1 = fmaxf(mx1, fmaxf(s[n][2], s[n][3]));
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mn0 = fmaxf(m[0], mx0);
+    const float mn1 = fmaxf(m[1], mx1);
+    const float a0 = fast_exp2(m[0] - mn0);
+    const float a1 = fast_exp2(m[1] - mn1);
+    m[0] = mn0;
+    m[1] = mn1;
+    float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      s[n][0] = fast_exp2(s[n][0] - mn0);
+      s[n][1] = fast_exp2(s[n][1] - mn0);
+      s[n][2] = fast_exp2(s[n][2] - mn1);
+      s[n][3] = fast_exp2(s[n][3] - mn1);
+      r0 += s[n][0] + s[n][1];
+      r1 += s[n][2] + s[n][3];
+    }
+    l[0] = l[0] * a0 + r0;
+    l[1] = l[1] * a1 + r1;
+#pragma unroll
+    for (int n = 0; n < ND; ++n) {
+      o[n][0] *= a0;
+      o[n][1] *= a0;
+      o[n][2] *= a1;
+      o[n][3] *= a1;
+    }
+    // Rows of V past the context may hold anything (even NaN bit patterns);
+    // p is 0 there but 0 * NaN is NaN, so clear them in shared memory.
+    if (nvalid < BS) {
+      constexpr int kUnitsPerRow = Geo::kRowBytes / 16;
+      const int units = (BS - nvalid) * kUnitsPerRow;
+      for (int u = lane; u < units; u += 32) {
+        const int row = nvalid + u / kUnitsPerRow;
+        const int b = (u % kUnitsPerRow) * 16;
+        *reinterpret_cast<uint4*>(vt + Geo::offset(row, b)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();  // the stage is refilled by TMA later
+      __syncwarp();
+    }
+#pragma unroll
+    for (int kk = 0; kk < BS / 16; ++kk) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
+      pa[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
+      pa[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pa[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+      for (int nd = 0; nd < D / 16; ++nd) {
+        const int tok = kk * 16 + (mj & 1) * 8 + mr;
+        const int dim = nd * 16 + (mj >> 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(vbase + Geo::offset(tok, dim * 2), b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * nd], pa, b0, b1);
+        mma_bf16_16816(o[2 * nd + 1], pa, b2, b3);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void publish(float* sm_m, float* sm_l, float* sm_acc, int group,
+                                          int lane) {
+    const int g = lane >> 2;
+    const int t4 = lane & 3;
+    float l0 = l[0], l1 = l[1];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (g < group) {
+      if (t4 == 0) {
+        sm_m[g] = m[0];
+        sm_l[g] = l0;
+      }
+#pragma unroll
+      for (int n = 0; n < ND; ++n) {
+        sm_acc[g * D + n * 8 + 2 * t4] = o[n][0];
+        sm_acc[g * D + n * 8 + 2 * t4 + 1] = o[n][1];
+      }
+    }
+    if (g + 8 < group) {
+      if (t4 == 0) {
+        sm_m[g + 8] = m[1];
+        sm_l[g + 8] = l1;
+      }
+#pragma unroll
+      for (int n = 0; n < ND; ++n) {
+        sm_acc[(g + 8) * D + n * 8 + 2 * t4] = o[n][2];
+        sm_acc[(g + 8) * D + n * 8 + 2 * t4 + 1] = o[n][3];
+      }
+    }
+  }
+};
+
+// Number of partitions of a sequence with context length ctx (at least one, so
+// that an empty sequence still gets its zero output written).
+__device__ __forceinline__ int partitions_of(int ctx, int bs, int pb) {
+  const int nb = (ctx + bs - 1) / bs;
+  const int p = (nb + pb - 1) / pb;
+  return p > 1 ? p : 1;
+}
+
+__device__ __forceinline__ int clamp_ctx(int raw, int max_tokens) {
+  return (raw < 0 || raw > max_tokens) ? 0 : raw;
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::kThreads)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
+  using T = typename Cfg::Elt;
+  using Geo = typename Cfg::Geo;
+  constexpr int W = Cfg::W;
+  constexpr int NS = Cfg::NS;
+  constexpr int BS = Cfg::BS;
+  constexpr int D = Cfg::D;
+  constexpr int NT = Cfg::kThreads;
+  using WarpT = typename std::conditional<Cfg::kMma, MmaWarp<Cfg>, SimtWarp<Cfg>>::type;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* ring = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kMainBytes);
+  int* misc = reinterpret_cast<int*>(smem + Cfg::kMainBytes + Cfg::kBarBytes);
+  int* prefix = misc + Cfg::kMiscInts;  // [num_seqs + 1], persistent mode only
+  float* sm_m = reinterpret_cast<float*>(smem);                // [W][rows]
+  float* sm_l = sm_m + W * Cfg::kRowsMax;                      // [W][rows]
+  float* sm_acc = sm_l + W * Cfg::kRowsMax;                    // [W][rows][D]
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int B = a.num_seqs;
+  const int Hkv = a.num_kv_heads;
+  const int G = a.group;
+  const int max_tokens = a.max_blocks_per_seq * BS;
+
+  if (tid == 0) {
+    for (int i = 0; i < W * NS; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+    tma_prefetch_descriptor(&tm_k);
+    tma_prefetch_descriptor(&tm_v);
+    misc[0] = 0;  // timeout flag
+  }
+
+  int total_items;
+  if (a.persistent) {
+    // prefix[i] = number of partitions of sequences 0..i-1 (exclusive scan).
+    __shared__ int warp_tot[W];
+    const int chunk = (B + NT - 1) / NT;
+    const int lo = min(B, tid * chunk);
+    const int hi = min(B, lo + chunk);
+    int mine = 0;
+    for (int i = lo; i < hi; ++i)
+      mine += partitions_of(clamp_ctx(a.context_lens[i], max_tokens), BS, a.partition_blocks);
+    int incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_tot[w];
+    int run = base + incl - mine;
+    for (int i = lo; i < hi; ++i) {
+      prefix[i] = run;
+      run += partitions_of(clamp_ctx(a.context_lens[i], max_tokens), BS, a.partition_blocks);
+    }
+    if (tid == NT - 1) prefix[B] = base + incl;
+    __syncthreads();
+    total_items = prefix[B] * Hkv;
+  } else {
+    total_items = B * Hkv;
+  }
+  __syncthreads();
+
+  const uint64_t policy = l2_policy(a.l2_hint);
+  uint32_t gcount = 0;  // blocks this warp has consumed so far (ring position)
+
+  int item;
+  if (a.persistent) {
+    if (tid == 0) misc[2] = static_cast<int>(atomicAdd(&a.counters[0], 1u));
+    __syncthreads();
+    item = misc[2];
+  } else {
+    item = blockIdx.x;
+  }
+  int iter = 0;
+
+  while (item < total_items) {
+    // Ask for the next ticket now; the atomic's latency overlaps this item.
+    if (a.persistent && tid == 0)
+      misc[3 + (iter & 1)] = static_cast<int>(atomicAdd(&a.counters[0], 1u));
+
+    // ---- decode the item ----------------------------------------------------
+    int s, p, kvh, nparts;
+    if (a.persistent) {
+      const int pi = item / Hkv;
+      kvh = item - pi * Hkv;
+      int lo = 0, hi = B - 1;  // last s with prefix[s] <= pi
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= pi) lo = mid; else hi = mid - 1;
+      }
+      s = lo;
+      p = pi - prefix[s];
+      nparts = prefix[s + 1] - prefix[s];
+    } else {
+      s = item / Hkv;
+      kvh = item - s * Hkv;
+      p = 0;
+      nparts = 1;
+    }
+    const int ctx_raw = a.context_lens[s];
+    const int ctx = clamp_ctx(ctx_raw, max_tokens);
+    if (ctx != ctx_raw && p == 0 && kvh == 0 && tid == 0) report(a.dev_err, PA_DEVERR_CONTEXT_LEN);
+    const int nb = (ctx + BS - 1) / BS;
+    const int b_begin = a.persistent ? p * a.partition_blocks : 0;
+    const int b_end = a.persistent ? min(nb, b_begin + a.partition_blocks) : nb;
+    const int nblk = max(0, b_end - b_begin);
+    const int nj = (nblk > warp) ? (nblk - warp + W - 1) / W : 0;
+
+    // ---- per-warp pipeline over blocks b_begin + warp + j*W ----------------------
+    const T* q_group = reinterpret_cast<const T*>(a.q) +
+                       (static_cast<int64_t>(s) * a.num_q_heads + static_cast<int64_t>(kvh) * G) * D;
+    WarpT st;
+    if constexpr (Cfg::kMma) {
+      st.begin(q_group, G, a.scale_log2, lane);
+    } else {
+      st.begin(q_group, a.scale_log2, lane);
+    }
+
+    const int32_t* bt = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq + b_begin + warp;
+    int bt_cur = (lane < nj) ? bt[lane * W] : -1;
+    int bt_nxt = (32 + lane < nj) ? bt[(32 + lane) * W] : -1;
+    int bt_chunk = 0;
+    uint32_t bad = 0;  // bit per stage: the stage's block id was out of range
+    uint8_t* my_ring = ring + warp * NS * Cfg::kStageBytes;
+    uint64_t* my_bars = bars + warp * NS;
+
+    auto issue = [&](int j) {
+      const int c = j >> 5;
+      if (c != bt_chunk) {  // advance the block-id window by one chunk
+        bt_cur = bt_nxt;
+        bt_nxt = ((c + 1) * 32 + lane < nj) ? bt[((c + 1) * 32 + lane) * W] : -1;
+        bt_chunk = c;
+      }
+      const int phys = __shfl_sync(0xffffffffu, bt_cur, j & 31);
+      const uint32_t stage = (gcount + j) % NS;
+      const bool good = phys >= 0 && phys < a.num_blocks;
+      bad = good ? (bad & ~(1u << stage)) : (bad | (1u << stage));
+      if (lane == 0) {
+        uint64_t* bar = &my_bars[stage];
+        fence_proxy_async_smem();
+        if (good) {
+          uint8_t* kdst = my_ring + stage * Cfg::kStageBytes;
+          uint8_t* vdst = kdst + Geo::kTileBytes;
+          const int32_t y = (phys * Hkv + kvh) * BS;
+          mbar_arrive_expect_tx(bar, 2 * Geo::kTileBytes);
+#pragma unroll
+          for (int c2 = 0; c2 < Geo::kChunks; ++c2) {
+            tma_load_2d(kdst + c2 * Geo::kChunkBytes, &tm_k, bar, c2 * Geo::kBoxCols, y, policy);
+            tma_load_2d(vdst + c2 * Geo::kChunkBytes, &tm_v, bar, c2 * Geo::kBoxCols, y, policy);
+          }
+        } else {
+          report(a.dev_err, PA_DEVERR_BLOCK_ID);
+          mbar_arrive(bar);  // completes the phase with no data
+        }
+      }
+    };
+
+    const int npre = min(NS, nj);
+    for (int j = 0; j < npre; ++j) issue(j);
+    bool timed_out = false;
+    int j = 0;
+    for (; j < nj; ++j) {
+      const uint32_t g = gcount + j;
+      const uint32_t stage = g % NS;
+      const uint32_t parity = (g / NS) & 1u;
+      const bool okw = mbar_wait_bounded(&my_bars[stage], parity, a.dev_err);
+      if (!__all_sync(0xffffffffu, okw)) {
+        timed_out = true;
+        break;
+      }
+      if (!(bad & (1u << stage))) {
+        const int lb = b_begin + warp + j * W;  // logical block
+        const int nvalid = min(BS, ctx - lb * BS);
+        uint8_t* kt = my_ring + stage * Cfg::kStageBytes;
+        st.block(kt, kt + Geo::kTileBytes, nvalid, lane);
+      }
+      __syncwarp();
+      if (j + NS < nj) issue(j + NS);
+    }
+    if (timed_out) {
+      // Give copies still in flight a bounded chance to land before leaving.
+      for (int jj = j; jj < min(nj, j + NS); ++jj) {
+        const uint32_t g = gcount + jj;
+        mbar_wait_bounded(&my_bars[g % NS], (g / NS) & 1u, a.dev_err);
+      }
+      if (lane == 0) misc[0] = 1;
+    }
+    gcount += nj;
+
+    // ---- merge the W warps' partial states ------------------------------------------
+    __syncthreads();  // every warp is done with the ring; it becomes the merge area
+    if constexpr (Cfg::kMma) {
+      st.publish(sm_m + warp * Cfg::kRowsMax, sm_l + warp * Cfg::kRowsMax,
+                 sm_acc + warp * Cfg::kRowsMax * D, G, lane);
+    } else {
+      st.publish(sm_m + warp * Cfg::kRowsMax, sm_l + warp * Cfg::kRowsMax,
+                 sm_acc + warp * Cfg::kRowsMax * D, lane);
+    }
+    __syncthreads();
+    const bool final_out = (nparts == 1);
+    for (int idx = tid; idx < G * D; idx += NT) {
+      const int h = idx / D;
+      const int d = idx - h * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < W; ++w) M = fmaxf(M, sm_m[w * Cfg::kRowsMax + h]);
+      float L = 0.f, A = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          const float e = fast_exp2(sm_m[w * Cfg::kRowsMax + h] - M);
+          L = fmaf(sm_l[w * Cfg::kRowsMax + h], e, L);
+          A = fmaf(sm_acc[(w * Cfg::kRowsMax + h) * D + d], e, A);
+        }
+      }
+      const int64_t row = static_cast<int64_t>(s) * a.num_q_heads + kvh * G + h;
+      if (final_out) {
+        reinterpret_cast<T*>(a.out)[row * D + d] = Elt<T>::from_f32(L > 0.f ? A / L : 0.f);
+      } else {
+        const int64_t pr = row * a.max_partitions + p;
+        a.part_acc[pr * D + d] = A;
+        if (d == 0) {
+          a.part_m[pr] = M;
+          a.part_l[pr] = L;
+        }
+      }
+    }
+    fence_proxy_async_smem();  // generic accesses to the ring precede the next TMA writes
+    __syncthreads();  // merge area reads done before the ring is refilled
+    if (misc[0]) break;
+
+    if (a.persistent) {
+      item = misc[3 + (iter & 1)];
+    } else {
+      item = total_items;
+    }
+    ++iter;
+  }
+
+  if (a.persistent && tid == 0) {
+    // The last CTA to get here resets the counters for the next call; every
+    // other CTA has already taken its final ticket.
+    __threadfence();
+    const uint32_t prev = atomicAdd(&a.counters[1], 1u);
+    if (prev == gridDim.x - 1) {
+      atomicExch(&a.counters[0], 0u);
+      atomicExch(&a.counters[1], 0u);
+      __threadfence();
+    }
+  }
+}
+
+// Log-sum-exp merge of partition partials: one warp per (sequence, query head)
+// with more than one partition; single-partition sequences were written by
+// the decode kernel. out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.
+template <typename T, int D>
+__global__ void __launch_bounds__(128)
+    lse_merge_kernel(const DecodeArgs a, int block_size) {
+  constexpr int VEC = D / 32;
+  const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= a.num_seqs * a.num_q_heads) return;
+  const int s = wid / a.num_q_heads;
+  const int ctx = clamp_ctx(a.context_lens[s], a.max_blocks_per_seq * block_size);
+  const int np = partitions_of(ctx, block_size, a.partition_blocks);
+  if (np <= 1) return;
+  const int64_t base = static_cast<int64_t>(wid) * a.max_partitions;
+  float M = -INFINITY;
+  for (int p = lane; p < np; p += 32) M = fmaxf(M, a.part_m[base + p]);
+  M = warp_max(M);
+  float L = 0.f;
+  for (int p = lane; p < np; p += 32) L += a.part_l[base + p] * fast_exp2(a.part_m[base + p] - M);
+  L = warp_sum(L);
+  float acc[VEC];
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
+  for (int p = 0; p < np; ++p) {
+    const float e = fast_exp2(a.part_m[base + p] - M);
+    const float* src = a.part_acc + (base + p) * D + lane * VEC;
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) acc[j] = fmaf(src[j], e, acc[j]);
+  }
+  T* dst = reinterpret_cast<T*>(a.out) + static_cast<int64_t>(wid) * D + lane * VEC;
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) dst[j] = Elt<T>::from_f32(acc[j] * inv);
+}
+
+}  // namespace pagedkv

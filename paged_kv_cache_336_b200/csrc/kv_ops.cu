@@ -1,0 +1,143 @@
+// KV-append scatter and whole-block copy (copy-on-write data movement), with
+// their C-ABI entry points (see include/pagedkv.h).
+//
+// * Append: decode writes each new token's K and V into its slot in the partly
+//   filled tail block ("What is PagedAttention?", How It Works / Map Logical
+//   to Physical Blocks; "PagedAttention: Optimizing KV Cache in vLLM",
+//   section 4, step 3: the write proceeds on the private block).
+// * Copy: the private block receives the shared block's contents (same
+//   section, step 3); the whole block is copied.
+//
+// Both are pure HBM copies moved as 16-byte vectors; every index is checked
+// on the device and an out-of-range one is reported and skipped.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "device_common.cuh"
+#include "pa_internal.h"
+
+namespace pagedkv {
+namespace {
+
+// One thread per 16-byte unit of (token, kv head, row unit); K and V together.
+__global__ void __launch_bounds__(256)
+    kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                     const int64_t* __restrict__ slots, int num_tokens, int num_kv_heads,
+                     int units_per_row, int block_size, int64_t num_slots, uint4* k_pool,
+                     uint4* v_pool, uint32_t* dev_err) {
+  const int64_t per_token = static_cast<int64_t>(num_kv_heads) * units_per_row;
+  const int64_t total = per_token * num_tokens;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_token;
+    const int64_t rem = i - t * per_token;
+    const int64_t h = rem / units_per_row;
+    const int64_t u = rem - h * units_per_row;
+    const int64_t slot = slots[t];
+    if (slot < 0) continue;  // padding
+    if (slot >= num_slots) {
+      if (rem == 0) report(dev_err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t blk = slot / block_size;
+    const int64_t off = slot - blk * block_size;
+    const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * units_per_row + u;
+    k_pool[dst] = k_new[i];
+    v_pool[dst] = v_new[i];
+  }
+}
+
+// grid.y walks pairs, grid.x x blockDim.x walks the 16-byte units of a block.
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* k_pool, uint4* v_pool, const int64_t* __restrict__ pairs,
+                       int num_pairs, int64_t units_per_block, int num_blocks,
+                       uint32_t* dev_err) {
+  for (int pr = blockIdx.y; pr < num_pairs; pr += gridDim.y) {
+    const int64_t src = pairs[2 * static_cast<int64_t>(pr)];
+    const int64_t dst = pairs[2 * static_cast<int64_t>(pr) + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) report(dev_err, PA_DEVERR_COPY_PAIR);
+      continue;
+    }
+    if (src == dst) continue;
+    const uint4* ks = k_pool + src * units_per_block;
+    const uint4* vs = v_pool + src * units_per_block;
+    uint4* kd = k_pool + dst * units_per_block;
+    uint4* vd = v_pool + dst * units_per_block;
+    for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units_per_block;
+         u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      kd[u] = ks[u];
+      vd[u] = vs[u];
+    }
+  }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+}  // namespace
+}  // namespace pagedkv
+
+using namespace pagedkv;
+
+extern "C" {
+
+pa_status_t pa_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                         int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype_t dtype, void* k_pool, void* v_pool,
+                         uint32_t* dev_err, void* stream) {
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens < 0");
+  if (num_tokens == 0) return ok();
+  if (k_new == nullptr || v_new == nullptr || slot_mapping == nullptr || k_pool == nullptr ||
+      v_pool == nullptr)
+    return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+  if (dtype != PA_F32 && dtype != PA_BF16) return fail(PA_ERR_INVALID_ARG, "unknown dtype");
+  if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "sizes must be positive");
+  const int eb = dtype == PA_F32 ? 4 : 2;
+  if ((head_dim * eb) % 16 != 0) return fail(PA_ERR_INVALID_ARG, "head_dim * element size must be a multiple of 16");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool))
+    return fail(PA_ERR_INVALID_ARG, "k_new, v_new and pools must be 16-byte aligned");
+  const int upr = head_dim * eb / 16;
+  const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * upr;
+  const int64_t want = (total + 255) / 256;
+  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sm_count()) * 8));
+  kv_append_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping, num_tokens,
+      num_kv_heads, upr, block_size, static_cast<int64_t>(num_blocks) * block_size,
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), dev_err);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "kv_append launch: %s", cudaGetErrorString(err));
+  return ok();
+}
+
+pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pairs, int num_pairs,
+                           size_t block_bytes, int num_blocks, uint32_t* dev_err, void* stream) {
+  if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs < 0");
+  if (num_pairs == 0) return ok();
+  if (k_pool == nullptr || v_pool == nullptr || src_dst_pairs == nullptr)
+    return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+  if (block_bytes == 0 || block_bytes % 16 != 0)
+    return fail(PA_ERR_INVALID_ARG, "block_bytes must be a positive multiple of 16");
+  if (num_blocks <= 0) return fail(PA_ERR_INVALID_ARG, "num_blocks must be positive");
+  if (!aligned16(k_pool) || !aligned16(v_pool)) return fail(PA_ERR_INVALID_ARG, "pools must be 16-byte aligned");
+  const int64_t upb = static_cast<int64_t>(block_bytes / 16);
+  const int gx = static_cast<int>(std::min<int64_t>((upb + 1023) / 1024, 64));
+  const int gy = std::min(num_pairs, 65535);
+  copy_blocks_kernel<<<dim3(gx, gy), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), src_dst_pairs, num_pairs, upb,
+      num_blocks, dev_err);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "copy_blocks launch: %s", cudaGetErrorString(err));
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,239 @@
+"""CPU tests of the C ABI (no GPU needed).
+
+* The shared library loads and exports every function declared in
+  include/pagedkv.h.
+* The C++ block manager matches the Python reference manager bit for bit:
+  the hand-worked golden trace, seeded random operation sequences (slots,
+  copy pairs, tables, counts, free-queue order, statistics, failures), and
+  the block tables of every synthetic workload.
+* Kernel entry points reject bad arguments before touching the device.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.block_manager import BlockManager as RefBM, InvalidArgument, NoFreeBlocks
+from paged_kv_cache_336_b200 import binding, workloads
+from paged_kv_cache_336_b200.binding import (
+    BlockManager as LibBM, InvalidArgumentError, NoFreeBlocksError, PagedKVError)
+
+from test_oracle_block_manager import TraceRunner, random_ops, apply_op, _check_invariants
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "pagedkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    lib = binding.library()
+    names = declared_functions()
+    assert len(names) >= 20
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in binding._SIGNATURES, f"{name} has no binding signature"
+    assert lib.pa_version().decode().startswith("pagedkv")
+    assert lib.pa_status_string(2).decode() == "PA_ERR_NO_FREE_BLOCKS"
+
+
+def test_library_is_built_for_sm100a_only():
+    # the fatbin inside the library is produced by `-gencode arch=compute_100a,code=sm_100a`;
+    # the build script is the single place that sets it
+    from paged_kv_cache_336_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+class _LibAdapter:
+    """Maps the library manager onto the oracle's exception types for the trace."""
+
+    def __init__(self, *args):
+        self.bm = LibBM(*args)
+
+    def __getattr__(self, name):
+        fn = getattr(self.bm, name)
+
+        def call(*a, **k):
+            try:
+                return fn(*a, **k)
+            except NoFreeBlocksError as e:
+                raise NoFreeBlocks(str(e))
+            except InvalidArgumentError as e:
+                raise InvalidArgument(str(e))
+        return call
+
+
+def test_golden_trace_library():
+    runner = TraceRunner(lambda nb, bs, mbs, order: _LibAdapter(nb, bs, mbs, order))
+    assert runner.run() > 40
+
+
+def _lib_state(bm: LibBM, seqs):
+    tables = tuple(sorted((s, tuple(bm.block_table(s))) for s in seqs))
+    ctx = tuple(sorted((s, bm.context_len(s)) for s in seqs))
+    rc = tuple(bm.refcount_of(b) for b in range(bm.num_blocks))
+    return (tuple(bm.free_queue_list()), rc, tables, ctx, bm.stats()["cow_copies"])
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_ops_match_reference(seed):
+    (nb, bs, mbs, order), ops = random_ops(seed, n_ops=300)
+    ref = RefBM(nb, bs, mbs, order)
+    lib = _LibAdapter(nb, bs, mbs, order)
+    for op in ops:
+        r_ref = apply_op(ref, op)
+        r_lib = apply_op(lib, op)
+        assert r_ref == r_lib, op
+        assert _lib_state(lib.bm, list(ref.tables)) == ref.snapshot(), op
+        st = lib.bm.stats()
+        want = ref.stats()
+        for k, v in want.items():
+            assert st[k] == v, (k, op)
+    _check_invariants(ref)
+
+
+def test_can_append_agrees_with_append():
+    bm = LibBM(6, 4, 3, list(range(6)))
+    bm.allocate(10, 5)
+    bm.fork(10, 11)
+    bm.fork(10, 12)
+    bm.allocate(13, 12)
+    assert not bm.can_append([10, 11, 12])
+    with pytest.raises(NoFreeBlocksError):
+        bm.append_slots([10, 11, 12])
+    assert bm.can_append([12])
+    bm.free(13)
+    assert bm.can_append([10, 11, 12])
+    slots, pairs = bm.append_slots_arrays([10, 11, 12])
+    assert slots.tolist() == [21, 9, 5]
+    assert pairs.tolist() == [[1, 5], [1, 2]]
+
+
+def build_tables(bm, w):
+    """Applies a workload's prefill/fork/extra-token plan to a manager."""
+    for s in w.prefill_seqs:
+        bm.allocate(s, int(w.context_lens[s]))
+    for parent, child in w.forks:
+        bm.fork(parent, child)
+    for s, n in sorted(w.extra_tokens.items()):
+        for _ in range(n):
+            bm.append_slot(s)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mha", "gqa", "prefix", "prefix_cow"])
+def test_workload_tables_match_reference(name):
+    w = workloads.WORKLOADS[name]()
+    ref = RefBM(w.num_blocks, w.block_size, w.max_blocks_per_seq, w.free_order)
+    lib = LibBM(w.num_blocks, w.block_size, w.max_blocks_per_seq, w.free_order)
+    build_tables(ref, w)
+    build_tables(lib, w)
+    seqs = sorted(ref.tables)
+    tables, ctx = lib.export(seqs)
+    for i, s in enumerate(seqs):
+        t = ref.block_table(s)
+        assert tables[i, :len(t)].tolist() == t
+        assert (tables[i, len(t):] == -1).all()
+        assert ctx[i] == ref.context_len(s)
+    if w.step_seqs:
+        r1 = ref.append_slots(w.step_seqs)
+        slots, pairs = lib.append_slots_arrays(w.step_seqs)
+        assert slots.tolist() == [r.slot for r in r1]
+        want_pairs = [[r.cow_src, r.cow_dst] for r in r1 if r.cow_src >= 0]
+        assert pairs.tolist() == want_pairs
+        if name == "prefix_cow":
+            assert len(want_pairs) == 8 * 15   # every branch but the last copies
+        if name == "tiny":
+            assert len(want_pairs) == 1        # sequence 3's shared tail is copied
+
+
+def test_long_workload_tables_match_reference():
+    w = workloads.long(block_size=32)
+    ref = RefBM(w.num_blocks, w.block_size, w.max_blocks_per_seq, w.free_order)
+    lib = LibBM(w.num_blocks, w.block_size, w.max_blocks_per_seq, w.free_order)
+    build_tables(ref, w)
+    build_tables(lib, w)
+    tables, ctx = lib.export(list(range(8)))
+    for s in range(8):
+        assert tables[s, :4096].tolist() == ref.block_table(s)
+    assert ref.num_free() == 0 and lib.num_free() == 0
+
+
+FAKE = 0x7000_0000  # aligned host address never dereferenced: validation fails first
+
+
+def _decode_args(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, bt=FAKE, ctx=FAKE, B=4, Hq=8, Hkv=2, D=128, BS=16, NB=64,
+             MBS=8, scale=0.1, dtype=binding.PA_BF16, out=FAKE, err=None, stream=None)
+    a.update(over)
+    return a
+
+
+def _call_decode(a):
+    lib = binding.library()
+    return lib.pa_decode(a["q"], a["k"], a["v"], a["bt"], a["ctx"], a["B"], a["Hq"], a["Hkv"],
+                         a["D"], a["BS"], a["NB"], a["MBS"], a["scale"], a["dtype"], a["out"],
+                         a["err"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=None), binding.PA_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), binding.PA_ERR_INVALID_ARG),
+    (dict(dtype=7), binding.PA_ERR_INVALID_ARG),
+    (dict(k=FAKE + 8), binding.PA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.PA_ERR_INVALID_ARG),
+    (dict(NB=1 << 30), binding.PA_ERR_INVALID_ARG),
+    (dict(D=96), binding.PA_ERR_UNSUPPORTED),
+    (dict(BS=8), binding.PA_ERR_UNSUPPORTED),
+    (dict(Hq=64, Hkv=2), binding.PA_ERR_UNSUPPORTED),
+    (dict(dtype=binding.PA_F32, Hq=6, Hkv=2), binding.PA_ERR_UNSUPPORTED),
+    (dict(dtype=binding.PA_F32, D=256, Hq=2), binding.PA_ERR_UNSUPPORTED),
+])
+def test_decode_rejects_bad_arguments(over, status):
+    assert _call_decode(_decode_args(**over)) == status
+    assert binding.library().pa_last_error_string() != b""
+
+
+def test_split_workspace_size():
+    lib = binding.library()
+    n = lib.pa_decode_split_workspace_size(8, 64, 128, 16, 8193, 512)
+    pmax = -(-8193 // 32)
+    rows = 8 * 64 * pmax
+    assert n >= 256 + rows * 4 * 2 + rows * 128 * 4
+    assert n % 256 == 0
+    assert lib.pa_decode_split_workspace_size(8, 64, 128, 16, 100, 500) == 0  # not a multiple
+
+
+def test_append_and_copy_reject_bad_arguments():
+    lib = binding.library()
+    assert lib.pa_kv_append(FAKE, FAKE, FAKE, 4, 2, 128, 16, 8, 9, FAKE, FAKE, None, None) == \
+        binding.PA_ERR_INVALID_ARG
+    assert lib.pa_kv_append(FAKE, FAKE, None, 4, 2, 128, 16, 8, binding.PA_BF16, FAKE, FAKE, None,
+                            None) == binding.PA_ERR_INVALID_ARG
+    assert lib.pa_kv_append(FAKE, FAKE, FAKE, 0, 2, 128, 16, 8, binding.PA_BF16, FAKE, FAKE, None,
+                            None) == binding.PA_OK  # nothing to do
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 3, 100, 8, None, None) == binding.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 0, 4096, 8, None, None) == binding.PA_OK
+
+
+def test_block_manager_rejects_bad_arguments():
+    with pytest.raises(InvalidArgumentError):
+        LibBM(3, 4, 2, [0, 0, 1])
+    bm = LibBM(4, 4, 2)
+    with pytest.raises(InvalidArgumentError):
+        bm.allocate(0, 9)
+    bm.allocate(0, 8)
+    with pytest.raises(InvalidArgumentError):
+        bm.append_slot(0)
+    with pytest.raises(InvalidArgumentError):
+        bm.fork(5, 6)
+    with pytest.raises(InvalidArgumentError):
+        bm.append_slots([0, 0])
+    with pytest.raises(PagedKVError):
+        bm.refcount_of(99)
