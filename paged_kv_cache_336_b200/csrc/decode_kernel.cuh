@@ -100,10 +100,11 @@ struct DecodeCfg {
   static constexpr int D = D_;
   static constexpr int G = G_;
   static constexpr bool kMma = (G_ == 0);
-  static constexpr int W = 4;
-  static constexpr int kThreads = 32 * W;
   using Geo = TileGeom<T, BS, D>;
   static constexpr int kStageBytes = 2 * Geo::kTileBytes;
+  // Four warps unless two stages each would not fit beside the prefix array.
+  static constexpr int W = (4 * 2 * kStageBytes <= 160 * 1024) ? 4 : 2;
+  static constexpr int kThreads = 32 * W;
   static constexpr int NS = cmin(4, cmax(2, 98304 / (W * kStageBytes)));
   static constexpr int kRingBytes = W * NS * kStageBytes;
   static constexpr int kRowsMax = kMma ? 16 : G;
@@ -114,6 +115,8 @@ struct DecodeCfg {
   // Dynamic shared memory = 1024 (alignment slack) + main + barriers + misc
   // + (num_seqs + 1) ints of partition prefix in persistent mode.
   static constexpr int kFixedSmem = 1024 + kMainBytes + kBarBytes + kMiscInts * 4;
+  // 227 KB per CTA, leaving room for the prefix array of up to 4096 sequences.
+  static_assert(kFixedSmem + 4097 * 4 <= 227 * 1024, "shared memory budget exceeded");
   static_assert(!kMma || sizeof(T) == 2, "tensor-core path is bf16 only");
   static_assert(kMma || D % 32 == 0, "CUDA-core path needs head_dim % 32 == 0");
 };
