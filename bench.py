@@ -1,0 +1,606 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode step on B200.
+
+One step = one pass of the whole hot path over one batch: the block
+manager's slot/copy-on-write decisions for one appended token per sequence
+(precomputed on the host before timing), the copy-on-write block copies,
+the KV-append scatter, and split-context decode attention (partition kernel
+plus log-sum-exp merge) over the paged cache.
+
+Default workload (N=1): MHA decode, 7B-style: batch 64, 32 query heads = 32
+KV heads, head_dim 128, bf16, block size 16, context lengths uniform in
+[1, 2048], pool 16384 blocks placed by a seeded shuffle, values N(0, 1).
+The per-step inputs (queries, new K/V, slots, block tables, lengths) of R
+consecutive decode steps are made ahead of time and cycled; every step does
+the full work of a real decode step at its context lengths. The KV bytes a
+step reads (~1 GB) exceed the 126 MB L2, so no flush is needed.
+
+value      = algorithmic bytes of the step (valid K/V tokens + q + out + block
+             table entries + lengths + append + copies) / device time, GB/s,
+             summed over ranks, time = max over ranks (CUDA events).
+roofline   = the decode call alone (partition kernel + merge), its algorithmic
+             bytes / its event-timed duration, against the measured HBM peak.
+e2e        = the same metric through the public API from pinned host buffers:
+             per step the host block manager step, H2D of the step's inputs,
+             the kernels, D2H of the output, stream synchronisation.
+cpu_baseline / --impl reference: the CPU oracle (float64 NumPy) timed on a
+             bounded sample of the same workload on the host cores.
+
+Multi-GPU (torchrun): every rank runs its own independent batch (different
+seed), no data-path collective; scaling is weak.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: KV GB/s achieved & % of B200 HBM peak; decode tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# workload selection and byte accounting
+
+def make_workload(name: str, rank: int, batch: int | None = None):
+    from paged_kv_cache_336_b200 import workloads
+    if name == "mha":
+        if batch:   # smaller pool for profiling captures: room for the batch plus growth
+            w = workloads.mha(repeat=rank, batch=batch)
+            need = int(np.sum((w.context_lens + 300) // w.block_size + 1))
+            w.num_blocks = need
+            w.free_order = np.random.default_rng(w.seed).permutation(need).astype(np.int32)
+            return w
+        return workloads.mha(repeat=rank)
+    if name == "gqa":
+        return workloads.gqa(repeat=rank)
+    if name == "prefix":
+        return workloads.prefix(repeat=rank)
+    if name == "prefix_cow":
+        return workloads.prefix_cow(repeat=rank)
+    if name == "long16":
+        return workloads.long(repeat=rank, block_size=16, slack=0.1)
+    if name == "long32":
+        return workloads.long(repeat=rank, block_size=32, slack=0.1)
+    if name == "tiny":
+        return workloads.tiny(repeat=rank)
+    raise SystemExit(f"unknown workload {name}")
+
+
+def workload_label(w) -> str:
+    return (f"{w.name}: batch {len(w.decode_seqs)}, {w.num_q_heads}q/{w.num_kv_heads}kv heads, "
+            f"head_dim {w.head_dim}, {w.dtype}, block {w.block_size}")
+
+
+def decode_bytes(w, ctx: np.ndarray) -> int:
+    """Algorithmic bytes of one decode call: valid K and V tokens, q, out,
+    the block-table entries read and the context lengths."""
+    e = w.elt_bytes
+    kv = int(np.sum(ctx)) * w.num_kv_heads * w.head_dim * e * 2
+    qo = 2 * len(ctx) * w.num_q_heads * w.head_dim * e
+    bt = int(np.sum((ctx + w.block_size - 1) // w.block_size)) * 4 + 4 * len(ctx)
+    return kv + qo + bt
+
+
+def append_bytes(w, num_tokens: int) -> int:
+    per = num_tokens * w.num_kv_heads * w.head_dim * w.elt_bytes * 2
+    return 2 * per + 8 * num_tokens   # read new K/V, write them, read slots
+
+
+def copy_bytes(w, num_pairs: int) -> int:
+    block = w.num_kv_heads * w.block_size * w.head_dim * w.elt_bytes
+    return num_pairs * (2 * 2 * block + 16)
+
+
+# ---------------------------------------------------------------------------
+# measured peaks, clocks, profile traffic
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_336_b200", "csrc")
+    for name in ("decode_kernel.cuh", "device_common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return int(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+
+class DeviceStep:
+    """Device-resident inputs of R consecutive decode steps, cycled."""
+
+    def __init__(self, w, states: int, partition_tokens: int, device, whole: bool = False):
+        import torch
+        from paged_kv_cache_336_b200 import binding, workloads
+        self.torch, self.binding = torch, binding
+        self.w = w
+        self.partition_tokens = partition_tokens
+        self.whole = whole
+        self.bm = binding.BlockManager(w.num_blocks, w.block_size, w.max_blocks_per_seq,
+                                       w.free_order)
+        for s in w.prefill_seqs:
+            self.bm.allocate(s, int(w.context_lens[s]))
+        for parent, child in w.forks:
+            self.bm.fork(parent, child)
+        for s, n in sorted(w.extra_tokens.items()):
+            for _ in range(n):
+                self.bm.append_slot(s)
+        self.k_pool, self.v_pool = workloads.draw_pools(w, device)
+        B = len(w.decode_seqs)
+        T = len(w.step_seqs)
+        self.B, self.T = B, T
+        self.states = []
+        for i in range(states):
+            st = {}
+            if T:
+                slots, pairs = self.bm.append_slots_arrays(w.step_seqs)
+            else:
+                slots, pairs = np.zeros(0, np.int64), np.zeros((0, 2), np.int64)
+            tables, ctx = self.bm.export(w.decode_seqs)
+            st["slots"] = torch.from_numpy(slots).to(device)
+            st["pairs"] = torch.from_numpy(pairs).to(device)
+            st["tables"] = torch.from_numpy(tables).to(device)
+            st["ctx"] = torch.from_numpy(ctx).to(device)
+            st["q"] = workloads.draw_queries(w, B, step=i, device=device)
+            kn, vn = workloads.draw_new_kv(w, max(T, 1), step=i, device=device)
+            st["k_new"], st["v_new"] = kn[:T].contiguous(), vn[:T].contiguous()
+            st["ctx_np"] = ctx.astype(np.int64)
+            st["n_pairs"] = int(pairs.shape[0])
+            st["decode_bytes"] = decode_bytes(w, st["ctx_np"])
+            st["step_bytes"] = (st["decode_bytes"] + append_bytes(w, T) + copy_bytes(w, st["n_pairs"]))
+            self.states.append(st)
+        self.out = torch.empty_like(self.states[0]["q"])
+        self.ws = binding.SplitWorkspace(B, w.num_q_heads, w.head_dim, w.block_size,
+                                         w.max_blocks_per_seq, partition_tokens, device)
+        pb = partition_tokens // w.block_size
+        self.merge_launched = (-(-w.max_blocks_per_seq // pb) > 1) and not whole
+
+    def launches(self, st) -> int:
+        return (1 if st["n_pairs"] else 0) + (1 if self.T else 0) + 1 + (1 if self.merge_launched else 0)
+
+    def run(self, i, ev=None):
+        st = self.states[i % len(self.states)]
+        b = self.binding
+        if st["n_pairs"]:
+            b.copy_blocks(self.k_pool, self.v_pool, st["pairs"])
+        if self.T:
+            b.kv_append(st["k_new"], st["v_new"], st["slots"], self.k_pool, self.v_pool)
+        if ev is not None:
+            ev[0].record()
+        if self.whole:
+            b.decode(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"], self.w.scale,
+                     out=self.out)
+        else:
+            b.decode_split(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"],
+                           self.w.scale, partition_tokens=self.partition_tokens, out=self.out,
+                           workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+        return st
+
+
+def run_ours(args, rank, world, device_index):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_336_b200 import binding
+
+    device = torch.device("cuda", device_index)
+    torch.cuda.set_device(device)
+    w = make_workload(args.workload, rank, args.batch)
+    R = max(1, min(args.states, args.steps + args.warmup)) if args.workload != "prefix_cow" else 1
+    ds = DeviceStep(w, R, args.partition_tokens, device, whole=args.decode_mode == "whole")
+
+    for i in range(args.warmup):
+        ds.run(i)
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(device_index)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record()
+    total_bytes = 0
+    decode_bytes_sum = 0
+    launches = 0
+    for i in range(args.steps):
+        st = ds.run(args.warmup + i, evs[i])
+        total_bytes += st["step_bytes"]
+        decode_bytes_sum += st["decode_bytes"]
+        launches += ds.launches(st)
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clock_info = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    decode_ms = sum(a.elapsed_time(b) for a, b in evs)
+
+    # max time over ranks, bytes summed over ranks
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+        b = torch.tensor([float(total_bytes), float(args.steps * ds.B)], device=device,
+                         dtype=torch.float64)
+        dist.all_reduce(b, op=dist.ReduceOp.SUM)
+        all_bytes, all_tokens = float(b[0].item()), float(b[1].item())
+    else:
+        ms_max, all_bytes, all_tokens = ms, float(total_bytes), float(args.steps * ds.B)
+
+    gbs = all_bytes / (ms_max * 1e-3) / 1e9
+    tok_s = all_tokens / (ms_max * 1e-3)
+    decode_gbs = decode_bytes_sum / (decode_ms * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+
+    # ---- end to end through the public API (host buffers, pinned) ----------------
+    e2e = run_e2e(args, ds, rank, world, device)
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC,
+            "value": round(gbs, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_max / args.steps, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": w.dtype,
+            "data": "synthetic (seeded N(0,1) values, seeded shuffled block placement)",
+            "config": {
+                "workload": workload_label(w),
+                "global_batch": ds.B * world,
+                "context_lens": ("uniform [1, 2048]" if w.name == "mha" else "see workload"),
+                "mean_context": round(float(np.mean([s["ctx_np"].mean() for s in ds.states])), 1),
+                "partition_tokens": args.partition_tokens,
+                "step": "bm slots/CoW (host, precomputed) + copy_blocks + kv_append + "
+                        "decode_split (partition + LSE merge)",
+                "decode_states_cycled": len(ds.states),
+                "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
+                "parallelism": f"independent batch per GPU x{world}",
+            },
+            "decode_tokens_per_s": round(tok_s, 1),
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "pa_decode_split (paged_decode_kernel + lse_merge_kernel)",
+                "achieved": round(decode_gbs, 2),
+                "peak": peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": round(decode_gbs / peak, 4),
+                "frac_of_8TBs_spec": round(decode_gbs / 8000.0, 4),
+                "traffic": profiled_traffic(args.workload),
+                "algorithmic_bytes_per_launch": int(decode_bytes_sum / args.steps),
+                "avg_launch_us": round(decode_ms / args.steps * 1e3, 2),
+            },
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clock_info,
+        }
+    return result
+
+
+def run_e2e(args, ds, rank, world, device):
+    """Same metric through the public API from pinned host buffers."""
+    import torch
+    import torch.distributed as dist
+    b = ds.binding
+    w = ds.w
+    steps = max(3, min(args.e2e_steps, args.steps))
+    B, T = ds.B, ds.T
+    # host-side inputs of every e2e step (pinned)
+    hq = [ds.states[i % len(ds.states)]["q"].cpu().pin_memory() for i in range(min(steps, 8))]
+    hk = [ds.states[i % len(ds.states)]["k_new"].cpu().pin_memory() for i in range(min(steps, 8))]
+    hv = [ds.states[i % len(ds.states)]["v_new"].cpu().pin_memory() for i in range(min(steps, 8))]
+    dq = torch.empty_like(ds.states[0]["q"])
+    dk = torch.empty_like(ds.states[0]["k_new"])
+    dv = torch.empty_like(ds.states[0]["v_new"])
+    dslots = torch.empty(max(T, 1), dtype=torch.int64, device=device)
+    dpairs = torch.empty((max(T, 1), 2), dtype=torch.int64, device=device)
+    dtables = torch.empty((B, w.max_blocks_per_seq), dtype=torch.int32, device=device)
+    dctx = torch.empty(B, dtype=torch.int32, device=device)
+    hslots = torch.empty(max(T, 1), dtype=torch.int64).pin_memory()
+    hpairs = torch.empty((max(T, 1), 2), dtype=torch.int64).pin_memory()
+    htables = torch.empty((B, w.max_blocks_per_seq), dtype=torch.int32).pin_memory()
+    hctx = torch.empty(B, dtype=torch.int32).pin_memory()
+    hout = torch.empty(ds.out.shape, dtype=ds.out.dtype).pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = d2h = 0
+    total = 0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = time.perf_counter()
+    for i in range(steps):
+        # host block manager step (C++), then uploads
+        if T:
+            slots, pairs = ds.bm.append_slots_arrays(w.step_seqs)
+            hslots[:T].copy_(torch.from_numpy(slots))
+            npairs = pairs.shape[0]
+            if npairs:
+                hpairs[:npairs].copy_(torch.from_numpy(pairs))
+        else:
+            npairs = 0
+        tables, ctx = ds.bm.export(w.decode_seqs)
+        htables.copy_(torch.from_numpy(tables))
+        hctx.copy_(torch.from_numpy(ctx))
+        j = i % len(hq)
+        dq.copy_(hq[j], non_blocking=True)
+        dk.copy_(hk[j], non_blocking=True)
+        dv.copy_(hv[j], non_blocking=True)
+        dtables.copy_(htables, non_blocking=True)
+        dctx.copy_(hctx, non_blocking=True)
+        step_h2d = dq.numel() * dq.element_size() + 2 * dk.numel() * dk.element_size() + \
+            htables.numel() * 4 + hctx.numel() * 4
+        if T:
+            dslots[:T].copy_(hslots[:T], non_blocking=True)
+            step_h2d += T * 8
+        if npairs:
+            dpairs[:npairs].copy_(hpairs[:npairs], non_blocking=True)
+            b.copy_blocks(ds.k_pool, ds.v_pool, dpairs[:npairs])
+            step_h2d += npairs * 16
+        if T:
+            b.kv_append(dk, dv, dslots[:T], ds.k_pool, ds.v_pool)
+        b.decode_split(dq, ds.k_pool, ds.v_pool, dtables, dctx, w.scale,
+                       partition_tokens=ds.partition_tokens, out=ds.out, workspace=ds.ws)
+        hout.copy_(ds.out, non_blocking=True)
+        stream.synchronize()   # the step's result is on the host
+        h2d += step_h2d
+        d2h += hout.numel() * hout.element_size()
+        total += decode_bytes(w, ctx.astype(np.int64)) + append_bytes(w, T) + copy_bytes(w, npairs)
+    elapsed = time.perf_counter() - t_start
+    if world > 1:
+        t = torch.tensor([elapsed], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+        bt = torch.tensor([float(total)], device=device, dtype=torch.float64)
+        dist.all_reduce(bt, op=dist.ReduceOp.SUM)
+        total = float(bt.item())
+    return {"value": round(total / elapsed / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d / steps), "d2h_bytes_per_step": int(d2h / steps),
+            "steps": steps, "ms_per_step": round(elapsed / steps * 1e3, 4),
+            "path": "python binding -> C ABI; host block manager step + pinned H2D + kernels "
+                    "+ D2H out + stream sync per step"}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (cpu_baseline leg and --impl reference)
+
+def time_oracle(w, budget_s: float, seed: int = 0):
+    """Times the float64 oracle on whole sequences of the workload (all query
+    heads of each), one thread, until ~budget_s seconds of work are done.
+    Returns (GB/s of algorithmic bytes, tokens/s, description)."""
+    import torch
+    from threadpoolctl import threadpool_limits
+    import oracle
+    from paged_kv_cache_336_b200 import workloads
+
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(len(w.decode_seqs))
+    Hkv, bs, D = w.num_kv_heads, w.block_size, w.head_dim
+    done_bytes = 0
+    done_seqs = 0
+    elapsed = 0.0
+    torch.set_num_threads(1)
+    with threadpool_limits(limits=1):
+        for idx in order:
+            ctx = int(w.context_lens[idx]) + (1 if w.step_seqs else 0)
+            nb = -(-ctx // bs)
+            # a contiguous one-sequence pool drawn from the same distribution
+            kp = workloads.draw_normal((nb, Hkv, bs, D), w.dtype, w.seed * 7 + int(idx)).double().numpy()
+            vp = workloads.draw_normal((nb, Hkv, bs, D), w.dtype, w.seed * 7 + 99991 + int(idx)).double().numpy()
+            q = workloads.draw_normal((1, w.num_q_heads, D), w.dtype, w.seed * 7 + 3 + int(idx)).double().numpy()
+            table = np.arange(nb)[None, :]
+            t0 = time.perf_counter()
+            for h in range(w.num_q_heads):
+                oracle.paged_decode_one(q, kp, vp, table, [ctx], w.scale, 0, h)
+            elapsed += time.perf_counter() - t0
+            done_bytes += decode_bytes(w, np.array([ctx]))
+            done_seqs += 1
+            if elapsed >= budget_s:   # at least one whole sequence per call
+                break
+    desc = (f"{done_seqs} of {len(w.decode_seqs)} sequences (all {w.num_q_heads} query heads each, "
+            f"the workload's context lengths and N(0,1) values) of the {w.name} workload, "
+            f"{elapsed:.2f} s, float64 NumPy oracle, 1 thread")
+    return done_bytes / elapsed / 1e9, done_seqs / elapsed, desc, elapsed
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = make_workload(args.workload, 0, args.batch)
+    # each step: a bounded sample of the workload (at least one whole sequence),
+    # sized so that the whole run ends within a few minutes
+    per_step = min(10.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        time_oracle(w, per_step / 4)
+    vals, tok, descs, secs = [], [], [], 0.0
+    for i in range(args.steps):
+        g, t, d, el = time_oracle(w, per_step, seed=i)
+        vals.append(g)
+        tok.append(t)
+        descs.append(d)
+        secs += el
+    value = statistics.mean(vals)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 5),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) values)",
+        "config": {"workload": workload_label(w), "partition_tokens": args.partition_tokens},
+        "decode_tokens_per_s": round(statistics.mean(tok), 4),
+        "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": descs[0]},
+        "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mha",
+                    choices=["mha", "gqa", "prefix", "prefix_cow", "long16", "long32", "tiny"])
+    ap.add_argument("--partition-tokens", type=int, default=512)
+    ap.add_argument("--decode-mode", choices=["split", "whole"], default="split",
+                    help="split: pa_decode_split (persistent, partitions + merge); "
+                         "whole: pa_decode (one CTA per sequence and KV head)")
+    ap.add_argument("--states", type=int, default=64, help="distinct decode steps cycled")
+    ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="mha only: smaller batch and pool (profiling captures)")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and args.cpu_budget > 0:
+                g, t, desc, _ = time_oracle(make_workload(args.workload, 0, args.batch),
+                                            args.cpu_budget)
+                res["cpu_baseline"] = {"value": round(g, 5), "unit": "GB/s", "cores": 1,
+                                       "kind": "oracle", "sample": desc,
+                                       "decode_tokens_per_s": round(t, 4)}
+            else:
+                res["cpu_baseline"] = None
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -34,7 +34,9 @@
  *   arithmetic is fp32 in both cases. out has q's dtype.
  * - Supported shapes: head_dim in {64, 128, 256} (256 for bf16 only),
  *   block_size in {16, 32}; bf16 takes any group size 1..16, fp32 takes group
- *   sizes 1, 2, 4, 8. num_blocks * num_kv_heads * block_size < 2^31.
+ *   sizes 1, 2, 4, 8. bf16 products run on tensor cores (P rounded to bf16
+ *   before P*V, fp32 accumulation); fp32 runs on CUDA cores.
+ *   num_blocks * num_kv_heads * block_size < 2^31.
  *   Pointers to pools, q, out, k_new and v_new must be 16-byte aligned.
  * - Errors: invalid arguments are rejected before anything is enqueued
  *   (PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED, nothing changes). Kernels never

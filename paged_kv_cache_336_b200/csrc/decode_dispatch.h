@@ -18,7 +18,6 @@ struct DecodeInstance {
 
 // Each returns false when (head_dim, block_size, group) has no instance.
 bool find_decode_f32(int head_dim, int block_size, int group, DecodeInstance* out);
-bool find_decode_bf16_simt(int head_dim, int block_size, int group, DecodeInstance* out);
 bool find_decode_bf16_mma(int head_dim, int block_size, DecodeInstance* out);
 
 }  // namespace pagedkv

@@ -1,5 +1,4 @@
-// bf16 instances of the paged decode kernel: CUDA-core path for group 1,
-// tensor-core path for groups 2..16.
+// bf16 instances of the paged decode kernel (tensor-core path, groups 1..16).
 #include "decode_dispatch.h"
 #include "decode_kernel.cuh"
 
@@ -16,17 +15,6 @@ static DecodeInstance make_bf16(const char* name) {
   r.stages = Cfg::NS;
   r.name = name;
   return r;
-}
-
-bool find_decode_bf16_simt(int head_dim, int block_size, int group, DecodeInstance* out) {
-  if (group != 1) return false;
-  if (block_size == 16 && head_dim == 64) { *out = make_bf16<16, 64, 1>("simt_bf16"); return true; }
-  if (block_size == 16 && head_dim == 128) { *out = make_bf16<16, 128, 1>("simt_bf16"); return true; }
-  if (block_size == 16 && head_dim == 256) { *out = make_bf16<16, 256, 1>("simt_bf16"); return true; }
-  if (block_size == 32 && head_dim == 64) { *out = make_bf16<32, 64, 1>("simt_bf16"); return true; }
-  if (block_size == 32 && head_dim == 128) { *out = make_bf16<32, 128, 1>("simt_bf16"); return true; }
-  if (block_size == 32 && head_dim == 256) { *out = make_bf16<32, 256, 1>("simt_bf16"); return true; }
-  return false;
 }
 
 bool find_decode_bf16_mma(int head_dim, int block_size, DecodeInstance* out) {

@@ -20,11 +20,11 @@
 // * Tiles land in 128-byte-swizzled layout: each 128-byte column chunk of a
 //   tile is one TMA box of block_size rows; unit (16 B) u of row r sits at
 //   u ^ (r % 8). Row-wise reads and 8x8 ldmatrix reads are bank-conflict free.
-// * MHA (and fp32) path: CUDA cores. Each lane owns head_dim/32 dims; per-token
+// * fp32 path: CUDA cores. Each lane owns head_dim/32 dims; per-token
 //   partial dot products are folded across lanes by a transposing butterfly
 //   (block_size values in log2(32) shuffle stages), one exp2 per token, p
 //   broadcast by shuffles for the p*V accumulate.
-// * GQA path (bf16, group 2..16): tensor cores via mma.sync m16n8k16. The
+// * bf16 path (any group 1..16, MHA included): tensor cores via mma.sync m16n8k16. The
 //   group's query rows (padded to 16) are the A operand held in registers;
 //   S = Q K^T comes from ldmatrix'ed K tiles, P stays in registers as the A
 //   operand of O += P V with V fragments from ldmatrix.trans.

@@ -168,7 +168,7 @@ def long(repeat: int = 0, block_size: int = 16, slack: float = 0.0, batch: int =
     return Workload(
         name=f"long_bs{block_size}", num_q_heads=64, num_kv_heads=8, head_dim=128,
         block_size=block_size, dtype=BF16, num_blocks=nb,
-        max_blocks_per_seq=per_seq + 1, context_lens=ctx, free_order=_perm(rng, nb),
+        max_blocks_per_seq=per_seq + 8, context_lens=ctx, free_order=_perm(rng, nb),
         seed=seed, prefill_seqs=list(range(batch)),
         step_seqs=list(range(batch)) if slack > 0 else [],
         decode_seqs=list(range(batch)), partition_tokens=512)
