@@ -138,6 +138,43 @@ pa_status_t pa_decode_split(const void* q, const void* k_pool, const void* v_poo
                             void* stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_decode_split_static - pa_decode_split for callers that cannot allocate
+ * device memory. (Not from the pages: the paper has no counterpart; this is
+ * an interface convenience of this library.)
+ *
+ * Some callers have no way to call cudaMalloc: their device memory is owned
+ * by another allocator (a framework's caching allocator or a fixed arena
+ * sized up front), or they run where an allocation that may synchronise the
+ * device or fail halfway through a decode loop is not acceptable. This entry
+ * point takes the same inputs and output as pa_decode_split, minus the
+ * workspace: its scratch (ticket counters and per-partition partials) lives
+ * in a fixed array of PA_STATIC_SCRATCH_BYTES inside the library's device
+ * image, which every GPU that loads the library holds until the process
+ * exits. It allocates no device memory and calls no allocating routine.
+ *
+ * - Sizes whose scratch would exceed PA_STATIC_SCRATCH_BYTES (see
+ *   pa_decode_split_workspace_size) are rejected with PA_ERR_INVALID_ARG and
+ *   a message naming both sizes, before anything is enqueued.
+ * - The first call on each device, with that device current, looks up the
+ *   array's device address (cudaGetSymbolAddress) and caches it; make that
+ *   first call before any stream capture.
+ * - All calls on a device share the one array, and it keeps the previous
+ *   call's contents. Each call clears the part that must start at zero (on
+ *   `stream`, before its kernels). Calls that may overlap on the GPU (other
+ *   streams, other host threads) race on the array and must be serialised
+ *   by the caller; calls issued in order on one stream are safe.
+ * ------------------------------------------------------------------------- */
+#define PA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void* v_pool,
+                                   const int32_t* block_tables, const int32_t* context_lens,
+                                   int num_seqs, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int block_size, int num_blocks,
+                                   int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                                   int partition_tokens, void* out, uint32_t* dev_err,
+                                   void* stream);
+
+/* ---------------------------------------------------------------------------
  * pa_kv_append - decode-step write of new tokens' keys and values into their
  * slots ([Q], Map Logical to Physical Blocks: decode appends into the partly
  * filled tail block; [G] section 4 step 3: the write proceeds on the private

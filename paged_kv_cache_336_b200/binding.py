@@ -74,6 +74,8 @@ _SIGNATURES = {
     "pa_decode_split_workspace_init": (_I, [_P, _SZ, _P]),
     "pa_decode_split": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ,
                              _P, _P, _P]),
+    "pa_decode_split_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
+                                    _P, _P, _P]),
     "pa_kv_append": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _P, _I, _SZ, _I, _P, _P]),
     "pa_bm_create": (_I, [_I, _I, _I, _P, ctypes.POINTER(_P)]),

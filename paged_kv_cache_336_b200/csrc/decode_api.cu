@@ -340,6 +340,38 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
   return launch_error("decode");
 }
 
+// ---- scratch for pa_decode_split_static ------------------------------------------
+// Callers that cannot allocate device memory get their split-decode scratch
+// (ticket counters + per-partition partials) from this fixed array instead of
+// a workspace argument. It is part of the library's device image: every GPU
+// that loads the library holds these bytes until the process exits.
+constexpr size_t kStaticScratchBytes = PA_STATIC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_static_split_scratch[kStaticScratchBytes];
+
+// Device address of the array on the current device. In host code the array's
+// name is only a host-side stand-in, so the address is fetched with
+// cudaGetSymbolAddress once per device (with that device current) and cached.
+pa_status_t static_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+  if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_UNSUPPORTED, "device %d >= %d", dev, kMaxDevices);
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_static_split_scratch);
+    if (err != cudaSuccess || p == nullptr)
+      return fail(PA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(err));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return PA_OK;
+}
+
 }  // namespace
 }  // namespace pagedkv
 
@@ -387,6 +419,42 @@ pa_status_t pa_decode_split(const void* q, const void* k_pool, const void* v_poo
               head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
               static_cast<cudaStream_t>(stream)};
   return run_decode(r, true, partition_tokens, workspace, workspace_bytes);
+}
+
+pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void* v_pool,
+                                   const int32_t* block_tables, const int32_t* context_lens,
+                                   int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                   int block_size, int num_blocks, int max_blocks_per_seq,
+                                   float scale, pa_dtype_t dtype, int partition_tokens, void* out,
+                                   uint32_t* dev_err, void* stream) {
+  DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+              head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
+              static_cast<cudaStream_t>(stream)};
+  // Everything that can be checked on the host is checked before the device
+  // is touched, the scratch size included.
+  DecodeInstance inst;
+  pa_status_t st = validate_and_pick(r, &inst);
+  if (st != PA_OK) return st;
+  if (partition_tokens <= 0 || partition_tokens % block_size != 0)
+    return fail(PA_ERR_INVALID_ARG, "partition_tokens (%d) must be a positive multiple of block_size",
+                partition_tokens);
+  if (num_seqs == 0) return ok();
+  const size_t need = split_layout(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
+                                   partition_tokens).total;
+  if (need > kStaticScratchBytes)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_decode_split_static needs %zu bytes of scratch for these sizes but its static "
+                "scratch holds %zu; use pa_decode_split with a caller workspace or a larger "
+                "partition_tokens",
+                need, kStaticScratchBytes);
+  void* scratch = nullptr;
+  st = static_scratch_address(&scratch);
+  if (st != PA_OK) return st;
+  // The array keeps whatever the last call left; the control header must
+  // start at zero.
+  cudaError_t err = cudaMemsetAsync(scratch, 0, kWorkspaceHeader, r.stream);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "clearing static scratch: %s", cudaGetErrorString(err));
+  return run_decode(r, true, partition_tokens, scratch, kStaticScratchBytes);
 }
 
 }  // extern "C"

@@ -1,0 +1,85 @@
+"""The no-allocation split decode entry point, pa_decode_split_static.
+
+It exists for callers that cannot call cudaMalloc (their device memory is
+owned by another allocator, or an allocation in the middle of a decode loop
+is not acceptable); its scratch is a fixed array inside the library. These
+tests call it through the C ABI and compare it with pa_decode_split, which
+takes a caller workspace, within the tolerances used by every decode test
+(fp32 max-abs 1e-5; bf16 max-abs 2e-2 and mean-abs 2e-3), on two calls in a
+row, since the array keeps the previous call's contents. Oversized requests
+must be refused before anything is enqueued.
+
+This file sorts last so that a run stopping at the first failure has run
+every other test first; it also passes when run alone in a fresh process.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_336_b200 import binding, workloads
+
+from gpu_util import check_close, device_tables, setup, to_f64
+
+pytestmark = pytest.mark.gpu
+
+STATIC_SCRATCH_BYTES = 16 * 1024 * 1024   # PA_STATIC_SCRATCH_BYTES in include/pagedkv.h
+
+
+def _call_static(q, k_pool, v_pool, bt, ctx, scale, partition_tokens, out, err):
+    lib = binding.library()
+    B, Hq, D = q.shape
+    NB, Hkv, BS, _ = k_pool.shape
+    dtype = binding.PA_F32 if q.dtype == torch.float32 else binding.PA_BF16
+    return lib.pa_decode_split_static(
+        q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), bt.data_ptr(), ctx.data_ptr(), B, Hq,
+        Hkv, D, BS, NB, bt.shape[1], float(scale), dtype, int(partition_tokens), out.data_ptr(),
+        err.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+
+@pytest.mark.parametrize("dtype,G", [(workloads.F32, 1), (workloads.BF16, 1), (workloads.BF16, 8)])
+def test_static_scratch_matches_workspace_entry_point(dtype, G):
+    torch.cuda.set_device(0)
+    w = workloads.random_small(31 + G, num_seqs=9, num_q_heads=2 * G, num_kv_heads=2,
+                               head_dim=128, block_size=16, dtype=dtype, max_ctx=400,
+                               fixed_lens=[0, 1, 400])
+    bm, k_pool, v_pool = setup(w)
+    q = workloads.draw_queries(w, 9, device="cuda")
+    bt, ctx, _, _ = device_tables(bm, list(range(9)))
+    partition = 48  # several partitions per sequence, ragged last one
+    need = binding.decode_split_workspace_size(9, 2 * G, 128, 16, bt.shape[1], partition)
+    assert need <= STATIC_SCRATCH_BYTES
+    ref = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=partition)
+    ref_np = to_f64(ref)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for call in range(2):
+        out = torch.full_like(q, float("nan"))
+        status = _call_static(q, k_pool, v_pool, bt, ctx, w.scale, partition, out, err)
+        assert status == binding.PA_OK, binding.library().pa_last_error_string()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0, f"call {call}: device error word {int(err.item()):#x}"
+        check_close(to_f64(out), ref_np, dtype, f"static scratch, call {call}")
+    assert torch.all(out[0] == 0)   # empty context
+
+
+def test_static_scratch_refuses_oversized_requests():
+    torch.cuda.set_device(0)
+    # small real buffers; the declared sizes are refused before any launch
+    q = torch.zeros(4, 64, 128, dtype=torch.bfloat16, device="cuda")
+    pool = torch.zeros(8, 8, 16, 128, dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros(4, 8, dtype=torch.int32, device="cuda")
+    ctx = torch.zeros(4, dtype=torch.int32, device="cuda")
+    out = torch.zeros_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lib = binding.library()
+    big_seqs, mbs = 4096, 8192
+    need = binding.decode_split_workspace_size(big_seqs, 64, 128, 16, mbs, 16)
+    assert need > STATIC_SCRATCH_BYTES
+    status = lib.pa_decode_split_static(
+        q.data_ptr(), pool.data_ptr(), pool.data_ptr(), bt.data_ptr(), ctx.data_ptr(), big_seqs,
+        64, 8, 128, 16, 8, mbs, 0.1, binding.PA_BF16, 16, out.data_ptr(), err.data_ptr(),
+        torch.cuda.current_stream().cuda_stream)
+    assert status == binding.PA_ERR_INVALID_ARG
+    assert b"static" in lib.pa_last_error_string() and b"scratch" in lib.pa_last_error_string()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and torch.all(out == 0)
