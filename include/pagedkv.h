@@ -114,11 +114,16 @@ pa_status_t pa_decode(const void* q, const void* k_pool, const void* v_pool,
  * the contiguous result ([G] section 3).
  *
  * workspace: caller-owned device memory of at least
- *   pa_decode_split_workspace_size(...) bytes, 256-byte aligned. Its first 256
- *   bytes are a control header that must be zero before the first call
- *   (pa_decode_split_workspace_init does that); every completed call leaves the
- *   header zero again, so one workspace serves any number of calls issued in
- *   stream order. Calls that may overlap on the GPU need separate workspaces.
+ *   pa_decode_split_workspace_size(...) bytes, 256-byte aligned. It starts
+ *   with a 256-byte control header (work-ticket counters) that must be zero
+ *   before the first call; pa_decode_split_workspace_init zeroes the whole
+ *   workspace. Every completed call leaves the header zero again, so one
+ *   workspace serves any number of calls issued in stream order. Calls that
+ *   may overlap on the GPU need separate workspaces. After a call that
+ *   reported PA_DEVERR_TIMEOUT, initialise the workspace again.
+ * Two kernels run: the partition kernel, then (when some sequence has more
+ *   than one partition) the merge kernel, launched as a programmatic
+ *   dependent so that it waits on the device rather than in the launch queue.
  * num_seqs must be <= 4096 (PA_ERR_UNSUPPORTED above that).
  * ------------------------------------------------------------------------- */
 size_t pa_decode_split_workspace_size(int num_seqs, int num_q_heads, int head_dim,

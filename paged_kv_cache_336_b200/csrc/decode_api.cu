@@ -44,7 +44,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // A pool [num_blocks][num_kv_heads][block_size][head_dim] viewed as a 2-D
 // tensor of rows = num_blocks*num_kv_heads*block_size, cols = head_dim; one
-// box = block_size rows x 128 bytes, 128-byte swizzle.
+// box = 16 rows x 128 bytes, 128-byte swizzle.
 struct MapKey {
   const void* base;
   int rows;
@@ -80,7 +80,9 @@ pa_status_t pool_tensor_map(const void* base, int rows, int head_dim, int block_
   const int eb = elt_bytes(dtype);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * eb};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(block_size)};
+  // One box = one 16-token pipeline unit x 128 bytes (block sizes 16 and 32
+  // are both multiples of it).
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), 16u};
   cuuint32_t estr[2] = {1, 1};
   CUtensorMap m;
   std::memset(&m, 0, sizeof(m));
@@ -234,8 +236,14 @@ pa_status_t launch_error(const char* what) {
   return ok();
 }
 
+// Workspace of the split decode:
+//   [0, 256)   control header: ticket counter, finished-CTA counter
+//   m, l       float [num_seqs][num_q_heads][pmax]
+//   acc        float [num_seqs][num_q_heads][pmax][head_dim]
+// The header must be zero before a call; calls leave it zero.
 struct SplitLayout {
   size_t m_off, l_off, acc_off, total;
+  size_t zero_bytes;  // bytes that must start at zero (the header)
   int pmax;
 };
 
@@ -246,6 +254,7 @@ SplitLayout split_layout(int num_seqs, int num_q_heads, int head_dim, int block_
   L.pmax = (max_blocks_per_seq + pb - 1) / pb;
   const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * L.pmax;
   L.m_off = kWorkspaceHeader;
+  L.zero_bytes = kWorkspaceHeader;
   L.l_off = L.m_off + align256(rows * 4);
   L.acc_off = L.l_off + align256(rows * 4);
   L.total = L.acc_off + align256(rows * head_dim * 4);
@@ -331,10 +340,22 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
   cudaError_t err = cudaLaunchKernel(inst.kernel, grid, dim3(inst.threads), args, smem, r.stream);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
   if (split && a.max_partitions > 1) {
+    // The merge grid is a programmatic dependent of the decode grid: it may be
+    // scheduled before the decode grid ends and waits on the device
+    // (griddepcontrol.wait) until the partials are complete and visible.
     int bs = r.block_size;
     void* margs[] = {&a, &bs};
-    const int warps = r.num_seqs * r.num_q_heads;
-    err = cudaLaunchKernel(inst.merge, dim3((warps + 3) / 4), dim3(128), margs, 0, r.stream);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(r.num_seqs * r.num_q_heads));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = r.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelExC(&cfg, inst.merge, margs);
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(err));
   }
   return launch_error("decode");
@@ -404,7 +425,7 @@ pa_status_t pa_decode_split_workspace_init(void* workspace, size_t workspace_byt
   if (workspace == nullptr || workspace_bytes < kWorkspaceHeader)
     return fail(PA_ERR_INVALID_ARG, "workspace must hold at least %zu bytes", kWorkspaceHeader);
   cudaError_t err =
-      cudaMemsetAsync(workspace, 0, kWorkspaceHeader, static_cast<cudaStream_t>(stream));
+      cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "workspace init: %s", cudaGetErrorString(err));
   return ok();
 }
@@ -439,8 +460,9 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
     return fail(PA_ERR_INVALID_ARG, "partition_tokens (%d) must be a positive multiple of block_size",
                 partition_tokens);
   if (num_seqs == 0) return ok();
-  const size_t need = split_layout(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
-                                   partition_tokens).total;
+  const SplitLayout layout = split_layout(num_seqs, num_q_heads, head_dim, block_size,
+                                         max_blocks_per_seq, partition_tokens);
+  const size_t need = layout.total;
   if (need > kStaticScratchBytes)
     return fail(PA_ERR_INVALID_ARG,
                 "pa_decode_split_static needs %zu bytes of scratch for these sizes but its static "
@@ -452,7 +474,7 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
   if (st != PA_OK) return st;
   // The array keeps whatever the last call left; the control header must
   // start at zero.
-  cudaError_t err = cudaMemsetAsync(scratch, 0, kWorkspaceHeader, r.stream);
+  cudaError_t err = cudaMemsetAsync(scratch, 0, layout.zero_bytes, r.stream);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "clearing static scratch: %s", cudaGetErrorString(err));
   return run_decode(r, true, partition_tokens, scratch, kStaticScratchBytes);
 }

@@ -11,9 +11,10 @@
 //
 // How (B200 design; the pages describe no kernel, so all of this is ours):
 // * Work item = (sequence, KV head, partition of PB blocks). A CTA of W warps
-//   takes an item; warp w walks the item's blocks w, w+W, w+2W, ... Each warp
+//   takes an item; the pipeline unit is 16 tokens (one block at block size
+//   16, half a block at 32). Warp w walks units w, w+W, w+2W, ... Each warp
 //   owns an NS-stage ring in shared memory fed by its lane 0 with 2-D TMA
-//   loads (cp.async.bulk.tensor) of the (block, head) K and V tiles, each
+//   loads (cp.async.bulk.tensor) of the unit's K and V tiles, each
 //   completing on an mbarrier. Block ids are prefetched 32 at a time into
 //   lane registers, one chunk ahead, so the dependent table load is off the
 //   critical path.
@@ -30,7 +31,8 @@
 //   operand of O += P V with V fragments from ldmatrix.trans.
 // * After an item, the warps' (m, l, acc) are merged through shared memory;
 //   a sequence that fits one partition is written to `out`, otherwise the
-//   partition's (m, l, acc) go to the workspace for the merge kernel.
+//   partition's (m, l, acc) go to the workspace for the merge kernel, which
+//   is launched as a programmatic dependent of this one.
 // * Persistent mode (split decode): grid = SMs x occupancy; CTAs pull item
 //   tickets from a device counter. Every CTA builds the per-sequence partition
 //   prefix sum in shared memory to map a ticket to (s, p, kvh). The last CTA to
@@ -100,11 +102,18 @@ struct DecodeCfg {
   static constexpr int D = D_;
   static constexpr int G = G_;
   static constexpr bool kMma = (G_ == 0);
-  using Geo = TileGeom<T, BS, D>;
+  // The pipeline moves 16-token units: one unit per block at block size 16,
+  // two at block size 32 (each warp then always reads the same half of its
+  // blocks), so a stage is the same size whatever the block size.
+  static constexpr int UR = 16;
+  static constexpr int UPB = BS / UR;
+  static_assert(BS % UR == 0, "block_size must be a multiple of 16");
+  using Geo = TileGeom<T, UR, D>;
   static constexpr int kStageBytes = 2 * Geo::kTileBytes;
   // Four warps unless two stages each would not fit beside the prefix array.
   static constexpr int W = (4 * 2 * kStageBytes <= 160 * 1024) ? 4 : 2;
   static constexpr int kThreads = 32 * W;
+  static_assert(W % UPB == 0, "warps must cover whole blocks");
   static constexpr int NS = cmin(4, cmax(2, 98304 / (W * kStageBytes)));
   static constexpr int kRingBytes = W * NS * kStageBytes;
   static constexpr int kRowsMax = kMma ? 16 : G;
@@ -113,7 +122,8 @@ struct DecodeCfg {
   static constexpr int kBarBytes = W * NS * 8;
   static constexpr int kMiscInts = 8;
   // Dynamic shared memory = 1024 (alignment slack) + main + barriers + misc
-  // + (num_seqs + 1) ints of partition prefix in persistent mode.
+  // + (num_seqs + 1) ints of partition prefix in persistent mode. The merge of
+  // a sequence's partitions reuses the main area.
   static constexpr int kFixedSmem = 1024 + kMainBytes + kBarBytes + kMiscInts * 4;
   // 227 KB per CTA, leaving room for the prefix array of up to 4096 sequences.
   static_assert(kFixedSmem + 4097 * 4 <= 227 * 1024, "shared memory budget exceeded");
@@ -148,7 +158,7 @@ struct SimtWarp {
   using T = typename Cfg::Elt;
   static constexpr int G = Cfg::G;
   static constexpr int D = Cfg::D;
-  static constexpr int BS = Cfg::BS;
+  static constexpr int BS = Cfg::UR;  // rows per unit
   static constexpr int VEC = D / 32;
   using Geo = typename Cfg::Geo;
 
@@ -229,7 +239,7 @@ struct SimtWarp {
 template <class Cfg>
 struct MmaWarp {
   static constexpr int D = Cfg::D;
-  static constexpr int BS = Cfg::BS;
+  static constexpr int BS = Cfg::UR;  // rows per unit
   static constexpr int KS = D / 16;   // k-steps of S = Q K^T
   static constexpr int NT = BS / 8;   // 8-token n-tiles of S
   static constexpr int ND = D / 8;    // 8-dim n-tiles of O
@@ -402,6 +412,7 @@ __device__ __forceinline__ int clamp_ctx(int raw, int max_tokens) {
   return (raw < 0 || raw > max_tokens) ? 0 : raw;
 }
 
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -411,6 +422,9 @@ __global__ void __launch_bounds__(Cfg::kThreads)
   constexpr int W = Cfg::W;
   constexpr int NS = Cfg::NS;
   constexpr int BS = Cfg::BS;
+  constexpr int UR = Cfg::UR;
+  constexpr int UPB = Cfg::UPB;
+  constexpr int WB = W / UPB;  // warps per unit-half: block lanes
   constexpr int D = Cfg::D;
   constexpr int NT = Cfg::kThreads;
   using WarpT = typename std::conditional<Cfg::kMma, MmaWarp<Cfg>, SimtWarp<Cfg>>::type;
@@ -429,10 +443,16 @@ __global__ void __launch_bounds__(Cfg::kThreads)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const int hu = warp % UPB;  // which 16-token half of each block this warp reads
+  const int wb = warp / UPB;  // this warp's block lane
   const int B = a.num_seqs;
   const int Hkv = a.num_kv_heads;
   const int G = a.group;
   const int max_tokens = a.max_blocks_per_seq * BS;
+
+  // Let the merge grid (launched as a programmatic dependent) be scheduled
+  // now; it waits on the device for this grid's completion before it reads.
+  grid_dependents_launch();
 
   if (tid == 0) {
     for (int i = 0; i < W * NS; ++i) mbar_init(&bars[i], 1);
@@ -476,7 +496,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
   __syncthreads();
 
   const uint64_t policy = l2_policy(a.l2_hint);
-  uint32_t gcount = 0;  // blocks this warp has consumed so far (ring position)
+  uint32_t gcount = 0;  // units this warp has consumed so far (ring position)
 
   int item;
   if (a.persistent) {
@@ -519,9 +539,15 @@ __global__ void __launch_bounds__(Cfg::kThreads)
     const int b_begin = a.persistent ? p * a.partition_blocks : 0;
     const int b_end = a.persistent ? min(nb, b_begin + a.partition_blocks) : nb;
     const int nblk = max(0, b_end - b_begin);
-    const int nj = (nblk > warp) ? (nblk - warp + W - 1) / W : 0;
+    // This warp reads half `hu` of blocks b_begin + wb + j*WB.
+    const int nbj = (nblk > wb) ? (nblk - wb + WB - 1) / WB : 0;
+    int nj = nbj;
+    if (UPB > 1 && hu > 0 && nbj > 0) {
+      const int last_lb = b_begin + wb + (nbj - 1) * WB;
+      if (ctx - last_lb * BS <= hu * UR) nj -= 1;  // the context ends before this half
+    }
 
-    // ---- per-warp pipeline over blocks b_begin + warp + j*W ----------------------
+    // ---- per-warp pipeline over its units -----------------------------------------
     const T* q_group = reinterpret_cast<const T*>(a.q) +
                        (static_cast<int64_t>(s) * a.num_q_heads + static_cast<int64_t>(kvh) * G) * D;
     WarpT st;
@@ -531,9 +557,9 @@ __global__ void __launch_bounds__(Cfg::kThreads)
       st.begin(q_group, a.scale_log2, lane);
     }
 
-    const int32_t* bt = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq + b_begin + warp;
-    int bt_cur = (lane < nj) ? bt[lane * W] : -1;
-    int bt_nxt = (32 + lane < nj) ? bt[(32 + lane) * W] : -1;
+    const int32_t* bt = a.block_tables + static_cast<int64_t>(s) * a.max_blocks_per_seq + b_begin + wb;
+    int bt_cur = (lane < nbj) ? bt[lane * WB] : -1;
+    int bt_nxt = (32 + lane < nbj) ? bt[(32 + lane) * WB] : -1;
     int bt_chunk = 0;
     uint32_t bad = 0;  // bit per stage: the stage's block id was out of range
     uint8_t* my_ring = ring + warp * NS * Cfg::kStageBytes;
@@ -543,7 +569,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
       const int c = j >> 5;
       if (c != bt_chunk) {  // advance the block-id window by one chunk
         bt_cur = bt_nxt;
-        bt_nxt = ((c + 1) * 32 + lane < nj) ? bt[((c + 1) * 32 + lane) * W] : -1;
+        bt_nxt = ((c + 1) * 32 + lane < nbj) ? bt[((c + 1) * 32 + lane) * WB] : -1;
         bt_chunk = c;
       }
       const int phys = __shfl_sync(0xffffffffu, bt_cur, j & 31);
@@ -556,7 +582,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
         if (good) {
           uint8_t* kdst = my_ring + stage * Cfg::kStageBytes;
           uint8_t* vdst = kdst + Geo::kTileBytes;
-          const int32_t y = (phys * Hkv + kvh) * BS;
+          const int32_t y = (phys * Hkv + kvh) * BS + hu * UR;
           mbar_arrive_expect_tx(bar, 2 * Geo::kTileBytes);
 #pragma unroll
           for (int c2 = 0; c2 < Geo::kChunks; ++c2) {
@@ -584,8 +610,8 @@ __global__ void __launch_bounds__(Cfg::kThreads)
         break;
       }
       if (!(bad & (1u << stage))) {
-        const int lb = b_begin + warp + j * W;  // logical block
-        const int nvalid = min(BS, ctx - lb * BS);
+        const int lb = b_begin + wb + j * WB;  // logical block
+        const int nvalid = min(UR, ctx - lb * BS - hu * UR);
         uint8_t* kt = my_ring + stage * Cfg::kStageBytes;
         st.block(kt, kt + Geo::kTileBytes, nvalid, lane);
       }
@@ -613,6 +639,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
     }
     __syncthreads();
     const bool final_out = (nparts == 1);
+    const int64_t row0 = static_cast<int64_t>(s) * a.num_q_heads + static_cast<int64_t>(kvh) * G;
     for (int idx = tid; idx < G * D; idx += NT) {
       const int h = idx / D;
       const int d = idx - h * D;
@@ -628,7 +655,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
           A = fmaf(sm_acc[(w * Cfg::kRowsMax + h) * D + d], e, A);
         }
       }
-      const int64_t row = static_cast<int64_t>(s) * a.num_q_heads + kvh * G + h;
+      const int64_t row = row0 + h;
       if (final_out) {
         reinterpret_cast<T*>(a.out)[row * D + d] = Elt<T>::from_f32(L > 0.f ? A / L : 0.f);
       } else {
@@ -665,40 +692,73 @@ __global__ void __launch_bounds__(Cfg::kThreads)
   }
 }
 
-// Log-sum-exp merge of partition partials: one warp per (sequence, query head)
-// with more than one partition; single-partition sequences were written by
-// the decode kernel. out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.
+// Log-sum-exp merge of partition partials. One CTA (4 warps) per (sequence,
+// query head) with more than one partition; single-partition sequences were
+// written by the decode kernel. All threads find M = max_p m_p and
+// L = sum_p l_p 2^(m_p - M); warp w accumulates partitions p = w, w+4, ...,
+// eight loads in flight per lane; the four partial sums meet in shared memory:
+//   out = sum_p acc_p 2^(m_p - M) / L.
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
     lse_merge_kernel(const DecodeArgs a, int block_size) {
   constexpr int VEC = D / 32;
-  const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (wid >= a.num_seqs * a.num_q_heads) return;
-  const int s = wid / a.num_q_heads;
+  constexpr int UNROLL = 8;
+  __shared__ float red[4];
+  __shared__ float accs[4][D];
+  grid_dependency_wait();  // the decode grid's partials are complete and visible
+  const int row = blockIdx.x;  // s * Hq + h
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int s = row / a.num_q_heads;
   const int ctx = clamp_ctx(a.context_lens[s], a.max_blocks_per_seq * block_size);
   const int np = partitions_of(ctx, block_size, a.partition_blocks);
   if (np <= 1) return;
-  const int64_t base = static_cast<int64_t>(wid) * a.max_partitions;
+  const int64_t base = static_cast<int64_t>(row) * a.max_partitions;
   float M = -INFINITY;
-  for (int p = lane; p < np; p += 32) M = fmaxf(M, a.part_m[base + p]);
+  for (int p = tid; p < np; p += 128) M = fmaxf(M, a.part_m[base + p]);
   M = warp_max(M);
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
   float L = 0.f;
-  for (int p = lane; p < np; p += 32) L += a.part_l[base + p] * fast_exp2(a.part_m[base + p] - M);
+  for (int p = tid; p < np; p += 128) L += a.part_l[base + p] * fast_exp2(a.part_m[base + p] - M);
   L = warp_sum(L);
+  if (lane == 0) red[warp] = L;
   float acc[VEC];
 #pragma unroll
   for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
-  for (int p = 0; p < np; ++p) {
-    const float e = fast_exp2(a.part_m[base + p] - M);
-    const float* src = a.part_acc + (base + p) * D + lane * VEC;
+  const float* src = a.part_acc + base * D + lane * VEC;
+  int p = warp;
+  for (; p + 4 * (UNROLL - 1) < np; p += 4 * UNROLL) {
+    float v[UNROLL][VEC];
+    float e[UNROLL];
 #pragma unroll
-    for (int j = 0; j < VEC; ++j) acc[j] = fmaf(src[j], e, acc[j]);
+    for (int u = 0; u < UNROLL; ++u) {
+      const int pp = p + 4 * u;
+      e[u] = a.part_m[base + pp];
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) v[u][j] = src[static_cast<int64_t>(pp) * D + j];
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const float w = fast_exp2(e[u] - M);
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) acc[j] = fmaf(v[u][j], w, acc[j]);
+    }
   }
-  T* dst = reinterpret_cast<T*>(a.out) + static_cast<int64_t>(wid) * D + lane * VEC;
-  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  for (; p < np; p += 4) {
+    const float w = fast_exp2(a.part_m[base + p] - M);
 #pragma unroll
-  for (int j = 0; j < VEC; ++j) dst[j] = Elt<T>::from_f32(acc[j] * inv);
+    for (int j = 0; j < VEC; ++j) acc[j] = fmaf(src[static_cast<int64_t>(p) * D + j], w, acc[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) accs[warp][lane * VEC + j] = acc[j];
+  __syncthreads();
+  L = red[0] + red[1] + red[2] + red[3];
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  T* dst = reinterpret_cast<T*>(a.out) + static_cast<int64_t>(row) * D;
+  for (int d = tid; d < D; d += 128)
+    dst[d] = Elt<T>::from_f32((accs[0][d] + accs[1][d] + accs[2][d] + accs[3][d]) * inv);
 }
 
 }  // namespace pagedkv

@@ -151,6 +151,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ---- programmatic dependent launch -----------------------------------------------
+// Primary grid: allow the dependent grid to be scheduled early.
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Dependent grid: wait until the primary grid has completed and its memory
+// operations are visible (returns at once when launched without the attribute).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---- scalar math --------------------------------------------------------------
 // 2^x by the hardware approximation (MUFU.EX2); 2^-inf = +0.
 __device__ __forceinline__ float fast_exp2(float x) {

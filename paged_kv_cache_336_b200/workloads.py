@@ -142,7 +142,7 @@ def _prefix_common(name: str, prompt_len: int, tail_max: int, seed: int,
     return Workload(
         name=name, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=bs,
         dtype=BF16, num_blocks=nb,
-        max_blocks_per_seq=-(-(prompt_len + tail_max + 8) // bs),
+        max_blocks_per_seq=-(-(prompt_len + tail_max + 80) // bs),
         context_lens=ctx, free_order=_perm(rng, nb), seed=seed,
         prefill_seqs=prefill, forks=forks, extra_tokens=extra,
         step_seqs=list(range(nseq)), decode_seqs=list(range(nseq)))
