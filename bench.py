@@ -184,7 +184,7 @@ def profiled_traffic(workload: str):
         kv = {}
         with open(path) as f:
             for line in f:
-                if ":" in line:
+                if ":" in line and not line.lstrip().startswith("#"):
                     k, v = line.split(":", 1)
                     kv[k.strip()] = v.strip()
         if kv.get("kernel_source_sha256_16") != kernel_source_hash():
