@@ -105,6 +105,20 @@ def copy_bytes(w, num_pairs: int) -> int:
     return num_pairs * (2 * 2 * block + 16)
 
 
+def reduce_over_ranks(local_ms: float, local_bytes: float, local_tokens: float, device):
+    """Job-wide (time, bytes, tokens): the slowest rank's time, everything
+    else summed. A single process returns its own values."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(local_ms), float(local_bytes), float(local_tokens)
+    t = torch.tensor([float(local_ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    b = torch.tensor([float(local_bytes), float(local_tokens)], device=device, dtype=torch.float64)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(b[0].item()), float(b[1].item())
+
+
 # ---------------------------------------------------------------------------
 # measured peaks, clocks, profile traffic
 
@@ -311,16 +325,7 @@ def run_ours(args, rank, world, device_index):
     decode_ms = sum(a.elapsed_time(b) for a, b in evs)
 
     # max time over ranks, bytes summed over ranks
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-        b = torch.tensor([float(total_bytes), float(args.steps * ds.B)], device=device,
-                         dtype=torch.float64)
-        dist.all_reduce(b, op=dist.ReduceOp.SUM)
-        all_bytes, all_tokens = float(b[0].item()), float(b[1].item())
-    else:
-        ms_max, all_bytes, all_tokens = ms, float(total_bytes), float(args.steps * ds.B)
+    ms_max, all_bytes, all_tokens = reduce_over_ranks(ms, total_bytes, args.steps * ds.B, device)
 
     gbs = all_bytes / (ms_max * 1e-3) / 1e9
     tok_s = all_tokens / (ms_max * 1e-3)
@@ -379,30 +384,26 @@ def run_ours(args, rank, world, device_index):
 
 
 def run_e2e(args, ds, rank, world, device):
-    """Same metric through the public API from pinned host buffers."""
+    """Same metric through the public API from pinned host buffers: one
+    pa_decode_step call per step (host block-manager step, H2D of the step's
+    inputs, copies + append + split decode, D2H of out, stream sync)."""
     import torch
     import torch.distributed as dist
     b = ds.binding
     w = ds.w
     steps = max(3, min(args.e2e_steps, args.steps))
-    B, T = ds.B, ds.T
-    # host-side inputs of every e2e step (pinned)
-    hq = [ds.states[i % len(ds.states)]["q"].cpu().pin_memory() for i in range(min(steps, 8))]
-    hk = [ds.states[i % len(ds.states)]["k_new"].cpu().pin_memory() for i in range(min(steps, 8))]
-    hv = [ds.states[i % len(ds.states)]["v_new"].cpu().pin_memory() for i in range(min(steps, 8))]
-    dq = torch.empty_like(ds.states[0]["q"])
-    dk = torch.empty_like(ds.states[0]["k_new"])
-    dv = torch.empty_like(ds.states[0]["v_new"])
-    dslots = torch.empty(max(T, 1), dtype=torch.int64, device=device)
-    dpairs = torch.empty((max(T, 1), 2), dtype=torch.int64, device=device)
-    dtables = torch.empty((B, w.max_blocks_per_seq), dtype=torch.int32, device=device)
-    dctx = torch.empty(B, dtype=torch.int32, device=device)
-    hslots = torch.empty(max(T, 1), dtype=torch.int64).pin_memory()
-    hpairs = torch.empty((max(T, 1), 2), dtype=torch.int64).pin_memory()
-    htables = torch.empty((B, w.max_blocks_per_seq), dtype=torch.int32).pin_memory()
-    hctx = torch.empty(B, dtype=torch.int32).pin_memory()
-    hout = torch.empty(ds.out.shape, dtype=ds.out.dtype).pin_memory()
-    stream = torch.cuda.current_stream()
+    seqs = np.ascontiguousarray(np.asarray(w.step_seqs or w.decode_seqs, dtype=np.int64))
+    n = int(seqs.shape[0])
+    stepper = b.DecodeStepper(ds.bm, ds.k_pool, ds.v_pool, w.num_q_heads, w.scale, max_seqs=n,
+                              partition_tokens=ds.partition_tokens)
+    ring = min(steps, 8)
+    hq = [ds.states[i % len(ds.states)]["q"][:n].cpu().pin_memory() for i in range(ring)]
+    hk, hv = [], []
+    for i in range(ring):
+        kn, vn = b_new_kv(w, n, i, device)
+        hk.append(kn.cpu().pin_memory())
+        hv.append(vn.cpu().pin_memory())
+    hout = torch.empty(hq[0].shape, dtype=hq[0].dtype).pin_memory()
     h2d = d2h = 0
     total = 0
     if world > 1:
@@ -410,55 +411,24 @@ def run_e2e(args, ds, rank, world, device):
     torch.cuda.synchronize()
     t_start = time.perf_counter()
     for i in range(steps):
-        # host block manager step (C++), then uploads
-        if T:
-            slots, pairs = ds.bm.append_slots_arrays(w.step_seqs)
-            hslots[:T].copy_(torch.from_numpy(slots))
-            npairs = pairs.shape[0]
-            if npairs:
-                hpairs[:npairs].copy_(torch.from_numpy(pairs))
-        else:
-            npairs = 0
-        tables, ctx = ds.bm.export(w.decode_seqs)
-        htables.copy_(torch.from_numpy(tables))
-        hctx.copy_(torch.from_numpy(ctx))
-        j = i % len(hq)
-        dq.copy_(hq[j], non_blocking=True)
-        dk.copy_(hk[j], non_blocking=True)
-        dv.copy_(hv[j], non_blocking=True)
-        dtables.copy_(htables, non_blocking=True)
-        dctx.copy_(hctx, non_blocking=True)
-        step_h2d = dq.numel() * dq.element_size() + 2 * dk.numel() * dk.element_size() + \
-            htables.numel() * 4 + hctx.numel() * 4
-        if T:
-            dslots[:T].copy_(hslots[:T], non_blocking=True)
-            step_h2d += T * 8
-        if npairs:
-            dpairs[:npairs].copy_(hpairs[:npairs], non_blocking=True)
-            b.copy_blocks(ds.k_pool, ds.v_pool, dpairs[:npairs])
-            step_h2d += npairs * 16
-        if T:
-            b.kv_append(dk, dv, dslots[:T], ds.k_pool, ds.v_pool)
-        b.decode_split(dq, ds.k_pool, ds.v_pool, dtables, dctx, w.scale,
-                       partition_tokens=ds.partition_tokens, out=ds.out, workspace=ds.ws)
-        hout.copy_(ds.out, non_blocking=True)
-        stream.synchronize()   # the step's result is on the host
-        h2d += step_h2d
-        d2h += hout.numel() * hout.element_size()
-        total += decode_bytes(w, ctx.astype(np.int64)) + append_bytes(w, T) + copy_bytes(w, npairs)
+        j = i % ring
+        ncow = stepper.step(seqs, hq[j], hk[j], hv[j], hout, synchronize=True)
+        h2d += stepper.h2d_bytes(n, ncow)
+        d2h += stepper.d2h_bytes(n)
+        ctx = stepper.h_ctx[:n].numpy().astype(np.int64)
+        total += decode_bytes(w, ctx) + append_bytes(w, n) + copy_bytes(w, ncow)
     elapsed = time.perf_counter() - t_start
-    if world > 1:
-        t = torch.tensor([elapsed], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
-        bt = torch.tensor([float(total)], device=device, dtype=torch.float64)
-        dist.all_reduce(bt, op=dist.ReduceOp.SUM)
-        total = float(bt.item())
+    elapsed, total, _ = reduce_over_ranks(elapsed, total, steps * n, device)
     return {"value": round(total / elapsed / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d / steps), "d2h_bytes_per_step": int(d2h / steps),
             "steps": steps, "ms_per_step": round(elapsed / steps * 1e3, 4),
-            "path": "python binding -> C ABI; host block manager step + pinned H2D + kernels "
-                    "+ D2H out + stream sync per step"}
+            "path": "pa_decode_step (C ABI) per step: host block manager step + pinned H2D "
+                    "of the step's inputs + copies/append/split decode + D2H out + stream sync"}
+
+
+def b_new_kv(w, n, i, device):
+    from paged_kv_cache_336_b200 import workloads
+    return workloads.draw_new_kv(w, n, step=10_000 + i, device=device)
 
 
 # ---------------------------------------------------------------------------

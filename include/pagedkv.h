@@ -284,6 +284,66 @@ pa_status_t pa_bm_refcount(pa_bm_t bm, int block_id, int* refcount);
 pa_status_t pa_bm_free_queue(pa_bm_t bm, int32_t* out, int capacity, int* n);
 pa_status_t pa_bm_stats(pa_bm_t bm, pa_bm_stats_t* stats);
 
+/* ===========================================================================
+ * pa_decode_step - one whole decode step from host buffers: the block
+ * manager reserves one slot per sequence (copy-on-write where a tail is
+ * shared), the step's inputs are uploaded, the copies, the KV append and the
+ * split decode run, and the output is downloaded. This is call stack A of the
+ * pages' flow in one call: decode appends into the tail block ([Q] How It
+ * Works), shared tails are copied before the write ([G] section 4), attention
+ * walks the block tables ([G] section 3).
+ *
+ * All buffers in pa_step_buffers_t are caller-owned and sized for max_seqs
+ * sequences; the library allocates nothing. Host staging buffers should be
+ * page-locked (cudaHostAlloc / cudaHostRegister) so the copies are
+ * asynchronous. Per call, with n = number of sequences:
+ *   q_host      [n][num_q_heads][head_dim]   (dtype)  query of each sequence
+ *   k_new_host  [n][num_kv_heads][head_dim]  (dtype)  the appended token's K
+ *   v_new_host  [n][num_kv_heads][head_dim]  (dtype)  ... and V
+ *   out_host    [n][num_q_heads][head_dim]   (dtype)  attention output
+ * Sequence i of seq_ids appends one token and is decoded with its new length.
+ * If synchronize is non-zero the call returns after out_host holds the
+ * result; otherwise the caller synchronises `stream` before reading it.
+ * A block-manager failure (PA_ERR_NO_FREE_BLOCKS / PA_ERR_INVALID_ARG)
+ * returns before anything is enqueued, state unchanged. A CUDA error after
+ * the manager step leaves the manager with the step applied.
+ * ========================================================================= */
+typedef struct {
+  /* shape and cache */
+  int max_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks;
+  int max_blocks_per_seq, partition_tokens;
+  float scale;
+  pa_dtype_t dtype;
+  void* k_pool;
+  void* v_pool;
+  void* workspace;          /* pa_decode_split workspace (initialised) */
+  size_t workspace_bytes;
+  /* device staging */
+  void* d_q;                /* [max_seqs][num_q_heads][head_dim] */
+  void* d_k_new;            /* [max_seqs][num_kv_heads][head_dim] */
+  void* d_v_new;
+  void* d_out;              /* [max_seqs][num_q_heads][head_dim] */
+  int64_t* d_slots;         /* [max_seqs] */
+  int64_t* d_pairs;         /* [max_seqs][2] */
+  int32_t* d_tables;        /* [max_seqs][max_blocks_per_seq] */
+  int32_t* d_context_lens;  /* [max_seqs] */
+  /* host staging (page-locked) */
+  int64_t* h_slots;         /* [max_seqs] */
+  int64_t* h_pairs;         /* [max_seqs][2] */
+  int32_t* h_tables;        /* [max_seqs][max_blocks_per_seq] */
+  int32_t* h_context_lens;  /* [max_seqs] */
+} pa_step_buffers_t;
+
+/* Number of host->device and device->host bytes one pa_decode_step call of
+ * n sequences moves when it makes `num_copies` copy-on-write copies. */
+size_t pa_decode_step_h2d_bytes(const pa_step_buffers_t* buf, int n, int num_copies);
+size_t pa_decode_step_d2h_bytes(const pa_step_buffers_t* buf, int n);
+
+pa_status_t pa_decode_step(pa_bm_t bm, const pa_step_buffers_t* buf, const int64_t* seq_ids,
+                           int n, const void* q_host, const void* k_new_host,
+                           const void* v_new_host, void* out_host, int* num_copies,
+                           int synchronize, uint32_t* dev_err, void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -12,6 +12,7 @@ needs it does, and raises ``RuntimeError`` if it has not been built
 
 from .binding import (  # noqa: F401
     BlockManager,
+    DecodeStepper,
     PagedKVError,
     NoFreeBlocksError,
     InvalidArgumentError,

@@ -64,6 +64,19 @@ _I64 = ctypes.c_int64
 _SZ = ctypes.c_size_t
 _F = ctypes.c_float
 
+
+class StepBuffers(ctypes.Structure):
+    """Mirror of pa_step_buffers_t (include/pagedkv.h)."""
+    _fields_ = [
+        ("max_seqs", _I), ("num_q_heads", _I), ("num_kv_heads", _I), ("head_dim", _I),
+        ("block_size", _I), ("num_blocks", _I), ("max_blocks_per_seq", _I),
+        ("partition_tokens", _I), ("scale", _F), ("dtype", _I),
+        ("k_pool", _P), ("v_pool", _P), ("workspace", _P), ("workspace_bytes", _SZ),
+        ("d_q", _P), ("d_k_new", _P), ("d_v_new", _P), ("d_out", _P),
+        ("d_slots", _P), ("d_pairs", _P), ("d_tables", _P), ("d_context_lens", _P),
+        ("h_slots", _P), ("h_pairs", _P), ("h_tables", _P), ("h_context_lens", _P),
+    ]
+
 # name -> (restype, argtypes); mirrors include/pagedkv.h
 _SIGNATURES = {
     "pa_version": (ctypes.c_char_p, []),
@@ -93,6 +106,10 @@ _SIGNATURES = {
     "pa_bm_refcount": (_I, [_P, _I, ctypes.POINTER(_I)]),
     "pa_bm_free_queue": (_I, [_P, _P, _I, ctypes.POINTER(_I)]),
     "pa_bm_stats": (_I, [_P, ctypes.POINTER(_Stats)]),
+    "pa_decode_step_h2d_bytes": (_SZ, [ctypes.POINTER(StepBuffers), _I, _I]),
+    "pa_decode_step_d2h_bytes": (_SZ, [ctypes.POINTER(StepBuffers), _I]),
+    "pa_decode_step": (_I, [_P, ctypes.POINTER(StepBuffers), _P, _I, _P, _P, _P, _P,
+                            ctypes.POINTER(_I), _I, _P, _P]),
 }
 
 
@@ -391,3 +408,71 @@ class BlockManager:
         st = _Stats()
         _check(library().pa_bm_stats(self._h, ctypes.byref(st)))
         return {name: int(getattr(st, name)) for name, _ in _Stats._fields_}
+
+
+# ---------------------------------------------------------------------------
+# One whole decode step from host buffers (pa_decode_step).
+
+class DecodeStepper:
+    """Owns the staging buffers of pa_decode_step for one cache and manager.
+
+    Device staging is torch-allocated once; host staging is page-locked. Each
+    ``step`` call is one C call: manager step, uploads, copies, append, split
+    decode, download (and, by default, stream synchronisation)."""
+
+    def __init__(self, bm: "BlockManager", k_pool, v_pool, num_q_heads: int, scale: float,
+                 max_seqs: int, partition_tokens: int = 512):
+        torch = _torch()
+        _require_cuda(k_pool, v_pool)
+        NB, Hkv, BS, D = k_pool.shape
+        dev = k_pool.device
+        self.bm = bm
+        self.k_pool, self.v_pool = k_pool, v_pool
+        self.dtype = k_pool.dtype
+        mbs = bm.max_blocks_per_seq
+        self.ws = SplitWorkspace(max_seqs, num_q_heads, D, BS, mbs, partition_tokens, dev)
+        self.d_q = torch.empty(max_seqs, num_q_heads, D, dtype=self.dtype, device=dev)
+        self.d_out = torch.empty_like(self.d_q)
+        self.d_k_new = torch.empty(max_seqs, Hkv, D, dtype=self.dtype, device=dev)
+        self.d_v_new = torch.empty_like(self.d_k_new)
+        self.d_slots = torch.empty(max_seqs, dtype=torch.int64, device=dev)
+        self.d_pairs = torch.empty(max_seqs, 2, dtype=torch.int64, device=dev)
+        self.d_tables = torch.empty(max_seqs, mbs, dtype=torch.int32, device=dev)
+        self.d_ctx = torch.empty(max_seqs, dtype=torch.int32, device=dev)
+        self.h_slots = torch.empty(max_seqs, dtype=torch.int64).pin_memory()
+        self.h_pairs = torch.empty(max_seqs, 2, dtype=torch.int64).pin_memory()
+        self.h_tables = torch.empty(max_seqs, mbs, dtype=torch.int32).pin_memory()
+        self.h_ctx = torch.empty(max_seqs, dtype=torch.int32).pin_memory()
+        b = StepBuffers()
+        b.max_seqs, b.num_q_heads, b.num_kv_heads, b.head_dim = max_seqs, num_q_heads, Hkv, D
+        b.block_size, b.num_blocks, b.max_blocks_per_seq = BS, NB, mbs
+        b.partition_tokens, b.scale, b.dtype = partition_tokens, float(scale), _dtype_code(k_pool)
+        b.k_pool, b.v_pool = _ptr(k_pool), _ptr(v_pool)
+        b.workspace, b.workspace_bytes = self.ws.ptr, self.ws.nbytes
+        b.d_q, b.d_k_new, b.d_v_new, b.d_out = (_ptr(self.d_q), _ptr(self.d_k_new),
+                                                _ptr(self.d_v_new), _ptr(self.d_out))
+        b.d_slots, b.d_pairs = _ptr(self.d_slots), _ptr(self.d_pairs)
+        b.d_tables, b.d_context_lens = _ptr(self.d_tables), _ptr(self.d_ctx)
+        b.h_slots, b.h_pairs = _ptr(self.h_slots), _ptr(self.h_pairs)
+        b.h_tables, b.h_context_lens = _ptr(self.h_tables), _ptr(self.h_ctx)
+        self.buffers = b
+
+    def h2d_bytes(self, n: int, num_copies: int) -> int:
+        return int(library().pa_decode_step_h2d_bytes(ctypes.byref(self.buffers), n, num_copies))
+
+    def d2h_bytes(self, n: int) -> int:
+        return int(library().pa_decode_step_d2h_bytes(ctypes.byref(self.buffers), n))
+
+    def step(self, seq_ids, q_host, k_new_host, v_new_host, out_host, synchronize: bool = True,
+             dev_err=None, stream=None) -> int:
+        """Runs one step; returns the number of copy-on-write copies it made.
+        ``seq_ids`` is a contiguous int64 numpy array; the host tensors are CPU
+        tensors (pinned for asynchronous copies) of the shapes in pagedkv.h."""
+        n = int(seq_ids.shape[0])
+        ncow = _I()
+        _check(library().pa_decode_step(
+            self.bm._h, ctypes.byref(self.buffers), seq_ids.ctypes.data, n, _ptr(q_host),
+            _ptr(k_new_host), _ptr(v_new_host), _ptr(out_host), ctypes.byref(ncow),
+            1 if synchronize else 0, _ptr(dev_err), _stream_ptr(stream)))
+        return int(ncow.value)
+

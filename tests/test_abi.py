@@ -237,3 +237,37 @@ def test_block_manager_rejects_bad_arguments():
         bm.append_slots([0, 0])
     with pytest.raises(PagedKVError):
         bm.refcount_of(99)
+
+
+def test_decode_step_rejects_before_touching_the_device():
+    import ctypes
+    lib = binding.library()
+    bm = LibBM(2, 4, 2, [0, 1])
+    bm.allocate(7, 8)                       # two full blocks: the next append needs a third
+    b = binding.StepBuffers()
+    b.max_seqs, b.num_q_heads, b.num_kv_heads, b.head_dim = 2, 2, 2, 64
+    b.block_size, b.num_blocks, b.max_blocks_per_seq = 4, 2, 2
+    b.partition_tokens, b.scale, b.dtype = 4, 0.1, binding.PA_BF16
+    for name in ("k_pool", "v_pool", "workspace", "d_q", "d_k_new", "d_v_new", "d_out",
+                 "d_slots", "d_pairs", "d_tables", "d_context_lens"):
+        setattr(b, name, FAKE)
+    host = {n: np.zeros(16, dtype=np.int64) for n in ("h_slots", "h_pairs", "h_tables", "h_context_lens")}
+    for n, a in host.items():
+        setattr(b, n, a.ctypes.data)
+    ids = np.array([7], dtype=np.int64)
+    ncow = ctypes.c_int(-1)
+    args = (FAKE, FAKE, FAKE, FAKE, ctypes.byref(ncow), 1, None, None)
+    # more sequences than the staging holds
+    assert lib.pa_decode_step(bm._h, ctypes.byref(b), np.zeros(3, np.int64).ctypes.data, 3, *args) == \
+        binding.PA_ERR_INVALID_ARG
+    # block manager failure: reported, nothing changed, nothing enqueued
+    before = (bm.block_table(7), bm.context_len(7), bm.free_queue_list())
+    assert lib.pa_decode_step(bm._h, ctypes.byref(b), ids.ctypes.data, 1, *args) == \
+        binding.PA_ERR_INVALID_ARG          # at max_blocks_per_seq
+    assert (bm.block_table(7), bm.context_len(7), bm.free_queue_list()) == before
+    bm2 = LibBM(2, 4, 4, [0, 1])
+    bm2.allocate(7, 8)
+    assert lib.pa_decode_step(bm2._h, ctypes.byref(b), ids.ctypes.data, 1, *args) == \
+        binding.PA_ERR_NO_FREE_BLOCKS
+    assert bm2.context_len(7) == 8 and bm2.free_queue_list() == []
+    assert ctypes.sizeof(binding.StepBuffers) == 168
