@@ -19,6 +19,7 @@ namespace pagedkv {
 namespace {
 
 constexpr size_t kWorkspaceHeader = 256;
+constexpr int64_t kDeepContextTokens = 32768;
 constexpr int kMaxSplitSeqs = 4096;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -140,7 +141,10 @@ pa_status_t validate_and_pick(const DecodeReq& r, DecodeInstance* inst) {
   if (r.dtype == PA_F32) {
     found = find_decode_f32(r.head_dim, r.block_size, group, inst);
   } else if (group <= 16) {
-    found = find_decode_bf16_mma(r.head_dim, r.block_size, inst);
+    // Tables that can hold 32k tokens or more mark long-context batches: the
+    // deeper, narrower CTA shape streams them faster.
+    const bool deep = static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size >= kDeepContextTokens;
+    found = find_decode_bf16_mma(r.head_dim, r.block_size, deep, inst);
   }
   if (!found)
     return fail(PA_ERR_UNSUPPORTED,

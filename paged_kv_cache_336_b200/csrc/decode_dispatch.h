@@ -18,6 +18,7 @@ struct DecodeInstance {
 
 // Each returns false when (head_dim, block_size, group) has no instance.
 bool find_decode_f32(int head_dim, int block_size, int group, DecodeInstance* out);
-bool find_decode_bf16_mma(int head_dim, int block_size, DecodeInstance* out);
+// deep: the CTA shape for long contexts (see decode_inst_bf16.cu).
+bool find_decode_bf16_mma(int head_dim, int block_size, bool deep, DecodeInstance* out);
 
 }  // namespace pagedkv

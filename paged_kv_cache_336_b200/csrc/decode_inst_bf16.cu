@@ -1,12 +1,21 @@
 // bf16 instances of the paged decode kernel (tensor-core path, groups 1..16).
+//
+// Two CTA shapes per (block size, head_dim), chosen by the host:
+//  * wide: 4 warps x 2 ring stages (64 KB of ring at head_dim 128; three CTAs
+//    and 12 warps per SM). Best measured for contexts up to a few thousand
+//    tokens: MHA batch 64 and GQA batch 256 stream at ~96.7% of the measured
+//    HBM copy peak against ~92% for 4 x 3.
+//  * deep: 2 warps x 3 stages (48 KB; four CTAs per SM). Best measured for
+//    131072-token contexts in 512-token partitions (96.9% against 91.7% for
+//    wide): each warp walks more units of an item per fill and drain.
 #include "decode_dispatch.h"
 #include "decode_kernel.cuh"
 
 namespace pagedkv {
 
-template <int BS, int D, int G>
+template <int BS, int D, int W, int NS>
 static DecodeInstance make_bf16(const char* name) {
-  using Cfg = DecodeCfg<__nv_bfloat16, BS, D, G>;
+  using Cfg = DecodeCfg<__nv_bfloat16, BS, D, 0, W, NS>;
   DecodeInstance r;
   r.kernel = reinterpret_cast<const void*>(&paged_decode_kernel<Cfg>);
   r.merge = reinterpret_cast<const void*>(&lse_merge_kernel<__nv_bfloat16, D>);
@@ -17,13 +26,24 @@ static DecodeInstance make_bf16(const char* name) {
   return r;
 }
 
-bool find_decode_bf16_mma(int head_dim, int block_size, DecodeInstance* out) {
-  if (block_size == 16 && head_dim == 64) { *out = make_bf16<16, 64, 0>("mma_bf16"); return true; }
-  if (block_size == 16 && head_dim == 128) { *out = make_bf16<16, 128, 0>("mma_bf16"); return true; }
-  if (block_size == 16 && head_dim == 256) { *out = make_bf16<16, 256, 0>("mma_bf16"); return true; }
-  if (block_size == 32 && head_dim == 64) { *out = make_bf16<32, 64, 0>("mma_bf16"); return true; }
-  if (block_size == 32 && head_dim == 128) { *out = make_bf16<32, 128, 0>("mma_bf16"); return true; }
-  if (block_size == 32 && head_dim == 256) { *out = make_bf16<32, 256, 0>("mma_bf16"); return true; }
+template <int BS, int D>
+static void pick(bool deep, DecodeInstance* out) {
+  if constexpr (D == 256) {
+    // 16 KB stages: the default shape (4 warps x 2 stages) for both.
+    *out = make_bf16<BS, D, 0, 0>("mma_bf16");
+  } else {
+    if (deep) *out = make_bf16<BS, D, 2, 3>("mma_bf16_deep");
+    else *out = make_bf16<BS, D, 4, 2>("mma_bf16_wide");
+  }
+}
+
+bool find_decode_bf16_mma(int head_dim, int block_size, bool deep, DecodeInstance* out) {
+  if (block_size == 16 && head_dim == 64) { pick<16, 64>(deep, out); return true; }
+  if (block_size == 16 && head_dim == 128) { pick<16, 128>(deep, out); return true; }
+  if (block_size == 16 && head_dim == 256) { pick<16, 256>(deep, out); return true; }
+  if (block_size == 32 && head_dim == 64) { pick<32, 64>(deep, out); return true; }
+  if (block_size == 32 && head_dim == 128) { pick<32, 128>(deep, out); return true; }
+  if (block_size == 32 && head_dim == 256) { pick<32, 256>(deep, out); return true; }
   return false;
 }
 

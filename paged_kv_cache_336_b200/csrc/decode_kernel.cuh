@@ -94,8 +94,9 @@ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 // G_ > 0: CUDA-core path with compile-time group; G_ == 0: tensor-core path,
-// runtime group 1..16 (bf16 only).
-template <typename T, int BS_, int D_, int G_>
+// runtime group 1..16 (bf16 only). W_ / NS_: warps per CTA and ring stages
+// per warp, 0 = the default below.
+template <typename T, int BS_, int D_, int G_, int W_ = 0, int NS_ = 0>
 struct DecodeCfg {
   using Elt = T;
   static constexpr int BS = BS_;
@@ -110,11 +111,13 @@ struct DecodeCfg {
   static_assert(BS % UR == 0, "block_size must be a multiple of 16");
   using Geo = TileGeom<T, UR, D>;
   static constexpr int kStageBytes = 2 * Geo::kTileBytes;
-  // Four warps unless two stages each would not fit beside the prefix array.
-  static constexpr int W = (4 * 2 * kStageBytes <= 160 * 1024) ? 4 : 2;
+  // Warps per CTA and ring stages per warp. Defaults: four warps (two when
+  // two stages each would not fit beside the prefix array) and as many
+  // stages, 2..4, as fit in 96 KB, so two CTAs share an SM.
+  static constexpr int W = W_ > 0 ? W_ : ((4 * 2 * kStageBytes <= 160 * 1024) ? 4 : 2);
   static constexpr int kThreads = 32 * W;
   static_assert(W % UPB == 0, "warps must cover whole blocks");
-  static constexpr int NS = cmin(4, cmax(2, 98304 / (W * kStageBytes)));
+  static constexpr int NS = NS_ > 0 ? NS_ : cmin(4, cmax(2, 98304 / (W * kStageBytes)));
   static constexpr int kRingBytes = W * NS * kStageBytes;
   static constexpr int kRowsMax = kMma ? 16 : G;
   static constexpr int kMergeBytes = W * kRowsMax * (D + 2) * 4;

@@ -71,6 +71,24 @@ def test_decode_matches_oracle_small(kind, dtype, Hq, Hkv, D, bs):
     assert torch.all(out[0] == 0)  # empty context gives zeros
 
 
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("G", [1, 8])
+def test_long_table_shape_matches_oracle(bs, G):
+    """Tables sized for >= 32k tokens select the deep CTA shape (2 warps x 3
+    stages); small contexts keep the comparison cheap."""
+    w = workloads.random_small(88 + G + bs, num_seqs=6, num_q_heads=2 * G, num_kv_heads=2,
+                               head_dim=128, block_size=bs, dtype=workloads.BF16,
+                               max_ctx=40 * bs, fixed_lens=[0, 1, 40 * bs, 17])
+    w.max_blocks_per_seq = 32768 // bs + 3
+    bm, k_pool, v_pool = setup(w)
+    q = workloads.draw_queries(w, 6, device="cuda")
+    bt, ctx, tables, ctx_np = device_tables(bm, list(range(6)))
+    want = _full_oracle(q, k_pool, v_pool, tables, ctx_np, w.scale)
+    for kind in ("decode", "split"):
+        out = _run_decode(kind, q, k_pool, v_pool, bt, ctx, w.scale, partition=3 * bs)
+        check_close(to_f64(out), want, w.dtype, f"deep {kind}")
+
+
 @pytest.mark.parametrize("dtype,G", [(workloads.F32, 1), (workloads.BF16, 1), (workloads.BF16, 8)])
 @pytest.mark.parametrize("partition_blocks", [1, 2, 3, 5, 64])
 def test_split_any_partition_equals_oracle(dtype, G, partition_blocks):
