@@ -95,6 +95,15 @@ def decode_bytes(w, ctx: np.ndarray) -> int:
     return kv + qo + bt
 
 
+def unique_decode_bytes(w, ctx: np.ndarray, skip: np.ndarray, group_blocks) -> int:
+    """Bytes a shared-prefix decode must read at least: each group's shared
+    blocks once, every sequence's own tokens, plus q, out, tables, lengths."""
+    per_token = w.num_kv_heads * w.head_dim * w.elt_bytes * 2
+    kv = (int(np.sum(group_blocks)) * w.block_size +
+          int(np.sum(ctx - skip * w.block_size))) * per_token
+    return kv + decode_bytes(w, ctx) - int(np.sum(ctx)) * per_token
+
+
 def append_bytes(w, num_tokens: int) -> int:
     per = num_tokens * w.num_kv_heads * w.head_dim * w.elt_bytes * 2
     return 2 * per + 8 * num_tokens   # read new K/V, write them, read slots
@@ -214,13 +223,14 @@ def profiled_traffic(workload: str):
 class DeviceStep:
     """Device-resident inputs of R consecutive decode steps, cycled."""
 
-    def __init__(self, w, states: int, partition_tokens: int, device, whole: bool = False):
+    def __init__(self, w, states: int, partition_tokens: int, device, mode: str = "split"):
         import torch
         from paged_kv_cache_336_b200 import binding, workloads
         self.torch, self.binding = torch, binding
         self.w = w
         self.partition_tokens = partition_tokens
-        self.whole = whole
+        self.mode = mode
+        self.whole = mode == "whole"
         self.bm = binding.BlockManager(w.num_blocks, w.block_size, w.max_blocks_per_seq,
                                        w.free_order)
         for s in w.prefill_seqs:
@@ -252,16 +262,32 @@ class DeviceStep:
             st["ctx_np"] = ctx.astype(np.int64)
             st["n_pairs"] = int(pairs.shape[0])
             st["decode_bytes"] = decode_bytes(w, st["ctx_np"])
+            st["unique_bytes"] = st["decode_bytes"]
+            if mode == "shared_prefix":
+                offs, members, gblocks = self.bm.prefix_groups(w.decode_seqs)
+                st["groups"] = (offs, members, gblocks)
+                skip = np.zeros(len(w.decode_seqs), dtype=np.int64)
+                for g in range(len(gblocks)):
+                    skip[members[offs[g]:offs[g + 1]]] = gblocks[g]
+                st["unique_bytes"] = unique_decode_bytes(w, st["ctx_np"], skip, gblocks)
             st["step_bytes"] = (st["decode_bytes"] + append_bytes(w, T) + copy_bytes(w, st["n_pairs"]))
             self.states.append(st)
         self.out = torch.empty_like(self.states[0]["q"])
-        self.ws = binding.SplitWorkspace(B, w.num_q_heads, w.head_dim, w.block_size,
-                                         w.max_blocks_per_seq, partition_tokens, device)
+        if mode == "shared_prefix":
+            self.ws = binding.shared_prefix_workspace(B, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                                      w.block_size, w.max_blocks_per_seq,
+                                                      partition_tokens, device)
+        else:
+            self.ws = binding.SplitWorkspace(B, w.num_q_heads, w.head_dim, w.block_size,
+                                             w.max_blocks_per_seq, partition_tokens, device)
         pb = partition_tokens // w.block_size
-        self.merge_launched = (-(-w.max_blocks_per_seq // pb) > 1) and not whole
+        self.merge_launched = (-(-w.max_blocks_per_seq // pb) > 1 or mode == "shared_prefix") \
+            and mode != "whole"
 
     def launches(self, st) -> int:
-        return (1 if st["n_pairs"] else 0) + (1 if self.T else 0) + 1 + (1 if self.merge_launched else 0)
+        prefix = 1 if (self.mode == "shared_prefix" and len(st["groups"][2])) else 0
+        return ((1 if st["n_pairs"] else 0) + (1 if self.T else 0) + 1 + prefix +
+                (1 if self.merge_launched else 0))
 
     def run(self, i, ev=None):
         st = self.states[i % len(self.states)]
@@ -275,6 +301,11 @@ class DeviceStep:
         if self.whole:
             b.decode(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"], self.w.scale,
                      out=self.out)
+        elif self.mode == "shared_prefix":
+            b.decode_shared_prefix(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"],
+                                   self.w.scale, st["groups"],
+                                   partition_tokens=self.partition_tokens, out=self.out,
+                                   workspace=self.ws)
         else:
             b.decode_split(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"],
                            self.w.scale, partition_tokens=self.partition_tokens, out=self.out,
@@ -293,7 +324,7 @@ def run_ours(args, rank, world, device_index):
     torch.cuda.set_device(device)
     w = make_workload(args.workload, rank, args.batch)
     R = max(1, min(args.states, args.steps + args.warmup)) if args.workload != "prefix_cow" else 1
-    ds = DeviceStep(w, R, args.partition_tokens, device, whole=args.decode_mode == "whole")
+    ds = DeviceStep(w, R, args.partition_tokens, device, mode=args.decode_mode)
 
     for i in range(args.warmup):
         ds.run(i)
@@ -310,11 +341,13 @@ def run_ours(args, rank, world, device_index):
     t0.record()
     total_bytes = 0
     decode_bytes_sum = 0
+    unique_bytes_sum = 0
     launches = 0
     for i in range(args.steps):
         st = ds.run(args.warmup + i, evs[i])
         total_bytes += st["step_bytes"]
         decode_bytes_sum += st["decode_bytes"]
+        unique_bytes_sum += st["unique_bytes"]
         launches += ds.launches(st)
     t1.record()
     torch.cuda.synchronize()
@@ -330,6 +363,7 @@ def run_ours(args, rank, world, device_index):
     gbs = all_bytes / (ms_max * 1e-3) / 1e9
     tok_s = all_tokens / (ms_max * 1e-3)
     decode_gbs = decode_bytes_sum / (decode_ms * 1e-3) / 1e9
+    unique_gbs = unique_bytes_sum / (decode_ms * 1e-3) / 1e9
     peak, peak_kind = hbm_peak()
 
     # ---- end to end through the public API (host buffers, pinned) ----------------
@@ -337,6 +371,11 @@ def run_ours(args, rank, world, device_index):
 
     result = None
     if rank == 0:
+        kernel_label = {
+            "split": "pa_decode_split (paged_decode_kernel + lse_merge_kernel)",
+            "whole": "pa_decode (paged_decode_kernel)",
+            "shared_prefix": "pa_decode_shared_prefix (prefix_decode_kernel + paged_decode_kernel "
+                             "+ lse_merge_kernel)"}[args.decode_mode]
         result = {
             "metric": METRIC,
             "value": round(gbs, 2),
@@ -356,8 +395,7 @@ def run_ours(args, rank, world, device_index):
                 "context_lens": ("uniform [1, 2048]" if w.name == "mha" else "see workload"),
                 "mean_context": round(float(np.mean([s["ctx_np"].mean() for s in ds.states])), 1),
                 "partition_tokens": args.partition_tokens,
-                "step": "bm slots/CoW (host, precomputed) + copy_blocks + kv_append + "
-                        "decode_split (partition + LSE merge)",
+                "step": "bm slots/CoW (host, precomputed) + copy_blocks + kv_append + " + kernel_label,
                 "decode_states_cycled": len(ds.states),
                 "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                 "parallelism": f"independent batch per GPU x{world}",
@@ -365,7 +403,7 @@ def run_ours(args, rank, world, device_index):
             "decode_tokens_per_s": round(tok_s, 1),
             "roofline": {
                 "bound": "hbm",
-                "kernel": "pa_decode_split (paged_decode_kernel + lse_merge_kernel)",
+                "kernel": kernel_label,
                 "achieved": round(decode_gbs, 2),
                 "peak": peak,
                 "peak_kind": peak_kind,
@@ -375,6 +413,11 @@ def run_ours(args, rank, world, device_index):
                 "traffic": profiled_traffic(args.workload),
                 "algorithmic_bytes_per_launch": int(decode_bytes_sum / args.steps),
                 "avg_launch_us": round(decode_ms / args.steps * 1e3, 2),
+                # bytes the call must read at least (shared prefixes once); equal to the
+                # algorithmic bytes unless blocks are shared
+                "unique_bytes_per_launch": int(unique_bytes_sum / args.steps),
+                "unique_achieved": round(unique_gbs, 2),
+                "unique_frac": round(unique_gbs / peak, 4),
             },
             "e2e": e2e,
             "gpu_launches": launches,
@@ -524,9 +567,10 @@ def main(argv=None):
     ap.add_argument("--workload", default="mha",
                     choices=["mha", "gqa", "prefix", "prefix_cow", "long16", "long32", "tiny"])
     ap.add_argument("--partition-tokens", type=int, default=512)
-    ap.add_argument("--decode-mode", choices=["split", "whole"], default="split",
+    ap.add_argument("--decode-mode", choices=["split", "whole", "shared_prefix"], default="split",
                     help="split: pa_decode_split (persistent, partitions + merge); "
-                         "whole: pa_decode (one CTA per sequence and KV head)")
+                         "whole: pa_decode (one CTA per sequence and KV head); "
+                         "shared_prefix: pa_decode_shared_prefix (shared prompt blocks read once)")
     ap.add_argument("--states", type=int, default=64, help="distinct decode steps cycled")
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--batch", type=int, default=None,

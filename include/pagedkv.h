@@ -180,6 +180,60 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
                                    void* stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_decode_shared_prefix - the same result as pa_decode, reading each
+ * shared prefix once. Sequences that share their first blocks (prefix
+ * sharing and parallel sampling, [G] section 4; [Q] Share Without Mutating
+ * State) are given as groups: group g lists positions group_members
+ * [group_offsets[g] .. group_offsets[g+1]) of the batch, which all hold the
+ * same physical blocks in table entries 0 .. group_blocks[g]-1, every one of
+ * them full (pa_bm_prefix_groups produces exactly this). A prefix kernel
+ * streams each group's shared blocks once per KV head for all of the group's
+ * query rows (members x heads per KV head, on tensor cores); the split kernel
+ * then covers each sequence's remaining blocks; the log-sum-exp merge joins
+ * the two ([G] section 3: any blockwise order gives the contiguous result).
+ * Sequences in no group are decoded as by pa_decode_split.
+ *
+ * Group arrays are HOST memory, read during the call; the library copies what
+ * the kernels need into the workspace. bf16 only. workspace: at least
+ * pa_decode_shared_prefix_workspace_size(...) bytes, 256-byte aligned,
+ * initialised once with pa_decode_split_workspace_init (the same contract as
+ * pa_decode_split).
+ * ------------------------------------------------------------------------- */
+size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                              int head_dim, int block_size,
+                                              int max_blocks_per_seq, int partition_tokens);
+
+pa_status_t pa_decode_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
+                                    const int32_t* block_tables, const int32_t* context_lens,
+                                    int num_seqs, int num_q_heads, int num_kv_heads,
+                                    int head_dim, int block_size, int num_blocks,
+                                    int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                                    int partition_tokens, int num_groups,
+                                    const int32_t* group_offsets, const int32_t* group_members,
+                                    const int32_t* group_blocks, void* workspace,
+                                    size_t workspace_bytes, void* out, uint32_t* dev_err,
+                                    void* stream);
+
+/* ---------------------------------------------------------------------------
+ * pa_decode_split_window - sliding-window decode: as pa_decode_split, but
+ * each query attends only to the last `window` tokens of its sequence
+ * (tokens max(0, ctx - window) .. ctx - 1; window >= 1). The block walk
+ * starts at the window's first block and the tokens before the window in
+ * that block are masked, so table entries before it are never read and may
+ * be -1 (pa_bm_release_before). Sliding-window attention is named beside
+ * paged attention as a KV-cache optimisation ([K] Core Facts). Same
+ * workspace and contract as pa_decode_split.
+ * ------------------------------------------------------------------------- */
+pa_status_t pa_decode_split_window(const void* q, const void* k_pool, const void* v_pool,
+                                   const int32_t* block_tables, const int32_t* context_lens,
+                                   int num_seqs, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int block_size, int num_blocks,
+                                   int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                                   int partition_tokens, int window, void* workspace,
+                                   size_t workspace_bytes, void* out, uint32_t* dev_err,
+                                   void* stream);
+
+/* ---------------------------------------------------------------------------
  * pa_kv_append - decode-step write of new tokens' keys and values into their
  * slots ([Q], Map Logical to Physical Blocks: decode appends into the partly
  * filled tail block; [G] section 4 step 3: the write proceeds on the private
@@ -267,6 +321,15 @@ pa_status_t pa_bm_can_append(pa_bm_t bm, const int64_t* seq_ids, int n, int* ok)
 /* Finish a sequence: counts drop by one; blocks reaching zero are reclaimed. */
 pa_status_t pa_bm_free(pa_bm_t bm, int64_t seq_id);
 
+/* Sliding window: drop the sequence's references to blocks whose tokens all
+ * lie before first_token (blocks 0 .. first_token/block_size - 1). Their table
+ * entries become -1, so logical positions stay where they were; blocks whose
+ * count reaches zero are reclaimed (back of the free queue, ascending).
+ * *num_reclaimed (may be NULL) gets how many. Decode with a window of
+ * ctx - first_token tokens or fewer never reads the released entries. */
+pa_status_t pa_bm_release_before(pa_bm_t bm, int64_t seq_id, int64_t first_token,
+                                 int* num_reclaimed);
+
 /* Copy one sequence's block table into row[0..row_capacity); *n_blocks gets
  * its length (PA_ERR_INVALID_ARG if row_capacity is too small). */
 pa_status_t pa_bm_block_table(pa_bm_t bm, int64_t seq_id, int32_t* row,
@@ -278,6 +341,19 @@ pa_status_t pa_bm_context_len(pa_bm_t bm, int64_t seq_id, int64_t* context_len);
  * for pa_decode. */
 pa_status_t pa_bm_export(pa_bm_t bm, const int64_t* seq_ids, int n, int32_t* tables,
                          int32_t* context_lens, int32_t pad_value);
+
+/* Shared-prefix groups of a batch, for pa_decode_shared_prefix. Sequences
+ * whose block tables start with the same physical blocks (created by fork,
+ * [G] section 4 step 1) form a group; its shared length is the longest
+ * common table prefix, counted in blocks that are full for every member
+ * (a partly filled shared tail is left to each sequence). Only groups of at
+ * least two sequences sharing at least min_shared_blocks blocks are kept.
+ * Outputs (host memory, capacities n+1 / n / n): group_offsets[g] ..
+ * group_offsets[g+1] index group_members, which lists positions in seq_ids
+ * (in seq_ids order); group_blocks[g] is the shared block count. */
+pa_status_t pa_bm_prefix_groups(pa_bm_t bm, const int64_t* seq_ids, int n, int min_shared_blocks,
+                                int32_t* group_offsets, int32_t* group_members,
+                                int32_t* group_blocks, int* num_groups);
 
 pa_status_t pa_bm_refcount(pa_bm_t bm, int block_id, int* refcount);
 /* Free queue front to back into out[0..capacity); *n gets its length. */

@@ -13,9 +13,10 @@ Modules
     Decode attention over a block-paged KV cache, written as its definition:
     gather each sequence's keys and values through its block table, then
     softmax(scale * K q) V in float64, two-pass (max, then exp/sum).
-    Also the partitioned form (per-partition max/sum/accumulator and a
-    log-sum-exp merge), the KV-append scatter and the block copy, as plain
-    array assignments.
+    Also the sliding-window form (the last ``window`` tokens only), the
+    partitioned form (per-partition max/sum/accumulator and a log-sum-exp
+    merge), the KV-append scatter and the block copy, as plain array
+    assignments.
 ``block_manager``
     Reference host block manager: FIFO free queue, reference counts,
     per-sequence block tables, copy-on-write on append, all-or-nothing
@@ -39,6 +40,7 @@ from .paged_attention import (  # noqa: F401
     gather_sequence,
     paged_decode,
     paged_decode_one,
+    paged_decode_window,
     partitioned_decode_one,
     kv_append,
     copy_blocks,

@@ -89,8 +89,11 @@ class BlockManager:
     def stats(self) -> dict:
         used = sum(1 for rc in self.refcount if rc > 0)
         shared = sum(1 for rc in self.refcount if rc > 1)
-        logical_slots = sum(len(t) for t in self.tables.values()) * self.block_size
-        tokens = sum(self.context.values())
+        # resident blocks and tokens (a released window prefix no longer counts)
+        resident = {s: sum(1 for b in t if b >= 0) for s, t in self.tables.items()}
+        logical_slots = sum(resident.values()) * self.block_size
+        tokens = sum(ctx - (len(self.tables[s]) - resident[s]) * self.block_size
+                     for s, ctx in self.context.items())
         return {
             "num_blocks": self.num_blocks,
             "free_blocks": len(self.free_queue),
@@ -128,7 +131,8 @@ class BlockManager:
             raise InvalidArgument(f"sequence {child} already exists")
         table = list(self.tables[parent])
         for b in table:
-            self.refcount[b] += 1
+            if b >= 0:
+                self.refcount[b] += 1
         self.tables[child] = table
         self.context[child] = self.context[parent]
 
@@ -191,11 +195,36 @@ class BlockManager:
         self.context[seq] = ctx + 1
         return result
 
+    def release_before(self, seq: int, first_token: int) -> list[int]:
+        """Sliding window: drop this sequence's references to blocks whose
+        tokens all lie before ``first_token``; their table entries become -1
+        (logical positions are kept). Returns the blocks reclaimed (count 0),
+        which go to the back of the free queue in ascending order."""
+        self._require(seq)
+        if first_token < 0:
+            raise InvalidArgument("first_token must be >= 0")
+        table = self.tables[seq]
+        n_out = min(first_token // self.block_size, len(table))
+        reclaimed = []
+        for i in range(n_out):
+            b = table[i]
+            if b < 0:
+                continue
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                reclaimed.append(b)
+            table[i] = -1
+        for b in sorted(reclaimed):
+            self.free_queue.append(b)
+        return sorted(reclaimed)
+
     def free(self, seq: int) -> None:
         """Drop a finished sequence; reclaim blocks whose count reaches zero."""
         self._require(seq)
         reclaimed = []
         for b in self.tables[seq]:
+            if b < 0:
+                continue
             self.refcount[b] -= 1
             if self.refcount[b] == 0:
                 reclaimed.append(b)

@@ -52,6 +52,9 @@ def gather_sequence(pool, block_table_row, context_len: int, kv_head: int) -> np
         logical_block = t // block_size
         offset = t % block_size
         physical_block = int(block_table_row[logical_block])
+        if physical_block < 0:   # released before a sliding window; never attended to
+            rows[t, :] = np.nan
+            continue
         rows[t, :] = pool[physical_block, kv_head, offset, :]
     return rows
 
@@ -106,6 +109,33 @@ def paged_decode(q, k_pool, v_pool, block_tables, context_lens, scale: float) ->
         for h in range(num_q_heads):
             out[s, h] = paged_decode_one(q, k_pool, v_pool, block_tables, context_lens,
                                          scale, s, h)
+    return out
+
+
+def paged_decode_window(q, k_pool, v_pool, block_tables, context_lens, scale: float,
+                        window: int) -> np.ndarray:
+    """Sliding-window decode: each query attends to the last ``window`` tokens
+    of its sequence only (all of them when the sequence is shorter). The
+    pages name sliding-window attention as a KV-cache optimisation beside
+    paged attention ("PagedAttention" knowledge page, Core Facts); the window
+    is the plain reading: tokens max(0, ctx - window) .. ctx - 1.
+
+    Returns float64 ``[num_seqs, num_q_heads, head_dim]``.
+    """
+    if window <= 0:
+        raise ValueError("window must be positive")
+    q = np.asarray(q)
+    num_seqs, num_q_heads, head_dim = q.shape
+    num_kv_heads = np.asarray(k_pool).shape[1]
+    group = _group(num_q_heads, num_kv_heads)
+    out = np.zeros((num_seqs, num_q_heads, head_dim), dtype=np.float64)
+    for s in range(num_seqs):
+        ctx = int(context_lens[s])
+        lo = max(0, ctx - window)
+        for h in range(num_q_heads):
+            K = gather_sequence(k_pool, block_tables[s], ctx, h // group)[lo:]
+            V = gather_sequence(v_pool, block_tables[s], ctx, h // group)[lo:]
+            out[s, h] = attention_definition(q[s, h], K, V, scale)
     return out
 
 

@@ -18,6 +18,8 @@ from .binding import (  # noqa: F401
     InvalidArgumentError,
     decode,
     decode_split,
+    decode_split_window,
+    decode_shared_prefix,
     decode_split_workspace_size,
     kv_append,
     copy_blocks,

@@ -89,6 +89,13 @@ _SIGNATURES = {
                              _P, _P, _P]),
     "pa_decode_split_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                                     _P, _P, _P]),
+    "pa_decode_shared_prefix_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "pa_decode_shared_prefix": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
+                                     _I, _P, _P, _P, _P, _SZ, _P, _P, _P]),
+    "pa_bm_prefix_groups": (_I, [_P, _P, _I, _I, _P, _P, _P, ctypes.POINTER(_I)]),
+    "pa_bm_release_before": (_I, [_P, _I64, _I64, ctypes.POINTER(_I)]),
+    "pa_decode_split_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
+                                    _I, _P, _SZ, _P, _P, _P]),
     "pa_kv_append": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "pa_copy_blocks": (_I, [_P, _P, _P, _I, _SZ, _I, _P, _P]),
     "pa_bm_create": (_I, [_I, _I, _I, _P, ctypes.POINTER(_P)]),
@@ -249,6 +256,68 @@ def decode_split(q, k_pool, v_pool, block_tables, context_lens, scale: float,
     return out
 
 
+def decode_split_window(q, k_pool, v_pool, block_tables, context_lens, scale: float,
+                        window: int, partition_tokens: int = 512, out=None,
+                        workspace: SplitWorkspace | None = None, dev_err=None, stream=None):
+    """pa_decode_split_window: attention over the last ``window`` tokens only."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty_like(q)
+    B, Hq, D, NB, Hkv, BS, MBS = _decode_common(q, k_pool, v_pool, block_tables, context_lens, out)
+    if workspace is None:
+        workspace = SplitWorkspace(B, Hq, D, BS, MBS, partition_tokens, q.device, stream)
+    _check(library().pa_decode_split_window(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv,
+        D, BS, NB, MBS, float(scale), _dtype_code(q), int(partition_tokens), int(window),
+        workspace.ptr, workspace.nbytes, _ptr(out), _ptr(dev_err), _stream_ptr(stream)))
+    return out
+
+
+class Workspace:
+    """Caller-owned, 256-byte aligned device workspace, zeroed once (the
+    contract of pa_decode_split_workspace_init)."""
+
+    def __init__(self, nbytes: int, device=None, stream=None):
+        torch = _torch()
+        self.nbytes = int(nbytes)
+        self.buffer = torch.empty(self.nbytes + 256, dtype=torch.uint8,
+                                  device=device or torch.device("cuda"))
+        self.ptr = (self.buffer.data_ptr() + 255) & ~255
+        _check(library().pa_decode_split_workspace_init(self.ptr, self.nbytes, _stream_ptr(stream)))
+
+
+def shared_prefix_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, partition_tokens, device=None) -> Workspace:
+    n = library().pa_decode_shared_prefix_workspace_size(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+        partition_tokens)
+    if n == 0:
+        raise InvalidArgumentError(PA_ERR_INVALID_ARG, "bad workspace size arguments")
+    return Workspace(n, device)
+
+
+def decode_shared_prefix(q, k_pool, v_pool, block_tables, context_lens, scale: float, groups,
+                         partition_tokens: int = 512, out=None, workspace: Workspace | None = None,
+                         dev_err=None, stream=None):
+    """pa_decode_shared_prefix. ``groups`` = (offsets, members, blocks) as host
+    int32 arrays, e.g. from BlockManager.prefix_groups()."""
+    import numpy as np
+    torch = _torch()
+    if out is None:
+        out = torch.empty_like(q)
+    B, Hq, D, NB, Hkv, BS, MBS = _decode_common(q, k_pool, v_pool, block_tables, context_lens, out)
+    offs, members, blocks = (np.ascontiguousarray(np.asarray(x, dtype=np.int32)) for x in groups)
+    if workspace is None:
+        workspace = shared_prefix_workspace(B, Hq, Hkv, D, BS, MBS, partition_tokens, q.device)
+    _check(library().pa_decode_shared_prefix(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv,
+        D, BS, NB, MBS, float(scale), _dtype_code(q), int(partition_tokens), int(blocks.shape[0]),
+        offs.ctypes.data, members.ctypes.data if members.size else None,
+        blocks.ctypes.data if blocks.size else None, workspace.ptr, workspace.nbytes, _ptr(out),
+        _ptr(dev_err), _stream_ptr(stream)))
+    return out
+
+
 def kv_append(k_new, v_new, slot_mapping, k_pool, v_pool, dev_err=None, stream=None):
     """pa_kv_append: pool[slot // bs, :, slot % bs, :] = new[t] for K and V."""
     torch = _torch()
@@ -388,6 +457,28 @@ class BlockManager:
         _check(library().pa_bm_export(self._h, ids.ctypes.data, n, tables.ctypes.data,
                                       ctx.ctypes.data, int(pad_value)))
         return tables, ctx
+
+    def release_before(self, seq: int, first_token: int) -> int:
+        """pa_bm_release_before; returns the number of blocks reclaimed."""
+        k = _I()
+        _check(library().pa_bm_release_before(self._h, int(seq), int(first_token), ctypes.byref(k)))
+        return int(k.value)
+
+    def prefix_groups(self, seqs, min_shared_blocks: int = 1):
+        """pa_bm_prefix_groups: (offsets [g+1], members [m], blocks [g]) int32
+        numpy arrays; members are positions in ``seqs``."""
+        import numpy as np
+        ids = np.ascontiguousarray(np.asarray(seqs, dtype=np.int64))
+        n = ids.shape[0]
+        offs = np.zeros(n + 1, dtype=np.int32)
+        members = np.zeros(max(n, 1), dtype=np.int32)
+        blocks = np.zeros(max(n, 1), dtype=np.int32)
+        k = _I()
+        _check(library().pa_bm_prefix_groups(self._h, ids.ctypes.data, n, int(min_shared_blocks),
+                                             offs.ctypes.data, members.ctypes.data,
+                                             blocks.ctypes.data, ctypes.byref(k)))
+        g = k.value
+        return offs[:g + 1].copy(), members[:offs[g]].copy(), blocks[:g].copy()
 
     def refcount_of(self, block: int) -> int:
         rc = _I()

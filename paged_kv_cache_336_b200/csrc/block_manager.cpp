@@ -15,6 +15,7 @@
 // in ascending id order; a batched step processes sequences in the order given
 // and is all-or-nothing.
 #include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <deque>
 #include <new>
@@ -187,7 +188,8 @@ pa_status_t pa_bm_fork(pa_bm_t bm, int64_t parent_id, int64_t child_id) {
   if (!find_seq(bm, parent_id, &p)) return fail(PA_ERR_INVALID_ARG, "unknown parent %lld", (long long)parent_id);
   if (bm->seqs.count(child_id)) return fail(PA_ERR_INVALID_ARG, "sequence %lld exists", (long long)child_id);
   pa_bm::Seq c = *p;  // copy before emplace may rehash
-  for (int32_t b : c.table) bm->refcount[b] += 1;
+  for (int32_t b : c.table)
+    if (b >= 0) bm->refcount[b] += 1;  // released entries (-1) hold nothing
   bm->seqs.emplace(child_id, std::move(c));
   return ok();
 }
@@ -246,12 +248,34 @@ pa_status_t pa_bm_free(pa_bm_t bm, int64_t seq_id) {
   if (it == bm->seqs.end()) return fail(PA_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq_id);
   std::vector<int32_t> reclaimed;
   for (int32_t b : it->second.table) {
+    if (b < 0) continue;
     bm->refcount[b] -= 1;
     if (bm->refcount[b] == 0) reclaimed.push_back(b);
   }
   std::sort(reclaimed.begin(), reclaimed.end());
   for (int32_t b : reclaimed) bm->free_queue.push_back(b);
   bm->seqs.erase(it);
+  return ok();
+}
+
+pa_status_t pa_bm_release_before(pa_bm_t bm, int64_t seq_id, int64_t first_token, int* num_reclaimed) {
+  if (bm == nullptr) return fail(PA_ERR_INVALID_ARG, "bm is NULL");
+  if (first_token < 0) return fail(PA_ERR_INVALID_ARG, "first_token < 0");
+  pa_bm::Seq* s = nullptr;
+  if (!find_seq(bm, seq_id, &s)) return fail(PA_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq_id);
+  const int64_t n_out = std::min<int64_t>(first_token / bm->block_size,
+                                          static_cast<int64_t>(s->table.size()));
+  std::vector<int32_t> reclaimed;
+  for (int64_t i = 0; i < n_out; ++i) {
+    const int32_t b = s->table[i];
+    if (b < 0) continue;
+    bm->refcount[b] -= 1;
+    if (bm->refcount[b] == 0) reclaimed.push_back(b);
+    s->table[i] = -1;
+  }
+  std::sort(reclaimed.begin(), reclaimed.end());
+  for (int32_t b : reclaimed) bm->free_queue.push_back(b);
+  if (num_reclaimed) *num_reclaimed = static_cast<int>(reclaimed.size());
   return ok();
 }
 
@@ -298,6 +322,58 @@ pa_status_t pa_bm_export(pa_bm_t bm, const int64_t* seq_ids, int n, int32_t* tab
   return ok();
 }
 
+pa_status_t pa_bm_prefix_groups(pa_bm_t bm, const int64_t* seq_ids, int n, int min_shared_blocks,
+                                int32_t* group_offsets, int32_t* group_members,
+                                int32_t* group_blocks, int* num_groups) {
+  if (bm == nullptr || num_groups == nullptr || n < 0 ||
+      (n > 0 && (seq_ids == nullptr || group_offsets == nullptr || group_members == nullptr ||
+                 group_blocks == nullptr)))
+    return fail(PA_ERR_INVALID_ARG, "NULL argument");
+  std::vector<const pa_bm::Seq*> seqs(n);
+  for (int i = 0; i < n; ++i) {
+    pa_bm::Seq* s = nullptr;
+    if (!find_seq(bm, seq_ids[i], &s))
+      return fail(PA_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq_ids[i]);
+    seqs[i] = s;
+  }
+  // Bucket by first physical block, keeping batch order inside a bucket.
+  std::unordered_map<int32_t, std::vector<int32_t>> buckets;
+  std::vector<int32_t> first_seen;
+  for (int i = 0; i < n; ++i) {
+    if (seqs[i]->table.empty() || seqs[i]->table[0] < 0) continue;  // none, or released
+    const int32_t b0 = seqs[i]->table[0];
+    auto it = buckets.find(b0);
+    if (it == buckets.end()) {
+      buckets.emplace(b0, std::vector<int32_t>{i});
+      first_seen.push_back(b0);
+    } else {
+      it->second.push_back(i);
+    }
+  }
+  int groups = 0, written = 0;
+  group_offsets[0] = 0;
+  for (int32_t b0 : first_seen) {
+    const std::vector<int32_t>& mem = buckets[b0];
+    if (mem.size() < 2) continue;
+    // shared = longest common table prefix, limited to blocks full for all
+    int64_t shared = INT64_MAX;
+    for (int32_t i : mem) shared = std::min<int64_t>(shared, seqs[i]->ctx / bm->block_size);
+    const std::vector<int32_t>& t0 = seqs[mem[0]]->table;
+    for (int32_t i : mem) {
+      const std::vector<int32_t>& t = seqs[i]->table;
+      int64_t k = 0;
+      while (k < shared && t[k] == t0[k]) ++k;
+      shared = k;
+    }
+    if (shared < std::max(1, min_shared_blocks)) continue;
+    for (int32_t i : mem) group_members[written++] = i;
+    group_blocks[groups] = static_cast<int32_t>(shared);
+    group_offsets[++groups] = written;
+  }
+  *num_groups = groups;
+  return ok();
+}
+
 pa_status_t pa_bm_refcount(pa_bm_t bm, int block_id, int* refcount) {
   if (bm == nullptr || refcount == nullptr) return fail(PA_ERR_INVALID_ARG, "NULL argument");
   if (block_id < 0 || block_id >= bm->num_blocks) return fail(PA_ERR_INVALID_ARG, "block %d out of range", block_id);
@@ -325,9 +401,12 @@ pa_status_t pa_bm_stats(pa_bm_t bm, pa_bm_stats_t* st) {
     r.shared_blocks += c > 1;
   }
   r.num_seqs = static_cast<int64_t>(bm->seqs.size());
-  for (const auto& kv : bm->seqs) {
-    r.logical_tokens += kv.second.ctx;
-    r.logical_slots += static_cast<int64_t>(kv.second.table.size()) * bm->block_size;
+  for (const auto& kv : bm->seqs) {  // resident blocks and tokens only
+    int64_t resident = 0;
+    for (int32_t b : kv.second.table) resident += b >= 0;
+    const int64_t released = static_cast<int64_t>(kv.second.table.size()) - resident;
+    r.logical_tokens += kv.second.ctx - released * bm->block_size;
+    r.logical_slots += resident * bm->block_size;
   }
   r.tail_waste_slots = r.logical_slots - r.logical_tokens;
   r.cow_copies = bm->cow_copies;

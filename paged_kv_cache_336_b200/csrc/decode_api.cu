@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -14,6 +15,7 @@
 #include "decode_dispatch.h"
 #include "decode_kernel.cuh"
 #include "pa_internal.h"
+#include "prefix_kernel.cuh"
 
 namespace pagedkv {
 namespace {
@@ -265,8 +267,19 @@ SplitLayout split_layout(int num_seqs, int num_q_heads, int head_dim, int block_
   return L;
 }
 
+// Shared-prefix decode hands the split kernel per-sequence skip/base arrays
+// and its own partial-array layout.
+struct SplitExtras {
+  const int32_t* seq_skip_blocks = nullptr;
+  const int32_t* seq_part_base = nullptr;
+  size_t m_off = 0, l_off = 0, acc_off = 0, total = 0;
+  int pmax = 0;
+  bool after_prefix_kernel = false;  // launched right after the prefix kernel
+  int window = 0;                    // sliding window (0 = none)
+};
+
 pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, void* workspace,
-                       size_t workspace_bytes) {
+                       size_t workspace_bytes, const SplitExtras* extras = nullptr) {
   DecodeInstance inst;
   pa_status_t st = validate_and_pick(r, &inst);
   if (st != PA_OK) return st;
@@ -299,8 +312,19 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
       return fail(PA_ERR_UNSUPPORTED, "pa_decode_split takes at most %d sequences", kMaxSplitSeqs);
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
       return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
-    const SplitLayout L = split_layout(r.num_seqs, r.num_q_heads, r.head_dim, r.block_size,
-                                       r.max_blocks_per_seq, partition_tokens);
+    SplitLayout L = split_layout(r.num_seqs, r.num_q_heads, r.head_dim, r.block_size,
+                                 r.max_blocks_per_seq, partition_tokens);
+    if (extras != nullptr && extras->window > 0) {
+      a.window = extras->window;
+    } else if (extras != nullptr) {
+      L.m_off = extras->m_off;
+      L.l_off = extras->l_off;
+      L.acc_off = extras->acc_off;
+      L.total = extras->total;
+      L.pmax = extras->pmax;
+      a.seq_skip_blocks = extras->seq_skip_blocks;
+      a.seq_part_base = extras->seq_part_base;
+    }
     if (workspace_bytes < L.total)
       return fail(PA_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", workspace_bytes, L.total);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -341,9 +365,27 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
   if (st != PA_OK) return st;
 
   void* args[] = {&tmk, &tmv, &a};
-  cudaError_t err = cudaLaunchKernel(inst.kernel, grid, dim3(inst.threads), args, smem, r.stream);
+  cudaError_t err;
+  if (extras != nullptr && extras->after_prefix_kernel) {
+    // Runs alongside the shared-prefix kernel (disjoint partial slots) and
+    // waits for it at exit, so the merge that depends on this grid sees both.
+    a.wait_prior_at_exit = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(inst.threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = r.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelExC(&cfg, inst.kernel, args);
+  } else {
+    err = cudaLaunchKernel(inst.kernel, grid, dim3(inst.threads), args, smem, r.stream);
+  }
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
-  if (split && a.max_partitions > 1) {
+  if (split && (a.max_partitions > 1 || a.seq_part_base != nullptr)) {
     // The merge grid is a programmatic dependent of the decode grid: it may be
     // scheduled before the decode grid ends and waits on the device
     // (griddepcontrol.wait) until the partials are complete and visible.
@@ -363,6 +405,179 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
     if (err != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(err));
   }
   return launch_error("decode");
+}
+
+// ---- shared-prefix decode ------------------------------------------------------------
+// Workspace: [0,256) header | skip int32 [B] | part_base int32 [B] |
+// members int32 [B] | items PrefixItem [B*Hkv*kMaxPrefixParts] |
+// m, l float [B][Hq][pmax] | acc float [B][Hq][pmax][D], where
+// pmax = kMaxPrefixParts + ceil(max_blocks_per_seq / partition blocks) + 1.
+constexpr int kMaxPrefixParts = 16;
+constexpr int kPrefixRows = 64;  // query rows per prefix CTA (4 warps x 16)
+
+struct PrefixLayout {
+  size_t skip_off, base_off, members_off, items_off;
+  SplitExtras ex;
+  size_t max_items;
+};
+
+PrefixLayout prefix_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                           int block_size, int max_blocks_per_seq, int partition_tokens) {
+  PrefixLayout L{};
+  const int pb = partition_tokens / block_size;
+  L.ex.pmax = kMaxPrefixParts + (max_blocks_per_seq + pb - 1) / pb + 1;
+  const size_t B = static_cast<size_t>(num_seqs);
+  L.max_items = B * static_cast<size_t>(num_kv_heads) * kMaxPrefixParts;
+  L.skip_off = kWorkspaceHeader;
+  L.base_off = L.skip_off + align256(B * 4);
+  L.members_off = L.base_off + align256(B * 4);
+  L.items_off = L.members_off + align256(B * 4);
+  const size_t rows = B * num_q_heads * L.ex.pmax;
+  L.ex.m_off = L.items_off + align256(L.max_items * sizeof(PrefixItem));
+  L.ex.l_off = L.ex.m_off + align256(rows * 4);
+  L.ex.acc_off = L.ex.l_off + align256(rows * 4);
+  L.ex.total = L.ex.acc_off + align256(rows * static_cast<size_t>(head_dim) * 4);
+  return L;
+}
+
+pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_groups,
+                              const int32_t* offs, const int32_t* members, const int32_t* blocks,
+                              void* workspace, size_t workspace_bytes) {
+  DecodeInstance inst;
+  pa_status_t st = validate_and_pick(r, &inst);
+  if (st != PA_OK) return st;
+  if (r.dtype != PA_BF16) return fail(PA_ERR_UNSUPPORTED, "pa_decode_shared_prefix is bf16 only");
+  PrefixInstance pinst;
+  if (!find_prefix_bf16(r.head_dim, r.block_size, &pinst))
+    return fail(PA_ERR_UNSUPPORTED, "no shared-prefix kernel for head_dim=%d block_size=%d",
+                r.head_dim, r.block_size);
+  if (partition_tokens <= 0 || partition_tokens % r.block_size != 0)
+    return fail(PA_ERR_INVALID_ARG, "partition_tokens (%d) must be a positive multiple of block_size",
+                partition_tokens);
+  if (r.num_seqs > kMaxSplitSeqs)
+    return fail(PA_ERR_UNSUPPORTED, "at most %d sequences", kMaxSplitSeqs);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  const int G = r.num_q_heads / r.num_kv_heads;
+  const int B = r.num_seqs;
+  if (num_groups < 0 || (num_groups > 0 && (offs == nullptr || members == nullptr || blocks == nullptr)))
+    return fail(PA_ERR_INVALID_ARG, "bad group arrays");
+  const PrefixLayout L = prefix_layout(B, r.num_q_heads, r.num_kv_heads, r.head_dim, r.block_size,
+                                       r.max_blocks_per_seq, partition_tokens);
+  if (workspace_bytes < L.ex.total)
+    return fail(PA_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", workspace_bytes, L.ex.total);
+  if (B == 0) return ok();
+
+  thread_local std::vector<int32_t> skip, base, mem;
+  thread_local std::vector<PrefixItem> items;
+  thread_local std::vector<char> seen;
+  skip.assign(B, 0);
+  base.assign(B, 0);
+  seen.assign(B, 0);
+  mem.clear();
+  items.clear();
+  // groups: validate, and find the prefix partition size
+  int64_t total_blocks = 0;
+  int max_blocks = 0;
+  bool many_chunks = false;
+  if (num_groups > 0 && offs[0] != 0) return fail(PA_ERR_INVALID_ARG, "group_offsets[0] must be 0");
+  for (int g = 0; g < num_groups; ++g) {
+    const int b0 = offs[g], b1 = offs[g + 1];
+    if (b1 < b0 || b1 > B) return fail(PA_ERR_INVALID_ARG, "group_offsets not increasing within [0, %d]", B);
+    if (blocks[g] < 1 || blocks[g] > r.max_blocks_per_seq)
+      return fail(PA_ERR_INVALID_ARG, "group_blocks[%d] = %d out of range", g, blocks[g]);
+    for (int i = b0; i < b1; ++i) {
+      const int m = members[i];
+      if (m < 0 || m >= B || seen[m]) return fail(PA_ERR_INVALID_ARG, "group member %d invalid or repeated", m);
+      seen[m] = 1;
+    }
+    const int chunks = ((b1 - b0) * G + kPrefixRows - 1) / kPrefixRows;
+    many_chunks = many_chunks || chunks > 1;
+    total_blocks += static_cast<int64_t>(blocks[g]) * chunks * r.num_kv_heads;
+    max_blocks = std::max(max_blocks, blocks[g]);
+  }
+  DeviceInfo dinfo;
+  st = device_info(&dinfo);
+  if (st != PA_OK) return st;
+  // Partition so that there are about three items per SM (one wave at three
+  // CTAs per SM), at most kMaxPrefixParts per group, and at least four blocks
+  // each; fewer partitions mean fewer partials for the merge.
+  int pbp = static_cast<int>((total_blocks + 3LL * dinfo.sms - 1) / (3LL * dinfo.sms));
+  pbp = std::max(pbp, (max_blocks + kMaxPrefixParts - 1) / kMaxPrefixParts);
+  pbp = std::max(pbp, 4);
+  const int per_chunk = std::max(1, kPrefixRows / G);
+  for (int g = 0; g < num_groups; ++g) {
+    const int b0 = offs[g], b1 = offs[g + 1];
+    if (b1 - b0 == 0) continue;
+    const int nparts = (blocks[g] + pbp - 1) / pbp;
+    const int first = static_cast<int>(mem.size());
+    for (int i = b0; i < b1; ++i) {
+      skip[members[i]] = blocks[g];
+      base[members[i]] = nparts;
+      mem.push_back(members[i]);
+    }
+    for (int c = first; c < first + (b1 - b0); c += per_chunk) {
+      const int cnt = std::min(per_chunk, first + (b1 - b0) - c);
+      for (int h = 0; h < r.num_kv_heads; ++h)
+        for (int p = 0; p < nparts; ++p)
+          items.push_back(PrefixItem{members[b0], c, cnt, p * pbp, std::min(blocks[g], (p + 1) * pbp), h, p, 0});
+    }
+  }
+  if (items.size() > L.max_items) return fail(PA_ERR_INVALID_ARG, "too many prefix items");
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaError_t err;
+  if ((err = cudaMemcpyAsync(ws + L.skip_off, skip.data(), B * 4, cudaMemcpyHostToDevice, r.stream)) != cudaSuccess ||
+      (err = cudaMemcpyAsync(ws + L.base_off, base.data(), B * 4, cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
+    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
+  if (!mem.empty() &&
+      (err = cudaMemcpyAsync(ws + L.members_off, mem.data(), mem.size() * 4, cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
+    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
+  if (!items.empty() &&
+      (err = cudaMemcpyAsync(ws + L.items_off, items.data(), items.size() * sizeof(PrefixItem),
+                             cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
+    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
+
+  SplitExtras ex = L.ex;
+  ex.seq_skip_blocks = reinterpret_cast<const int32_t*>(ws + L.skip_off);
+  ex.seq_part_base = reinterpret_cast<const int32_t*>(ws + L.base_off);
+
+  if (!items.empty()) {
+    st = prepare_kernel(pinst.kernel, pinst.smem);
+    if (st != PA_OK) return st;
+    const int rows = r.num_blocks * r.num_kv_heads * r.block_size;
+    CUtensorMap tmk, tmv;
+    st = pool_tensor_map(r.k_pool, rows, r.head_dim, r.block_size, r.dtype, &tmk);
+    if (st != PA_OK) return st;
+    st = pool_tensor_map(r.v_pool, rows, r.head_dim, r.block_size, r.dtype, &tmv);
+    if (st != PA_OK) return st;
+    PrefixArgs pa{};
+    pa.d.q = r.q;
+    pa.d.block_tables = r.block_tables;
+    pa.d.context_lens = r.context_lens;
+    pa.d.part_m = reinterpret_cast<float*>(ws + ex.m_off);
+    pa.d.part_l = reinterpret_cast<float*>(ws + ex.l_off);
+    pa.d.part_acc = reinterpret_cast<float*>(ws + ex.acc_off);
+    pa.d.dev_err = r.dev_err;
+    pa.d.num_seqs = B;
+    pa.d.num_q_heads = r.num_q_heads;
+    pa.d.num_kv_heads = r.num_kv_heads;
+    pa.d.group = G;
+    pa.d.num_blocks = r.num_blocks;
+    pa.d.max_blocks_per_seq = r.max_blocks_per_seq;
+    pa.d.max_partitions = ex.pmax;
+    pa.d.scale_log2 = r.scale * 1.4426950408889634f;
+    // Tiles re-read by several row chunks stay in L2; otherwise read once.
+    pa.d.l2_hint = many_chunks ? 2 : 1;
+    pa.items = reinterpret_cast<const PrefixItem*>(ws + L.items_off);
+    pa.members = reinterpret_cast<const int32_t*>(ws + L.members_off);
+    void* args[] = {&tmk, &tmv, &pa};
+    err = cudaLaunchKernel(pinst.kernel, dim3(static_cast<unsigned>(items.size())), dim3(pinst.threads),
+                           args, pinst.smem, r.stream);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(err));
+    ex.after_prefix_kernel = true;
+  }
+  return run_decode(r, true, partition_tokens, workspace, workspace_bytes, &ex);
 }
 
 // ---- scratch for pa_decode_split_static ------------------------------------------
@@ -481,6 +696,50 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
   cudaError_t err = cudaMemsetAsync(scratch, 0, layout.zero_bytes, r.stream);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "clearing static scratch: %s", cudaGetErrorString(err));
   return run_decode(r, true, partition_tokens, scratch, kStaticScratchBytes);
+}
+
+size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                              int head_dim, int block_size,
+                                              int max_blocks_per_seq, int partition_tokens) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_blocks_per_seq <= 0 || partition_tokens <= 0 || partition_tokens % block_size != 0)
+    return 0;
+  return prefix_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                       max_blocks_per_seq, partition_tokens)
+      .ex.total;
+}
+
+pa_status_t pa_decode_shared_prefix(const void* q, const void* k_pool, const void* v_pool,
+                                    const int32_t* block_tables, const int32_t* context_lens,
+                                    int num_seqs, int num_q_heads, int num_kv_heads,
+                                    int head_dim, int block_size, int num_blocks,
+                                    int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                                    int partition_tokens, int num_groups,
+                                    const int32_t* group_offsets, const int32_t* group_members,
+                                    const int32_t* group_blocks, void* workspace,
+                                    size_t workspace_bytes, void* out, uint32_t* dev_err,
+                                    void* stream) {
+  DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+              head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
+              static_cast<cudaStream_t>(stream)};
+  return run_shared_prefix(r, partition_tokens, num_groups, group_offsets, group_members,
+                           group_blocks, workspace, workspace_bytes);
+}
+
+pa_status_t pa_decode_split_window(const void* q, const void* k_pool, const void* v_pool,
+                                   const int32_t* block_tables, const int32_t* context_lens,
+                                   int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                   int block_size, int num_blocks, int max_blocks_per_seq,
+                                   float scale, pa_dtype_t dtype, int partition_tokens, int window,
+                                   void* workspace, size_t workspace_bytes, void* out,
+                                   uint32_t* dev_err, void* stream) {
+  if (window < 1) return fail(PA_ERR_INVALID_ARG, "window must be >= 1");
+  DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+              head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
+              static_cast<cudaStream_t>(stream)};
+  SplitExtras ex;
+  ex.window = window;
+  return run_decode(r, true, partition_tokens, workspace, workspace_bytes, &ex);
 }
 
 }  // extern "C"

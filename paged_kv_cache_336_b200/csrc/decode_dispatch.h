@@ -21,4 +21,13 @@ bool find_decode_f32(int head_dim, int block_size, int group, DecodeInstance* ou
 // deep: the CTA shape for long contexts (see decode_inst_bf16.cu).
 bool find_decode_bf16_mma(int head_dim, int block_size, bool deep, DecodeInstance* out);
 
+struct PrefixInstance {
+  const void* kernel = nullptr;  // prefix_decode_kernel<PrefixCfg<BS, D>>
+  int threads = 0;
+  int smem = 0;
+};
+
+// Shared-prefix pass kernels (bf16); false when (head_dim, block_size) has none.
+bool find_prefix_bf16(int head_dim, int block_size, PrefixInstance* out);
+
 }  // namespace pagedkv

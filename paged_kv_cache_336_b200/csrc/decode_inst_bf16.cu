@@ -10,6 +10,7 @@
 //    wide): each warp walks more units of an item per fill and drain.
 #include "decode_dispatch.h"
 #include "decode_kernel.cuh"
+#include "prefix_kernel.cuh"
 
 namespace pagedkv {
 
@@ -44,6 +45,24 @@ bool find_decode_bf16_mma(int head_dim, int block_size, bool deep, DecodeInstanc
   if (block_size == 32 && head_dim == 64) { pick<32, 64>(deep, out); return true; }
   if (block_size == 32 && head_dim == 128) { pick<32, 128>(deep, out); return true; }
   if (block_size == 32 && head_dim == 256) { pick<32, 256>(deep, out); return true; }
+  return false;
+}
+
+template <int BS, int D>
+static PrefixInstance make_prefix() {
+  using Cfg = PrefixCfg<BS, D>;
+  PrefixInstance r;
+  r.kernel = reinterpret_cast<const void*>(&prefix_decode_kernel<Cfg>);
+  r.threads = Cfg::kThreads;
+  r.smem = Cfg::kSmem;
+  return r;
+}
+
+bool find_prefix_bf16(int head_dim, int block_size, PrefixInstance* out) {
+  if (block_size == 16 && head_dim == 64) { *out = make_prefix<16, 64>(); return true; }
+  if (block_size == 16 && head_dim == 128) { *out = make_prefix<16, 128>(); return true; }
+  if (block_size == 32 && head_dim == 64) { *out = make_prefix<32, 64>(); return true; }
+  if (block_size == 32 && head_dim == 128) { *out = make_prefix<32, 128>(); return true; }
   return false;
 }
 

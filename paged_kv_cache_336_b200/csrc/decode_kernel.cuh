@@ -57,6 +57,16 @@ struct DecodeArgs {
   float* part_l;      // [B][Hq][PMAX], running sum of 2^(logit - m)
   float* part_acc;    // [B][Hq][PMAX][D], unnormalised accumulators
   uint32_t* counters; // [0] ticket, [1] finished CTAs (persistent mode)
+  // Shared-prefix decode (nullable otherwise): blocks of each sequence
+  // already covered by its group's prefix pass, and the number of partial
+  // slots that pass filled before this kernel's partitions.
+  const int32_t* seq_skip_blocks;
+  const int32_t* seq_part_base;
+  // Launched as a programmatic dependent of an independent grid whose
+  // results the following merge also reads: wait for it before exiting.
+  int wait_prior_at_exit;
+  // Sliding window (0 = none): attend to tokens max(0, ctx - window) .. ctx-1.
+  int window;
   uint32_t* dev_err;
   int num_seqs;
   int num_q_heads;
@@ -184,7 +194,10 @@ struct SimtWarp {
     }
   }
 
-  __device__ __forceinline__ void block(const uint8_t* kt, uint8_t* vt, int nvalid, int lane) {
+  // Tokens nfirst <= t < nvalid of the unit take part (nfirst > 0 only in the
+  // first unit of a sliding window).
+  __device__ __forceinline__ void block(const uint8_t* kt, uint8_t* vt, int nfirst, int nvalid,
+                                        int lane) {
     const int byte_off = lane * VEC * Geo::kElt;
     const int my_token = (BS == 16) ? (lane >> 1) : lane;
     const bool counts = (BS == 32) || ((lane & 1) == 0);
@@ -201,7 +214,7 @@ struct SimtWarp {
         v[t] = d;
       }
       transpose_reduce<BS>(v, lane);
-      const float s = (my_token < nvalid) ? v[0] : -INFINITY;
+      const float s = (my_token >= nfirst && my_token < nvalid) ? v[0] : -INFINITY;
       const float m_new = fmaxf(m[h], warp_max(s));
       const float alpha = fast_exp2(m[h] - m_new);
       const float p = fast_exp2(s - m_new);
@@ -211,7 +224,7 @@ struct SimtWarp {
       for (int j = 0; j < VEC; ++j) acc[h][j] *= alpha;
 #pragma unroll
       for (int t = 0; t < BS; ++t) {
-        if (t < nvalid) {  // warp-uniform; rows past the context may hold anything
+        if (t >= nfirst && t < nvalid) {  // warp-uniform; rows outside may hold anything
           const float pt = __shfl_sync(0xffffffffu, p, (BS == 16) ? 2 * t : t);
           float vf[VEC];
           load_vec_f32<T, VEC>(reinterpret_cast<const T*>(vt + Geo::offset(t, byte_off)), vf);
@@ -257,15 +270,23 @@ struct MmaWarp {
   __device__ __forceinline__ void begin(const __nv_bfloat16* q_group, int group, float scale,
                                         int lane) {
     const int g = lane >> 2;
+    begin_rows(q_group + g * D, q_group + (g + 8) * D, g < group, g + 8 < group, scale, lane);
+  }
+
+  // Query rows g and g+8 of this warp's 16-row tile come from row0 / row1
+  // (each head_dim contiguous bf16); an invalid row contributes zeros.
+  __device__ __forceinline__ void begin_rows(const __nv_bfloat16* row0, const __nv_bfloat16* row1,
+                                             bool valid0, bool valid1, float scale, int lane) {
     const int t4 = lane & 3;
-    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(q_group);
+    const uint32_t* r0 = reinterpret_cast<const uint32_t*>(row0);
+    const uint32_t* r1 = reinterpret_cast<const uint32_t*>(row1);
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       const int c0 = ks * 16 + 2 * t4;
-      qa[ks][0] = (g < group) ? q32[(g * D + c0) >> 1] : 0u;
-      qa[ks][1] = (g + 8 < group) ? q32[((g + 8) * D + c0) >> 1] : 0u;
-      qa[ks][2] = (g < group) ? q32[(g * D + c0 + 8) >> 1] : 0u;
-      qa[ks][3] = (g + 8 < group) ? q32[((g + 8) * D + c0 + 8) >> 1] : 0u;
+      qa[ks][0] = valid0 ? r0[c0 >> 1] : 0u;
+      qa[ks][1] = valid1 ? r1[c0 >> 1] : 0u;
+      qa[ks][2] = valid0 ? r0[(c0 + 8) >> 1] : 0u;
+      qa[ks][3] = valid1 ? r1[(c0 + 8) >> 1] : 0u;
     }
 #pragma unroll
     for (int n = 0; n < ND; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
@@ -274,36 +295,53 @@ struct MmaWarp {
     scale_log2 = scale;
   }
 
-  __device__ __forceinline__ void block(const uint8_t* kt, uint8_t* vt, int nvalid, int lane) {
+  __device__ __forceinline__ void block(const uint8_t* kt, uint8_t* vt, int nfirst, int nvalid,
+                                        int lane) {
+    const uint8_t* kts[1] = {kt};
+    uint8_t* vts[1] = {vt};
+    block_units<1>(kts, vts, nfirst, nvalid, lane);
+  }
+
+  // U consecutive 16-token units (tiles kts[u], vts[u]) in one online-softmax
+  // step: the U*2 independent S tiles give the tensor pipe more to overlap
+  // and the max/sum shuffles are paid once per U*16 tokens. Tokens
+  // nfirst <= t < nvalid of the span (counted from its first token) take
+  // part; the caller guarantees at least one.
+  template <int U>
+  __device__ __forceinline__ void block_units(const uint8_t* const (&kts)[U], uint8_t* const (&vts)[U],
+                                              int nfirst, int nvalid, int lane) {
     const int t4 = lane & 3;
     const int mj = lane >> 3;  // which 8x8 matrix this lane addresses
     const int mr = lane & 7;   // which row of it
-    const uint32_t kbase = smem_addr(kt);
-    const uint32_t vbase = smem_addr(vt);
+    constexpr int NTU = NT * U;
 
-    float s[NT][4];
+    float s[NTU][4];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+    for (int n = 0; n < NTU; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
-      for (int sub = 0; sub < BS / 16; ++sub) {
-        const int tok = sub * 16 + (mj >> 1) * 8 + mr;
-        const int dim = ks * 16 + (mj & 1) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4(kbase + Geo::offset(tok, dim * 2), b0, b1, b2, b3);
-        mma_bf16_16816(s[2 * sub], qa[ks], b0, b1);
-        mma_bf16_16816(s[2 * sub + 1], qa[ks], b2, b3);
+      for (int u = 0; u < U; ++u) {
+        const uint32_t kbase = smem_addr(kts[u]);
+#pragma unroll
+        for (int sub = 0; sub < BS / 16; ++sub) {
+          const int tok = sub * 16 + (mj >> 1) * 8 + mr;
+          const int dim = ks * 16 + (mj & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4(kbase + Geo::offset(tok, dim * 2), b0, b1, b2, b3);
+          mma_bf16_16816(s[u * NT + 2 * sub], qa[ks], b0, b1);
+          mma_bf16_16816(s[u * NT + 2 * sub + 1], qa[ks], b2, b3);
+        }
       }
     }
     // Scale, mask tokens past the context, online softmax per query row.
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
+    for (int n = 0; n < NTU; ++n) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int tok = n * 8 + 2 * t4 + (e & 1);
-        s[n][e] = (tok < nvalid) ? s[n][e] * scale_log2 : -INFINITY;
+        s[n][e] = (tok >= nfirst && tok < nvalid) ? s[n][e] * scale_log2 : -INFINITY;
       }
       mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][1]));
       mx1 = fmaxf(mx1, fmaxf(s[n][2], s[n][3]));
@@ -320,7 +358,7 @@ struct MmaWarp {
     m[1] = mn1;
     float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
+    for (int n = 0; n < NTU; ++n) {
       s[n][0] = fast_exp2(s[n][0] - mn0);
       s[n][1] = fast_exp2(s[n][1] - mn0);
       s[n][2] = fast_exp2(s[n][2] - mn1);
@@ -337,35 +375,77 @@ struct MmaWarp {
       o[n][2] *= a1;
       o[n][3] *= a1;
     }
-    // Rows of V past the context may hold anything (even NaN bit patterns);
-    // p is 0 there but 0 * NaN is NaN, so clear them in shared memory.
-    if (nvalid < BS) {
-      constexpr int kUnitsPerRow = Geo::kRowBytes / 16;
-      const int units = (BS - nvalid) * kUnitsPerRow;
-      for (int u = lane; u < units; u += 32) {
-        const int row = nvalid + u / kUnitsPerRow;
-        const int b = (u % kUnitsPerRow) * 16;
-        *reinterpret_cast<uint4*>(vt + Geo::offset(row, b)) = make_uint4(0u, 0u, 0u, 0u);
+    // Rows of V outside [nfirst, nvalid) may hold anything (even NaN bit
+    // patterns); p is 0 there but 0 * NaN is NaN, so clear them in shared
+    // memory.
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int lo = nfirst - u * BS;   // rows [0, lo) and [hi, BS) are outside
+      const int hi = nvalid - u * BS;
+      if (lo > 0 || hi < BS) {
+        constexpr int kUnitsPerRow = Geo::kRowBytes / 16;
+        for (int x = lane; x < BS * kUnitsPerRow; x += 32) {
+          const int row = x / kUnitsPerRow;
+          if (row < lo || row >= hi) {
+            const int b = (x % kUnitsPerRow) * 16;
+            *reinterpret_cast<uint4*>(vts[u] + Geo::offset(row, b)) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        fence_proxy_async_smem();  // the stage is refilled by TMA later
+        __syncwarp();
       }
-      fence_proxy_async_smem();  // the stage is refilled by TMA later
-      __syncwarp();
     }
 #pragma unroll
-    for (int kk = 0; kk < BS / 16; ++kk) {
-      uint32_t pa[4];
-      pa[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-      pa[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-      pa[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+    for (int u = 0; u < U; ++u) {
+      const uint32_t vbase = smem_addr(vts[u]);
 #pragma unroll
-      for (int nd = 0; nd < D / 16; ++nd) {
-        const int tok = kk * 16 + (mj & 1) * 8 + mr;
-        const int dim = nd * 16 + (mj >> 1) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4_trans(vbase + Geo::offset(tok, dim * 2), b0, b1, b2, b3);
-        mma_bf16_16816(o[2 * nd], pa, b0, b1);
-        mma_bf16_16816(o[2 * nd + 1], pa, b2, b3);
+      for (int kk = 0; kk < BS / 16; ++kk) {
+        const int n0 = u * NT + 2 * kk;
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(s[n0][0], s[n0][1]);
+        pa[1] = pack_bf16x2(s[n0][2], s[n0][3]);
+        pa[2] = pack_bf16x2(s[n0 + 1][0], s[n0 + 1][1]);
+        pa[3] = pack_bf16x2(s[n0 + 1][2], s[n0 + 1][3]);
+#pragma unroll
+        for (int nd = 0; nd < D / 16; ++nd) {
+          const int tok = kk * 16 + (mj & 1) * 8 + mr;
+          const int dim = nd * 16 + (mj >> 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4_trans(vbase + Geo::offset(tok, dim * 2), b0, b1, b2, b3);
+          mma_bf16_16816(o[2 * nd], pa, b0, b1);
+          mma_bf16_16816(o[2 * nd + 1], pa, b2, b3);
+        }
       }
+    }
+  }
+
+  // Writes this warp's rows g (slot pr0) and g+8 (slot pr1) as partials
+  // (m, l, unnormalised acc); a negative slot is skipped.
+  __device__ __forceinline__ void store_partials(const DecodeArgs& a, int64_t pr0, int64_t pr1,
+                                                 int lane) {
+    const int t4 = lane & 3;
+    float l0 = l[0], l1 = l[1];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (pr0 >= 0) {
+      if (t4 == 0) {
+        a.part_m[pr0] = m[0];
+        a.part_l[pr0] = l0;
+      }
+#pragma unroll
+      for (int n = 0; n < ND; ++n)
+        *reinterpret_cast<float2*>(a.part_acc + pr0 * D + n * 8 + 2 * t4) = make_float2(o[n][0], o[n][1]);
+    }
+    if (pr1 >= 0) {
+      if (t4 == 0) {
+        a.part_m[pr1] = m[1];
+        a.part_l[pr1] = l1;
+      }
+#pragma unroll
+      for (int n = 0; n < ND; ++n)
+        *reinterpret_cast<float2*>(a.part_acc + pr1 * D + n * 8 + 2 * t4) = make_float2(o[n][2], o[n][3]);
     }
   }
 
@@ -413,6 +493,29 @@ __device__ __forceinline__ int partitions_of(int ctx, int bs, int pb) {
 
 __device__ __forceinline__ int clamp_ctx(int raw, int max_tokens) {
   return (raw < 0 || raw > max_tokens) ? 0 : raw;
+}
+
+// Leading blocks of sequence s that a shared-prefix pass already covered:
+// at most its full blocks.
+__device__ __forceinline__ int first_token(const DecodeArgs& a, int ctx) {
+  return (a.window > 0 && ctx > a.window) ? ctx - a.window : 0;
+}
+
+__device__ __forceinline__ int skip_blocks(const DecodeArgs& a, int s, int ctx, int bs) {
+  int k = first_token(a, ctx) / bs;  // blocks wholly before a sliding window
+  if (a.seq_skip_blocks != nullptr) {
+    const int full = ctx / bs;
+    const int g = a.seq_skip_blocks[s];
+    k = max(k, g < 0 ? 0 : (g > full ? full : g));
+  }
+  return k;
+}
+
+// Partitions the split kernel makes for sequence s (its blocks after the
+// skipped prefix; at least one).
+__device__ __forceinline__ int seq_partitions(const DecodeArgs& a, int s, int max_tokens, int bs) {
+  const int ctx = clamp_ctx(a.context_lens[s], max_tokens);
+  return partitions_of(ctx - skip_blocks(a, s, ctx, bs) * bs, bs, a.partition_blocks);
 }
 
 
@@ -473,8 +576,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
     const int lo = min(B, tid * chunk);
     const int hi = min(B, lo + chunk);
     int mine = 0;
-    for (int i = lo; i < hi; ++i)
-      mine += partitions_of(clamp_ctx(a.context_lens[i], max_tokens), BS, a.partition_blocks);
+    for (int i = lo; i < hi; ++i) mine += seq_partitions(a, i, max_tokens, BS);
     int incl = mine;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -488,7 +590,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
     int run = base + incl - mine;
     for (int i = lo; i < hi; ++i) {
       prefix[i] = run;
-      run += partitions_of(clamp_ctx(a.context_lens[i], max_tokens), BS, a.partition_blocks);
+      run += seq_partitions(a, i, max_tokens, BS);
     }
     if (tid == NT - 1) prefix[B] = base + incl;
     __syncthreads();
@@ -539,7 +641,10 @@ __global__ void __launch_bounds__(Cfg::kThreads)
     const int ctx = clamp_ctx(ctx_raw, max_tokens);
     if (ctx != ctx_raw && p == 0 && kvh == 0 && tid == 0) report(a.dev_err, PA_DEVERR_CONTEXT_LEN);
     const int nb = (ctx + BS - 1) / BS;
-    const int b_begin = a.persistent ? p * a.partition_blocks : 0;
+    const int skip = a.persistent ? skip_blocks(a, s, ctx, BS) : 0;
+    const int win_first = a.persistent ? first_token(a, ctx) : 0;
+    const int part_base = (a.persistent && a.seq_part_base) ? a.seq_part_base[s] : 0;
+    const int b_begin = a.persistent ? skip + p * a.partition_blocks : 0;
     const int b_end = a.persistent ? min(nb, b_begin + a.partition_blocks) : nb;
     const int nblk = max(0, b_end - b_begin);
     // This warp reads half `hu` of blocks b_begin + wb + j*WB.
@@ -614,9 +719,13 @@ __global__ void __launch_bounds__(Cfg::kThreads)
       }
       if (!(bad & (1u << stage))) {
         const int lb = b_begin + wb + j * WB;  // logical block
-        const int nvalid = min(UR, ctx - lb * BS - hu * UR);
-        uint8_t* kt = my_ring + stage * Cfg::kStageBytes;
-        st.block(kt, kt + Geo::kTileBytes, nvalid, lane);
+        const int u0 = lb * BS + hu * UR;      // first token of the unit
+        const int nvalid = min(UR, ctx - u0);
+        const int nfirst = win_first - u0;     // > 0 only inside a window's first block
+        if (nfirst < nvalid) {                 // a unit wholly before the window is skipped
+          uint8_t* kt = my_ring + stage * Cfg::kStageBytes;
+          st.block(kt, kt + Geo::kTileBytes, nfirst, nvalid, lane);
+        }
       }
       __syncwarp();
       if (j + NS < nj) issue(j + NS);
@@ -641,7 +750,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
                  sm_acc + warp * Cfg::kRowsMax * D, lane);
     }
     __syncthreads();
-    const bool final_out = (nparts == 1);
+    const bool final_out = (nparts == 1) && (part_base == 0);
     const int64_t row0 = static_cast<int64_t>(s) * a.num_q_heads + static_cast<int64_t>(kvh) * G;
     for (int idx = tid; idx < G * D; idx += NT) {
       const int h = idx / D;
@@ -662,7 +771,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
       if (final_out) {
         reinterpret_cast<T*>(a.out)[row * D + d] = Elt<T>::from_f32(L > 0.f ? A / L : 0.f);
       } else {
-        const int64_t pr = row * a.max_partitions + p;
+        const int64_t pr = row * a.max_partitions + part_base + p;
         a.part_acc[pr * D + d] = A;
         if (d == 0) {
           a.part_m[pr] = M;
@@ -682,6 +791,7 @@ __global__ void __launch_bounds__(Cfg::kThreads)
     ++iter;
   }
 
+  if (a.wait_prior_at_exit) grid_dependency_wait();
   if (a.persistent && tid == 0) {
     // The last CTA to get here resets the counters for the next call; every
     // other CTA has already taken its final ticket.
@@ -712,9 +822,9 @@ __global__ void __launch_bounds__(128)
   const int row = blockIdx.x;  // s * Hq + h
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int s = row / a.num_q_heads;
-  const int ctx = clamp_ctx(a.context_lens[s], a.max_blocks_per_seq * block_size);
-  const int np = partitions_of(ctx, block_size, a.partition_blocks);
-  if (np <= 1) return;
+  const int base_parts = a.seq_part_base ? a.seq_part_base[s] : 0;
+  const int np = base_parts + seq_partitions(a, s, a.max_blocks_per_seq * block_size, block_size);
+  if (np <= 1 && base_parts == 0) return;
   const int64_t base = static_cast<int64_t>(row) * a.max_partitions;
   float M = -INFINITY;
   for (int p = tid; p < np; p += 128) M = fmaxf(M, a.part_m[base + p]);

@@ -271,3 +271,88 @@ def test_decode_step_rejects_before_touching_the_device():
         binding.PA_ERR_NO_FREE_BLOCKS
     assert bm2.context_len(7) == 8 and bm2.free_queue_list() == []
     assert ctypes.sizeof(binding.StepBuffers) == 168
+
+
+def _reference_groups(tables_by_pos, ctx_by_pos, bs, min_shared=1):
+    """Independent statement of the grouping: bucket by first block in batch
+    order; shared = longest common table prefix, capped at blocks full for all."""
+    buckets, order = {}, []
+    for i, t in enumerate(tables_by_pos):
+        if not t:
+            continue
+        if t[0] not in buckets:
+            buckets[t[0]] = []
+            order.append(t[0])
+        buckets[t[0]].append(i)
+    offs, members, blocks = [0], [], []
+    for b0 in order:
+        mem = buckets[b0]
+        if len(mem) < 2:
+            continue
+        shared = min(ctx_by_pos[i] // bs for i in mem)
+        for i in mem:
+            k = 0
+            while k < shared and tables_by_pos[i][k] == tables_by_pos[mem[0]][k]:
+                k += 1
+            shared = k
+        if shared < max(1, min_shared):
+            continue
+        members += mem
+        blocks.append(shared)
+        offs.append(len(members))
+    return offs, members, blocks
+
+
+@pytest.mark.parametrize("name", ["prefix", "prefix_cow", "tiny", "gqa"])
+def test_prefix_groups_match_reference(name):
+    w = workloads.WORKLOADS[name]()
+    bm = LibBM(w.num_blocks, w.block_size, w.max_blocks_per_seq, w.free_order)
+    build_tables(bm, w)
+    if w.step_seqs:
+        bm.append_slots_arrays(w.step_seqs)
+    seqs = list(w.decode_seqs)
+    rng = np.random.default_rng(3)
+    rng.shuffle(seqs)
+    offs, members, blocks = bm.prefix_groups(seqs)
+    tabs = [bm.block_table(s) for s in seqs]
+    ctxs = [bm.context_len(s) for s in seqs]
+    want = _reference_groups(tabs, ctxs, w.block_size)
+    assert (offs.tolist(), members.tolist(), blocks.tolist()) == want
+    if name.startswith("prefix"):
+        assert len(blocks) == 8 and all(b == 250 for b in blocks)
+        assert all(offs[g + 1] - offs[g] == 16 for g in range(8))
+    if name == "gqa":
+        assert len(blocks) == 0   # no sharing
+
+
+def test_prefix_groups_partial_sharing_and_threshold():
+    bm = LibBM(40, 4, 10, list(range(40)))
+    bm.allocate(0, 17)          # blocks 0..4, tail holds 1 token
+    bm.fork(0, 1)
+    bm.fork(0, 2)
+    for _ in range(3):
+        bm.append_slot(1)       # 1 copies block 4 on its first append
+    bm.allocate(3, 8)
+    offs, members, blocks = bm.prefix_groups([3, 2, 1, 0])
+    assert offs.tolist() == [0, 3] and members.tolist() == [1, 2, 3] and blocks.tolist() == [4]
+    offs, members, blocks = bm.prefix_groups([3, 2, 1, 0], min_shared_blocks=5)
+    assert offs.tolist() == [0] and members.size == 0
+
+
+def test_shared_prefix_rejects_bad_groups_on_host():
+    lib = binding.library()
+    a = _decode_args()
+    base = [a["q"], a["k"], a["v"], a["bt"], a["ctx"], a["B"], a["Hq"], a["Hkv"], a["D"], a["BS"],
+            a["NB"], a["MBS"], a["scale"], a["dtype"], 512]
+    ws = FAKE
+
+    def call(offs, members, blocks, ng):
+        o = np.asarray(offs, np.int32); m = np.asarray(members, np.int32); b = np.asarray(blocks, np.int32)
+        return lib.pa_decode_shared_prefix(*base, ng, o.ctypes.data, m.ctypes.data, b.ctypes.data,
+                                           ws, 1 << 40, a["out"], None, None)
+    assert call([0, 2], [0, 0], [1], 1) == binding.PA_ERR_INVALID_ARG      # repeated member
+    assert call([0, 2], [0, 9], [1], 1) == binding.PA_ERR_INVALID_ARG      # member past the batch
+    assert call([1, 2], [0, 1], [1], 1) == binding.PA_ERR_INVALID_ARG      # offsets start at 1
+    assert call([0, 2], [0, 1], [99], 1) == binding.PA_ERR_INVALID_ARG     # more blocks than the table
+    base[13] = binding.PA_F32
+    assert call([0, 2], [0, 1], [1], 1) == binding.PA_ERR_UNSUPPORTED      # bf16 only

@@ -1,0 +1,100 @@
+"""pa_decode_shared_prefix against the oracle.
+
+Forked sequences share their prompt's blocks; the shared-prefix route reads
+them once per KV head for the whole group and must still return plain decode
+attention. Small cases are compared with the full float64 oracle (several
+groups, a group wider than one 64-row CTA, sequences in no group, block
+sizes 16 and 32); the full-size prefix-sharing workloads with sampled rows.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_336_b200 import binding, workloads
+
+from gpu_util import (build_tables, check_close, device_tables, oracle_one, sample_pairs, setup,
+                      to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("G,bs,branches", [(1, 16, 5), (4, 16, 16), (8, 32, 12), (4, 32, 3)])
+def test_shared_prefix_small_matches_oracle(G, bs, branches):
+    Hkv, D = 2, 128
+    rng = np.random.default_rng(40 + G + bs)
+    NB = 400
+    bm = binding.BlockManager(NB, bs, 64, rng.permutation(NB).astype(np.int32))
+    seqs = []
+    nid = 0
+    for prompt_len in (7 * bs + 3, 4 * bs, 2 * bs + 9):     # partial, exact, partial prompt tails
+        root = nid
+        bm.allocate(root, prompt_len)
+        seqs.append(root)
+        nid += 1
+        for _ in range(branches - 1):
+            bm.fork(root, nid)
+            seqs.append(nid)
+            nid += 1
+    for s in seqs:                                            # private tokens (copy-on-write on the way)
+        for _ in range(int(rng.integers(0, 2 * bs))):
+            r = bm.append_slot(s)
+    for extra in range(3):                                    # sequences in no group
+        bm.allocate(nid, int(rng.integers(0, 6 * bs)))
+        seqs.append(nid)
+        nid += 1
+    order = list(rng.permutation(seqs))
+    w = workloads.random_small(7, num_seqs=1, num_q_heads=G * Hkv, num_kv_heads=Hkv, head_dim=D,
+                               block_size=bs, dtype=workloads.BF16, max_ctx=1)
+    w.num_blocks = NB
+    k_pool, v_pool = workloads.draw_pools(w, "cuda")
+    q = workloads.draw_queries(w, len(order), device="cuda")
+    bt, ctx, tables, ctx_np = device_tables(bm, order)
+    groups = bm.prefix_groups(order)
+    assert len(groups[2]) >= 2
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = binding.decode_shared_prefix(q, k_pool, v_pool, bt, ctx, w.scale, groups,
+                                       partition_tokens=2 * bs, dev_err=err)
+    ref = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=2 * bs)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    want = oracle.paged_decode(to_f64(q), to_f64(k_pool), to_f64(v_pool), tables, ctx_np, w.scale)
+    check_close(to_f64(out), want, w.dtype, "shared prefix")
+    check_close(to_f64(ref), want, w.dtype, "split")
+    # twice in a row on the same workspace-less call path, and with no groups at all
+    out2 = binding.decode_shared_prefix(q, k_pool, v_pool, bt, ctx, w.scale, groups,
+                                        partition_tokens=2 * bs)
+    assert torch.equal(out, out2)
+    empty = (np.zeros(1, np.int32), np.zeros(0, np.int32), np.zeros(0, np.int32))
+    out3 = binding.decode_shared_prefix(q, k_pool, v_pool, bt, ctx, w.scale, empty,
+                                        partition_tokens=2 * bs)
+    check_close(to_f64(out3), want, w.dtype, "no groups")
+
+
+@pytest.mark.parametrize("name", ["prefix", "prefix_cow"])
+def test_shared_prefix_full_size(name):
+    w = workloads.WORKLOADS[name]()
+    bm, k_pool, v_pool = setup(w)
+    slots, pairs = bm.append_slots_arrays(w.step_seqs)
+    kn, vn = workloads.draw_new_kv(w, len(w.step_seqs), device="cuda")
+    if len(pairs):
+        binding.copy_blocks(k_pool, v_pool, torch.from_numpy(pairs).cuda())
+    binding.kv_append(kn, vn, torch.from_numpy(slots).cuda(), k_pool, v_pool)
+    seqs = w.decode_seqs
+    bt, ctx, tables, ctx_np = device_tables(bm, seqs)
+    groups = bm.prefix_groups(seqs)
+    assert len(groups[2]) == 8
+    q = workloads.draw_queries(w, len(seqs), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = binding.decode_shared_prefix(q, k_pool, v_pool, bt, ctx, w.scale, groups, dev_err=err)
+    ref = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    check_close(to_f64(out), to_f64(ref), w.dtype, "shared prefix vs split")
+    rng = np.random.default_rng(w.seed)
+    got, want = [], []
+    for s, h in sample_pairs(rng, len(seqs), w.num_q_heads, 8, [(0, 0), (len(seqs) - 1, 31)]):
+        want.append(oracle_one(q, k_pool, v_pool, tables[s], ctx_np[s], w.scale, s, h))
+        got.append(to_f64(out[s, h]))
+    check_close(np.stack(got), np.stack(want), w.dtype, name)

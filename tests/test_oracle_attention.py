@@ -226,3 +226,45 @@ def test_copy_blocks_hand_example():
     assert np.array_equal(k_pool[3], k0[1]) and np.array_equal(v_pool[3], v0[1])
     assert np.array_equal(k_pool[2], k0[0]) and np.array_equal(v_pool[2], v0[0])
     assert np.array_equal(k_pool[:2], k0[:2]) and np.array_equal(v_pool[:2], v0[:2])
+
+
+def test_window_covering_the_context_is_plain_decode():
+    rng = np.random.default_rng(8)
+    k_pool = rng.standard_normal((6, 2, 16, 8))
+    v_pool = rng.standard_normal((6, 2, 16, 8))
+    q = rng.standard_normal((2, 4, 8))
+    tables = np.array([[5, 1, 3, 0], [2, 4, -1, -1]])
+    lens = np.array([50, 20])
+    full = oracle.paged_decode(q, k_pool, v_pool, tables, lens, 0.3)
+    for w in (50, 64, 10_000):
+        assert np.array_equal(oracle.paged_decode_window(q, k_pool, v_pool, tables, lens, 0.3, w)[0], full[0])
+
+
+def test_window_of_one_returns_the_last_value():
+    rng = np.random.default_rng(9)
+    k_pool = rng.standard_normal((4, 1, 16, 8))
+    v_pool = rng.standard_normal((4, 1, 16, 8))
+    q = rng.standard_normal((1, 2, 8)) * 20
+    tables = np.array([[3, 0, 2]])
+    out = oracle.paged_decode_window(q, k_pool, v_pool, tables, np.array([37]), 0.2, 1)
+    assert np.array_equal(out[0, 0], v_pool[2, 0, 4]) and np.array_equal(out[0, 1], v_pool[2, 0, 4])
+
+
+@pytest.mark.parametrize("window", [1, 5, 16, 17, 33, 100])
+def test_window_matches_sdpa_on_the_slice(window):
+    rng = np.random.default_rng(10 + window)
+    lens = [40, 3, 64, 90]
+    contig_k = [rng.standard_normal((n, 2, 16)) for n in lens]
+    contig_v = [rng.standard_normal((n, 2, 16)) for n in lens]
+    k_pool, v_pool, tables = _place(contig_k, contig_v, 16, 30, rng)
+    q = rng.standard_normal((4, 4, 16))
+    got = oracle.paged_decode_window(q, k_pool, v_pool, tables, np.array(lens), 0.25, window)
+    sliced_k = [k[max(0, len(k) - window):] for k in contig_k]
+    sliced_v = [v[max(0, len(v) - window):] for v in contig_v]
+    want = _sdpa_reference(q, sliced_k, sliced_v, 0.25)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    # released blocks before the window are never touched
+    t2 = tables.copy()
+    for s, n in enumerate(lens):
+        t2[s, :max(0, n - window) // 16] = -1
+    assert np.array_equal(oracle.paged_decode_window(q, k_pool, v_pool, t2, np.array(lens), 0.25, window), got)

@@ -126,7 +126,8 @@ def _check_invariants(bm: BlockManager):
     counts = np.zeros(bm.num_blocks, dtype=np.int64)
     for table in bm.tables.values():
         for b in table:
-            counts[b] += 1
+            if b >= 0:
+                counts[b] += 1
     assert list(counts) == list(bm.refcount)
     used = int(np.sum(counts > 0))
     assert used + len(bm.free_queue) == bm.num_blocks
@@ -137,6 +138,8 @@ def _check_invariants(bm: BlockManager):
         waste = len(table) * bm.block_size - ctx
         assert 0 <= waste <= bm.block_size - 1 or (ctx == 0 and len(table) == 0)
         assert len(table) <= bm.max_blocks_per_seq
+        released = [i for i, b in enumerate(table) if b < 0]
+        assert released == list(range(len(released)))   # only a leading run is released
 
 
 def random_ops(seed, n_ops=400, num_blocks=40, block_size=4, mbs=12):
@@ -157,9 +160,12 @@ def random_ops(seed, n_ops=400, num_blocks=40, block_size=4, mbs=12):
             next_id += 1
         elif r < 0.7:
             ops.append(("append", int(rng.choice(live))))
-        elif r < 0.85:
+        elif r < 0.8:
             k = int(rng.integers(1, min(4, len(live)) + 1))
             ops.append(("appends",) + tuple(int(x) for x in rng.choice(live, size=k, replace=False)))
+        elif r < 0.85:
+            # sliding window: release everything before a random token position
+            ops.append(("release", int(rng.choice(live)), int(rng.integers(0, 4 * block_size * 2))))
         else:
             victim = int(rng.choice(live))
             ops.append(("free", victim))
@@ -183,6 +189,10 @@ def apply_op(bm, op):
             return ("ok", tuple((r.slot, r.cow_src, r.cow_dst) for r in rs))
         elif kind == "free":
             bm.free(op[1])
+        elif kind == "release":
+            first = min(op[2], bm.context_len(op[1]))
+            r = bm.release_before(op[1], first)
+            return ("ok", len(r) if isinstance(r, list) else r)
         return ("ok", None)
     except NoFreeBlocks:
         return ("nofree", None)
@@ -256,3 +266,20 @@ def test_rejects_bad_arguments():
         bm.fork(7, 8)                  # unknown parent
     with pytest.raises(InvalidArgument):
         BlockManager(3, 4, 2, [0, 0, 1])
+
+
+def test_release_before_hand_example():
+    bm = BlockManager(8, 4, 6, [3, 1, 4, 0, 5, 2, 6, 7])
+    bm.allocate(0, 10)             # blocks 3, 1, 4
+    bm.fork(0, 1)                  # shared: counts 2
+    assert bm.release_before(0, 9) == []          # blocks 0,1 of seq 0 out: 3, 1 still held by seq 1
+    assert bm.block_table(0) == [-1, -1, 4]
+    assert bm.refcount[3] == 1 and bm.refcount[1] == 1
+    assert bm.release_before(1, 4) == [3]         # seq 1 drops block 3 (count 0 -> reclaimed)
+    assert bm.block_table(1) == [-1, 1, 4]
+    assert list(bm.free_queue) == [0, 5, 2, 6, 7, 3]
+    st = bm.stats()
+    assert st["logical_slots"] == 3 * 4 and st["logical_tokens"] == (10 - 8) + (10 - 4)
+    bm.free(0)
+    bm.free(1)
+    assert sorted(bm.free_queue) == list(range(8))
