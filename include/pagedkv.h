@@ -234,6 +234,24 @@ pa_status_t pa_decode_split_window(const void* q, const void* k_pool, const void
                                    void* stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_swap_out / pa_swap_in - the data movement of swapping: whole blocks
+ * (K and V, all heads; block_bytes each) between the device pools and two
+ * host buffers of num_host_slots blocks each. pairs (device int64
+ * [num_pairs][2]): swap-out (device block, host slot), swap-in (host slot,
+ * device block). The host buffers must be page-locked and mapped
+ * (cudaHostAlloc / cudaHostRegister; the library looks up their device
+ * addresses); the copies are kernels that read or write them directly over
+ * the host link, 16-byte vectors. Bit-exact. Indices out of range set
+ * PA_DEVERR_COPY_PAIR and are skipped.
+ * ------------------------------------------------------------------------- */
+pa_status_t pa_swap_out(const void* k_pool, const void* v_pool, void* host_k, void* host_v,
+                        const int64_t* pairs, int num_pairs, size_t block_bytes, int num_blocks,
+                        int num_host_slots, uint32_t* dev_err, void* stream);
+pa_status_t pa_swap_in(const void* host_k, const void* host_v, void* k_pool, void* v_pool,
+                       const int64_t* pairs, int num_pairs, size_t block_bytes, int num_blocks,
+                       int num_host_slots, uint32_t* dev_err, void* stream);
+
+/* ---------------------------------------------------------------------------
  * pa_kv_append - decode-step write of new tokens' keys and values into their
  * slots ([Q], Map Logical to Physical Blocks: decode appends into the partly
  * filled tail block; [G] section 4 step 3: the write proceeds on the private
@@ -329,6 +347,19 @@ pa_status_t pa_bm_free(pa_bm_t bm, int64_t seq_id);
  * ctx - first_token tokens or fewer never reads the released entries. */
 pa_status_t pa_bm_release_before(pa_bm_t bm, int64_t seq_id, int64_t first_token,
                                  int* num_reclaimed);
+
+/* Preemption by swap ([Q] How It Works: an allocation failure is met by
+ * admission control, preemption, swap or rejection). pa_bm_swap_out gives up
+ * the sequence's blocks (counts drop by one, blocks reaching zero are
+ * reclaimed) but keeps its context length; blocks[0..*n) receives its table
+ * at that moment (-1 for released entries). Copy those blocks to host memory
+ * (pa_swap_out) on the stream before any later work can reuse them. A
+ * swapped-out sequence cannot append, fork or release until pa_bm_swap_in,
+ * which takes one new private block per resident entry (all or nothing,
+ * PA_ERR_NO_FREE_BLOCKS otherwise) and writes the new table to blocks[0..*n);
+ * copy the host copies into those blocks (pa_swap_in) before decoding it. */
+pa_status_t pa_bm_swap_out(pa_bm_t bm, int64_t seq_id, int32_t* blocks, int capacity, int* n);
+pa_status_t pa_bm_swap_in(pa_bm_t bm, int64_t seq_id, int32_t* blocks, int capacity, int* n);
 
 /* Copy one sequence's block table into row[0..row_capacity); *n_blocks gets
  * its length (PA_ERR_INVALID_ARG if row_capacity is too small). */

@@ -72,6 +72,7 @@ class BlockManager:
         self.refcount = [0] * num_blocks
         self.tables: dict[int, list[int]] = {}
         self.context: dict[int, int] = {}
+        self.swapped: dict[int, list[int]] = {}   # table at swap-out time
         self.cow_copies = 0
 
     # -- queries -----------------------------------------------------------
@@ -92,7 +93,8 @@ class BlockManager:
         # resident blocks and tokens (a released window prefix no longer counts)
         resident = {s: sum(1 for b in t if b >= 0) for s, t in self.tables.items()}
         logical_slots = sum(resident.values()) * self.block_size
-        tokens = sum(ctx - (len(self.tables[s]) - resident[s]) * self.block_size
+        tokens = sum(0 if s in self.swapped else
+                     ctx - (len(self.tables[s]) - resident[s]) * self.block_size
                      for s, ctx in self.context.items())
         return {
             "num_blocks": self.num_blocks,
@@ -127,6 +129,8 @@ class BlockManager:
     def fork(self, parent: int, child: int) -> None:
         """Child shares all of the parent's blocks; counts go up, no data moves."""
         self._require(parent)
+        if parent in self.swapped:
+            raise InvalidArgument(f"sequence {parent} is swapped out")
         if child in self.tables:
             raise InvalidArgument(f"sequence {child} already exists")
         table = list(self.tables[parent])
@@ -137,6 +141,8 @@ class BlockManager:
         self.context[child] = self.context[parent]
 
     def _need_for_append(self, seq: int, refcount_view) -> int:
+        if seq in self.swapped:
+            raise InvalidArgument(f"sequence {seq} is swapped out")
         ctx = self.context[seq]
         table = self.tables[seq]
         if ctx % self.block_size == 0:
@@ -203,6 +209,8 @@ class BlockManager:
         self._require(seq)
         if first_token < 0:
             raise InvalidArgument("first_token must be >= 0")
+        if seq in self.swapped:
+            raise InvalidArgument(f"sequence {seq} is swapped out")
         table = self.tables[seq]
         n_out = min(first_token // self.block_size, len(table))
         reclaimed = []
@@ -218,6 +226,55 @@ class BlockManager:
             self.free_queue.append(b)
         return sorted(reclaimed)
 
+    def swap_out(self, seq: int) -> list[int]:
+        """Preemption by swapping ("What is PagedAttention?", How It Works:
+        an allocation failure is met by admission control, preemption, swap
+        or rejection). The sequence keeps its context length but gives up
+        its blocks: every resident table entry's count drops by one (blocks
+        reaching zero are reclaimed, ascending, to the back of the queue).
+        Returns the blocks in table order (-1 for released entries): the
+        caller copies them to host memory before the pool reuses them."""
+        self._require(seq)
+        if seq in self.swapped:
+            raise InvalidArgument(f"sequence {seq} is already swapped out")
+        table = self.tables[seq]
+        reclaimed = []
+        for b in table:
+            if b < 0:
+                continue
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                reclaimed.append(b)
+        for b in sorted(reclaimed):
+            self.free_queue.append(b)
+        self.swapped[seq] = list(table)
+        self.tables[seq] = [-1 if b >= 0 else b for b in table]
+        return list(table)
+
+    def swap_in(self, seq: int) -> list[int]:
+        """Bring a swapped-out sequence back: one new private block per
+        previously resident entry, popped from the queue in table order, all
+        or nothing. Returns the new table (the caller copies the host copies
+        into the new blocks)."""
+        self._require(seq)
+        if seq not in self.swapped:
+            raise InvalidArgument(f"sequence {seq} is not swapped out")
+        old = self.swapped[seq]
+        need = sum(1 for b in old if b >= 0)
+        if need > len(self.free_queue):
+            raise NoFreeBlocks(f"swap-in needs {need} blocks, {len(self.free_queue)} free")
+        table = []
+        for b in old:
+            if b < 0:
+                table.append(b)
+            else:
+                nb = self.free_queue.popleft()
+                self.refcount[nb] = 1
+                table.append(nb)
+        self.tables[seq] = table
+        del self.swapped[seq]
+        return list(table)
+
     def free(self, seq: int) -> None:
         """Drop a finished sequence; reclaim blocks whose count reaches zero."""
         self._require(seq)
@@ -232,6 +289,7 @@ class BlockManager:
             self.free_queue.append(b)
         del self.tables[seq]
         del self.context[seq]
+        self.swapped.pop(seq, None)
 
     def _require(self, seq: int) -> None:
         if seq not in self.tables:
@@ -246,6 +304,10 @@ class BlockManager:
             tuple(sorted(self.context.items())),
             self.cow_copies,
         )
+
+    def is_swapped(self, seq: int) -> bool:
+        self._require(seq)
+        return seq in self.swapped
 
 
 class _Overlay:

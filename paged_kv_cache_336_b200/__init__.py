@@ -23,5 +23,7 @@ from .binding import (  # noqa: F401
     decode_split_workspace_size,
     kv_append,
     copy_blocks,
+    swap_out,
+    swap_in,
     library,
 )

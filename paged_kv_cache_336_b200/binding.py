@@ -94,6 +94,10 @@ _SIGNATURES = {
                                      _I, _P, _P, _P, _P, _SZ, _P, _P, _P]),
     "pa_bm_prefix_groups": (_I, [_P, _P, _I, _I, _P, _P, _P, ctypes.POINTER(_I)]),
     "pa_bm_release_before": (_I, [_P, _I64, _I64, ctypes.POINTER(_I)]),
+    "pa_bm_swap_out": (_I, [_P, _I64, _P, _I, ctypes.POINTER(_I)]),
+    "pa_bm_swap_in": (_I, [_P, _I64, _P, _I, ctypes.POINTER(_I)]),
+    "pa_swap_out": (_I, [_P, _P, _P, _P, _P, _I, _SZ, _I, _I, _P, _P]),
+    "pa_swap_in": (_I, [_P, _P, _P, _P, _P, _I, _SZ, _I, _I, _P, _P]),
     "pa_decode_split_window": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                                     _I, _P, _SZ, _P, _P, _P]),
     "pa_kv_append": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
@@ -271,6 +275,30 @@ def decode_split_window(q, k_pool, v_pool, block_tables, context_lens, scale: fl
         D, BS, NB, MBS, float(scale), _dtype_code(q), int(partition_tokens), int(window),
         workspace.ptr, workspace.nbytes, _ptr(out), _ptr(dev_err), _stream_ptr(stream)))
     return out
+
+
+def _swap(fn_name, src_k, src_v, dst_k, dst_v, pairs, pool, host, dev_err, stream):
+    torch = _torch()
+    if pairs.dtype != torch.int64 or pairs.dim() != 2 or pairs.shape[1] != 2 or not pairs.is_cuda:
+        raise InvalidArgumentError(PA_ERR_INVALID_ARG, "pairs must be a CUDA int64 [n, 2] tensor")
+    if host.is_cuda or not host.is_pinned():
+        raise InvalidArgumentError(PA_ERR_INVALID_ARG, "host buffers must be pinned CPU tensors")
+    if host.shape[1:] != pool.shape[1:] or host.dtype != pool.dtype:
+        raise InvalidArgumentError(PA_ERR_INVALID_ARG, "host buffer must be [slots, *block shape]")
+    block_bytes = pool[0].numel() * pool.element_size()
+    _check(getattr(library(), fn_name)(
+        _ptr(src_k), _ptr(src_v), _ptr(dst_k), _ptr(dst_v), _ptr(pairs), pairs.shape[0],
+        block_bytes, pool.shape[0], host.shape[0], _ptr(dev_err), _stream_ptr(stream)))
+
+
+def swap_out(k_pool, v_pool, host_k, host_v, pairs, dev_err=None, stream=None):
+    """pa_swap_out: pairs (device block, host slot) copy whole blocks to pinned host buffers."""
+    _swap("pa_swap_out", k_pool, v_pool, host_k, host_v, pairs, k_pool, host_k, dev_err, stream)
+
+
+def swap_in(host_k, host_v, k_pool, v_pool, pairs, dev_err=None, stream=None):
+    """pa_swap_in: pairs (host slot, device block) copy whole blocks back to the pools."""
+    _swap("pa_swap_in", host_k, host_v, k_pool, v_pool, pairs, k_pool, host_k, dev_err, stream)
 
 
 class Workspace:
@@ -457,6 +485,24 @@ class BlockManager:
         _check(library().pa_bm_export(self._h, ids.ctypes.data, n, tables.ctypes.data,
                                       ctx.ctypes.data, int(pad_value)))
         return tables, ctx
+
+    def swap_out(self, seq: int) -> list[int]:
+        """pa_bm_swap_out: the sequence's table at swap-out (blocks to copy out)."""
+        import numpy as np
+        buf = np.empty(self.max_blocks_per_seq, dtype=np.int32)
+        n = _I()
+        _check(library().pa_bm_swap_out(self._h, int(seq), buf.ctypes.data, buf.shape[0],
+                                        ctypes.byref(n)))
+        return [int(x) for x in buf[:n.value]]
+
+    def swap_in(self, seq: int) -> list[int]:
+        """pa_bm_swap_in: the new table (blocks to copy the host copies into)."""
+        import numpy as np
+        buf = np.empty(self.max_blocks_per_seq, dtype=np.int32)
+        n = _I()
+        _check(library().pa_bm_swap_in(self._h, int(seq), buf.ctypes.data, buf.shape[0],
+                                       ctypes.byref(n)))
+        return [int(x) for x in buf[:n.value]]
 
     def release_before(self, seq: int, first_token: int) -> int:
         """pa_bm_release_before; returns the number of blocks reclaimed."""

@@ -32,6 +32,8 @@ struct pa_bm {
   struct Seq {
     std::vector<int32_t> table;
     int64_t ctx = 0;
+    bool swapped = false;
+    std::vector<int32_t> swapped_table;  // table at swap-out time
   };
   int num_blocks = 0;
   int block_size = 0;
@@ -74,6 +76,7 @@ pa_status_t plan_step(pa_bm* bm, const int64_t* ids, int n, int64_t* need_out) {
       return fail(PA_ERR_INVALID_ARG, "unknown sequence %lld", (long long)ids[i]);
     if (!seen.insert(ids[i]).second)
       return fail(PA_ERR_INVALID_ARG, "sequence %lld appears twice in one step", (long long)ids[i]);
+    if (s->swapped) return fail(PA_ERR_INVALID_ARG, "sequence %lld is swapped out", (long long)ids[i]);
     int tail_count = 0;
     int32_t tail = -1;
     if (s->ctx % bm->block_size != 0) {
@@ -187,6 +190,7 @@ pa_status_t pa_bm_fork(pa_bm_t bm, int64_t parent_id, int64_t child_id) {
   pa_bm::Seq* p = nullptr;
   if (!find_seq(bm, parent_id, &p)) return fail(PA_ERR_INVALID_ARG, "unknown parent %lld", (long long)parent_id);
   if (bm->seqs.count(child_id)) return fail(PA_ERR_INVALID_ARG, "sequence %lld exists", (long long)child_id);
+  if (p->swapped) return fail(PA_ERR_INVALID_ARG, "sequence %lld is swapped out", (long long)parent_id);
   pa_bm::Seq c = *p;  // copy before emplace may rehash
   for (int32_t b : c.table)
     if (b >= 0) bm->refcount[b] += 1;  // released entries (-1) hold nothing
@@ -263,6 +267,7 @@ pa_status_t pa_bm_release_before(pa_bm_t bm, int64_t seq_id, int64_t first_token
   if (first_token < 0) return fail(PA_ERR_INVALID_ARG, "first_token < 0");
   pa_bm::Seq* s = nullptr;
   if (!find_seq(bm, seq_id, &s)) return fail(PA_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq_id);
+  if (s->swapped) return fail(PA_ERR_INVALID_ARG, "sequence %lld is swapped out", (long long)seq_id);
   const int64_t n_out = std::min<int64_t>(first_token / bm->block_size,
                                           static_cast<int64_t>(s->table.size()));
   std::vector<int32_t> reclaimed;
@@ -276,6 +281,60 @@ pa_status_t pa_bm_release_before(pa_bm_t bm, int64_t seq_id, int64_t first_token
   std::sort(reclaimed.begin(), reclaimed.end());
   for (int32_t b : reclaimed) bm->free_queue.push_back(b);
   if (num_reclaimed) *num_reclaimed = static_cast<int>(reclaimed.size());
+  return ok();
+}
+
+pa_status_t pa_bm_swap_out(pa_bm_t bm, int64_t seq_id, int32_t* blocks, int capacity, int* n) {
+  if (bm == nullptr || n == nullptr) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+  pa_bm::Seq* s = nullptr;
+  if (!find_seq(bm, seq_id, &s)) return fail(PA_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq_id);
+  if (s->swapped) return fail(PA_ERR_INVALID_ARG, "sequence %lld is already swapped out", (long long)seq_id);
+  const int len = static_cast<int>(s->table.size());
+  if (len > capacity || (len > 0 && blocks == nullptr))
+    return fail(PA_ERR_INVALID_ARG, "capacity %d < %d blocks", capacity, len);
+  std::vector<int32_t> reclaimed;
+  for (int32_t b : s->table) {
+    if (b < 0) continue;
+    bm->refcount[b] -= 1;
+    if (bm->refcount[b] == 0) reclaimed.push_back(b);
+  }
+  std::sort(reclaimed.begin(), reclaimed.end());
+  for (int32_t b : reclaimed) bm->free_queue.push_back(b);
+  std::copy(s->table.begin(), s->table.end(), blocks);
+  s->swapped_table = s->table;
+  for (int32_t& b : s->table) b = -1;
+  s->swapped = true;
+  *n = len;
+  return ok();
+}
+
+pa_status_t pa_bm_swap_in(pa_bm_t bm, int64_t seq_id, int32_t* blocks, int capacity, int* n) {
+  if (bm == nullptr || n == nullptr) return fail(PA_ERR_INVALID_ARG, "NULL argument");
+  pa_bm::Seq* s = nullptr;
+  if (!find_seq(bm, seq_id, &s)) return fail(PA_ERR_INVALID_ARG, "unknown sequence %lld", (long long)seq_id);
+  if (!s->swapped) return fail(PA_ERR_INVALID_ARG, "sequence %lld is not swapped out", (long long)seq_id);
+  const int len = static_cast<int>(s->swapped_table.size());
+  if (len > capacity || (len > 0 && blocks == nullptr))
+    return fail(PA_ERR_INVALID_ARG, "capacity %d < %d blocks", capacity, len);
+  int64_t need = 0;
+  for (int32_t b : s->swapped_table) need += b >= 0;
+  if (need > static_cast<int64_t>(bm->free_queue.size()))
+    return fail(PA_ERR_NO_FREE_BLOCKS, "swap-in needs %lld blocks, %zu free", (long long)need,
+                bm->free_queue.size());
+  for (int i = 0; i < len; ++i) {
+    if (s->swapped_table[i] < 0) {
+      s->table[i] = s->swapped_table[i];
+      continue;
+    }
+    const int32_t b = bm->free_queue.front();
+    bm->free_queue.pop_front();
+    bm->refcount[b] = 1;
+    s->table[i] = b;
+  }
+  std::copy(s->table.begin(), s->table.end(), blocks);
+  s->swapped = false;
+  s->swapped_table.clear();
+  *n = len;
   return ok();
 }
 
@@ -405,7 +464,7 @@ pa_status_t pa_bm_stats(pa_bm_t bm, pa_bm_stats_t* st) {
     int64_t resident = 0;
     for (int32_t b : kv.second.table) resident += b >= 0;
     const int64_t released = static_cast<int64_t>(kv.second.table.size()) - resident;
-    r.logical_tokens += kv.second.ctx - released * bm->block_size;
+    if (!kv.second.swapped) r.logical_tokens += kv.second.ctx - released * bm->block_size;
     r.logical_slots += resident * bm->block_size;
   }
   r.tail_waste_slots = r.logical_slots - r.logical_tokens;

@@ -8,8 +8,12 @@
 // * Copy: the private block receives the shared block's contents (same
 //   section, step 3); the whole block is copied.
 //
-// Both are pure HBM copies moved as 16-byte vectors; every index is checked
-// on the device and an out-of-range one is reported and skipped.
+// * Swap: whole blocks to and from page-locked host memory when a sequence is
+//   preempted ("What is PagedAttention?", How It Works: allocation failure is
+//   met by admission control, preemption, swap or rejection).
+//
+// All are copies moved as 16-byte vectors; every index is checked on the
+// device and an out-of-range one is reported and skipped.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -74,7 +78,66 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Whole-block copies between two differently indexed block arrays (device
+// pool <-> mapped host buffer). grid.y walks pairs; pair p copies block
+// pairs[2p] of `src` to block pairs[2p+1] of `dst`, K and V.
+__global__ void __launch_bounds__(256)
+    swap_blocks_kernel(const uint4* src_k, const uint4* src_v, uint4* dst_k, uint4* dst_v,
+                       const int64_t* __restrict__ pairs, int num_pairs, int64_t units_per_block,
+                       int src_blocks, int dst_blocks, uint32_t* dev_err) {
+  for (int pr = blockIdx.y; pr < num_pairs; pr += gridDim.y) {
+    const int64_t src = pairs[2 * static_cast<int64_t>(pr)];
+    const int64_t dst = pairs[2 * static_cast<int64_t>(pr) + 1];
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) report(dev_err, PA_DEVERR_COPY_PAIR);
+      continue;
+    }
+    const uint4* ks = src_k + src * units_per_block;
+    const uint4* vs = src_v + src * units_per_block;
+    uint4* kd = dst_k + dst * units_per_block;
+    uint4* vd = dst_v + dst * units_per_block;
+    for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units_per_block;
+         u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      kd[u] = ks[u];
+      vd[u] = vs[u];
+    }
+  }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device address of a page-locked, mapped host buffer.
+pa_status_t mapped(void* host, void** dev) {
+  cudaError_t err = cudaHostGetDevicePointer(dev, host, 0);
+  if (err != cudaSuccess) {
+    cudaGetLastError();
+    return fail(PA_ERR_INVALID_ARG, "host buffer is not page-locked and mapped: %s",
+                cudaGetErrorString(err));
+  }
+  return PA_OK;
+}
+
+pa_status_t launch_swap(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                        const int64_t* pairs, int num_pairs, size_t block_bytes, int src_blocks,
+                        int dst_blocks, uint32_t* dev_err, cudaStream_t stream) {
+  if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs < 0");
+  if (num_pairs == 0) return ok();
+  if (src_k == nullptr || src_v == nullptr || dst_k == nullptr || dst_v == nullptr || pairs == nullptr)
+    return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+  if (block_bytes == 0 || block_bytes % 16 != 0 || src_blocks <= 0 || dst_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "bad block_bytes or block counts");
+  if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v))
+    return fail(PA_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
+  const int64_t upb = static_cast<int64_t>(block_bytes / 16);
+  const int gx = static_cast<int>(std::min<int64_t>((upb + 1023) / 1024, 64));
+  const int gy = std::min(num_pairs, 65535);
+  swap_blocks_kernel<<<dim3(gx, gy), 256, 0, stream>>>(
+      static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v), static_cast<uint4*>(dst_k),
+      static_cast<uint4*>(dst_v), pairs, num_pairs, upb, src_blocks, dst_blocks, dev_err);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "swap launch: %s", cudaGetErrorString(err));
+  return ok();
+}
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -138,6 +201,32 @@ pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pa
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "copy_blocks launch: %s", cudaGetErrorString(err));
   return ok();
+}
+
+pa_status_t pa_swap_out(const void* k_pool, const void* v_pool, void* host_k, void* host_v,
+                        const int64_t* pairs, int num_pairs, size_t block_bytes, int num_blocks,
+                        int num_host_slots, uint32_t* dev_err, void* stream) {
+  if (num_pairs == 0) return ok();
+  if (host_k == nullptr || host_v == nullptr) return fail(PA_ERR_INVALID_ARG, "NULL host buffer");
+  void *dk = nullptr, *dv = nullptr;
+  pa_status_t st = mapped(host_k, &dk);
+  if (st != PA_OK) return st;
+  if ((st = mapped(host_v, &dv)) != PA_OK) return st;
+  return launch_swap(k_pool, v_pool, dk, dv, pairs, num_pairs, block_bytes, num_blocks,
+                     num_host_slots, dev_err, static_cast<cudaStream_t>(stream));
+}
+
+pa_status_t pa_swap_in(const void* host_k, const void* host_v, void* k_pool, void* v_pool,
+                       const int64_t* pairs, int num_pairs, size_t block_bytes, int num_blocks,
+                       int num_host_slots, uint32_t* dev_err, void* stream) {
+  if (num_pairs == 0) return ok();
+  if (host_k == nullptr || host_v == nullptr) return fail(PA_ERR_INVALID_ARG, "NULL host buffer");
+  void *dk = nullptr, *dv = nullptr;
+  pa_status_t st = mapped(const_cast<void*>(host_k), &dk);
+  if (st != PA_OK) return st;
+  if ((st = mapped(const_cast<void*>(host_v), &dv)) != PA_OK) return st;
+  return launch_swap(dk, dv, k_pool, v_pool, pairs, num_pairs, block_bytes, num_host_slots,
+                     num_blocks, dev_err, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

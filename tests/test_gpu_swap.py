@@ -1,0 +1,61 @@
+"""Swap round trip on the GPU: a sequence is preempted (its blocks copied to
+pinned host memory and reclaimed), the pool reuses the blocks, the sequence
+comes back into new blocks; the host copies are bit-exact and its decode
+output is bit-identical to before (placement does not matter)."""
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_336_b200 import binding, workloads
+
+from gpu_util import device_tables, setup
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype,G", [(workloads.BF16, 4), (workloads.F32, 1)])
+def test_swap_out_reuse_swap_in(dtype, G):
+    w = workloads.random_small(90 + G, num_seqs=4, num_q_heads=2 * G, num_kv_heads=2, head_dim=128,
+                               block_size=16, dtype=dtype, max_ctx=150, min_ctx=40, spare_blocks=2)
+    bm, k_pool, v_pool = setup(w)
+    q = workloads.draw_queries(w, 4, device="cuda")
+    bt, ctx, tables, _ = device_tables(bm, [0, 1, 2, 3])
+    before = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=32)
+
+    # preempt sequence 1: copy its blocks to host slots 0..n-1
+    old = bm.swap_out(1)
+    n = len(old)
+    host_k = torch.empty((n,) + tuple(k_pool.shape[1:]), dtype=k_pool.dtype).pin_memory()
+    host_v = torch.empty_like(host_k).pin_memory()
+    out_pairs = torch.tensor([[b, i] for i, b in enumerate(old)], dtype=torch.int64, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    binding.swap_out(k_pool, v_pool, host_k, host_v, out_pairs, dev_err=err)
+    torch.cuda.synchronize()
+    idx = torch.tensor(old, device="cuda")
+    assert torch.equal(host_k, k_pool[idx].cpu()) and torch.equal(host_v, v_pool[idx].cpu())
+
+    # the pool reuses the reclaimed blocks: another sequence overwrites them
+    bm.allocate(10, n * 16)
+    reused = torch.tensor(bm.block_table(10), device="cuda")
+    k_pool[reused] = torch.randn_like(k_pool[reused].float()).to(k_pool.dtype)
+    v_pool[reused] = torch.randn_like(v_pool[reused].float()).to(v_pool.dtype)
+    bm.free(0)                                   # room for the swap-in
+    new = bm.swap_in(1)
+    assert len(new) == n and set(new).isdisjoint(set(bm.block_table(10)))
+    in_pairs = torch.tensor([[i, b] for i, b in enumerate(new)], dtype=torch.int64, device="cuda")
+    binding.swap_in(host_k, host_v, k_pool, v_pool, in_pairs, dev_err=err)
+
+    bt2, ctx2, _, _ = device_tables(bm, [1, 2, 3])
+    after = binding.decode_split(q[1:], k_pool, v_pool, bt2, ctx2, w.scale, partition_tokens=32)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(after, before[1:])
+
+
+def test_swap_rejects_pageable_host_memory():
+    k = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16, device="cuda")
+    host = torch.zeros(2, 2, 16, 128, dtype=torch.bfloat16)      # not pinned
+    pairs = torch.tensor([[0, 0]], dtype=torch.int64, device="cuda")
+    with pytest.raises(binding.InvalidArgumentError):
+        binding.swap_out(k, k, host, host, pairs)

@@ -166,6 +166,9 @@ def random_ops(seed, n_ops=400, num_blocks=40, block_size=4, mbs=12):
         elif r < 0.85:
             # sliding window: release everything before a random token position
             ops.append(("release", int(rng.choice(live)), int(rng.integers(0, 4 * block_size * 2))))
+        elif r < 0.9:
+            # preemption by swap, and bringing a sequence back
+            ops.append((("swap_out", "swap_in")[int(rng.integers(0, 2))], int(rng.choice(live))))
         else:
             victim = int(rng.choice(live))
             ops.append(("free", victim))
@@ -193,6 +196,10 @@ def apply_op(bm, op):
             first = min(op[2], bm.context_len(op[1]))
             r = bm.release_before(op[1], first)
             return ("ok", len(r) if isinstance(r, list) else r)
+        elif kind == "swap_out":
+            return ("ok", tuple(bm.swap_out(op[1])))
+        elif kind == "swap_in":
+            return ("ok", tuple(bm.swap_in(op[1])))
         return ("ok", None)
     except NoFreeBlocks:
         return ("nofree", None)
@@ -283,3 +290,22 @@ def test_release_before_hand_example():
     bm.free(0)
     bm.free(1)
     assert sorted(bm.free_queue) == list(range(8))
+
+
+def test_swap_hand_example():
+    bm = BlockManager(6, 4, 4, [2, 5, 0, 1, 3, 4])
+    bm.allocate(0, 6)              # blocks 2, 5
+    bm.fork(0, 1)                  # shared
+    assert bm.swap_out(0) == [2, 5]          # still held by seq 1: nothing reclaimed
+    assert bm.block_table(0) == [-1, -1] and bm.context_len(0) == 6
+    assert list(bm.free_queue) == [0, 1, 3, 4]
+    with pytest.raises(InvalidArgument):
+        bm.append_slot(0)                    # swapped out
+    bm.allocate(2, 12)                       # takes 0, 1, 3
+    with pytest.raises(NoFreeBlocks):
+        bm.swap_in(0)                        # needs 2, one free: nothing changes
+    assert bm.block_table(0) == [-1, -1]
+    bm.free(1)                               # reclaims 2, 5
+    assert bm.swap_in(0) == [4, 2]           # private copies, in queue order
+    assert bm.refcount[4] == 1 and bm.refcount[2] == 1
+    assert bm.append_slot(0).slot == 2 * 4 + 2   # appends go on as before
