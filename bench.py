@@ -223,13 +223,15 @@ def profiled_traffic(workload: str):
 class DeviceStep:
     """Device-resident inputs of R consecutive decode steps, cycled."""
 
-    def __init__(self, w, states: int, partition_tokens: int, device, mode: str = "split"):
+    def __init__(self, w, states: int, partition_tokens: int, device, mode: str = "split",
+                 window: int = 0):
         import torch
         from paged_kv_cache_336_b200 import binding, workloads
         self.torch, self.binding = torch, binding
         self.w = w
         self.partition_tokens = partition_tokens
         self.mode = mode
+        self.window = window
         self.whole = mode == "whole"
         self.bm = binding.BlockManager(w.num_blocks, w.block_size, w.max_blocks_per_seq,
                                        w.free_order)
@@ -262,6 +264,8 @@ class DeviceStep:
             st["ctx_np"] = ctx.astype(np.int64)
             st["n_pairs"] = int(pairs.shape[0])
             st["decode_bytes"] = decode_bytes(w, st["ctx_np"])
+            if mode == "window":   # only the last `window` tokens are read
+                st["decode_bytes"] = decode_bytes(w, np.minimum(st["ctx_np"], self.window))
             st["unique_bytes"] = st["decode_bytes"]
             if mode == "shared_prefix":
                 offs, members, gblocks = self.bm.prefix_groups(w.decode_seqs)
@@ -301,6 +305,11 @@ class DeviceStep:
         if self.whole:
             b.decode(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"], self.w.scale,
                      out=self.out)
+        elif self.mode == "window":
+            b.decode_split_window(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"],
+                                  self.w.scale, self.window,
+                                  partition_tokens=self.partition_tokens, out=self.out,
+                                  workspace=self.ws)
         elif self.mode == "shared_prefix":
             b.decode_shared_prefix(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"],
                                    self.w.scale, st["groups"],
@@ -324,7 +333,7 @@ def run_ours(args, rank, world, device_index):
     torch.cuda.set_device(device)
     w = make_workload(args.workload, rank, args.batch)
     R = max(1, min(args.states, args.steps + args.warmup)) if args.workload != "prefix_cow" else 1
-    ds = DeviceStep(w, R, args.partition_tokens, device, mode=args.decode_mode)
+    ds = DeviceStep(w, R, args.partition_tokens, device, mode=args.decode_mode, window=args.window)
 
     for i in range(args.warmup):
         ds.run(i)
@@ -375,7 +384,9 @@ def run_ours(args, rank, world, device_index):
             "split": "pa_decode_split (paged_decode_kernel + lse_merge_kernel)",
             "whole": "pa_decode (paged_decode_kernel)",
             "shared_prefix": "pa_decode_shared_prefix (prefix_decode_kernel + paged_decode_kernel "
-                             "+ lse_merge_kernel)"}[args.decode_mode]
+                             "+ lse_merge_kernel)",
+            "window": f"pa_decode_split_window (window {args.window}; paged_decode_kernel + "
+                      "lse_merge_kernel)"}[args.decode_mode]
         result = {
             "metric": METRIC,
             "value": round(gbs, 2),
@@ -558,6 +569,46 @@ def run_reference(args, rank, world):
 
 # ---------------------------------------------------------------------------
 
+def run_swap_bench(args, device_index):
+    """Swap throughput: whole blocks of the workload's pool to pinned host
+    memory and back (pa_swap_out / pa_swap_in), CUDA-event timed."""
+    import torch
+    from paged_kv_cache_336_b200 import binding, workloads
+    device = torch.device("cuda", device_index)
+    torch.cuda.set_device(device)
+    w = make_workload(args.workload, 0, args.batch)
+    k_pool, v_pool = workloads.draw_pools(w, device)
+    nslots = min(2048, w.num_blocks)
+    host_k = torch.empty((nslots,) + tuple(k_pool.shape[1:]), dtype=k_pool.dtype).pin_memory()
+    host_v = torch.empty_like(host_k).pin_memory()
+    rng = np.random.default_rng(1)
+    blocks = torch.from_numpy(rng.permutation(w.num_blocks)[:nslots].astype(np.int64)).to(device)
+    slots = torch.arange(nslots, dtype=torch.int64, device=device)
+    out_pairs = torch.stack([blocks, slots], 1).contiguous()
+    in_pairs = torch.stack([slots, blocks], 1).contiguous()
+    block_bytes = k_pool[0].numel() * k_pool.element_size()
+    res = {}
+    for name, fn, pairs in (("swap_out", lambda p: binding.swap_out(k_pool, v_pool, host_k, host_v, p), out_pairs),
+                            ("swap_in", lambda p: binding.swap_in(host_k, host_v, k_pool, v_pool, p), in_pairs)):
+        for _ in range(args.warmup):
+            fn(pairs)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(3, min(args.steps, 50))
+        t0.record()
+        for _ in range(reps):
+            fn(pairs)
+        t1.record()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / reps
+        nbytes = 2 * nslots * block_bytes
+        res[name] = {"GB/s": round(nbytes / (ms * 1e-3) / 1e9, 2), "ms": round(ms, 4), "bytes": nbytes}
+    return {"metric": "swap of whole KV blocks between HBM and pinned host memory (K and V)",
+            "unit": "GB/s", "value": res["swap_out"]["GB/s"], "impl": "ours",
+            "config": {"workload": workload_label(w), "blocks": nslots,
+                       "block_bytes_each_pool": block_bytes}, **res}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -567,7 +618,11 @@ def main(argv=None):
     ap.add_argument("--workload", default="mha",
                     choices=["mha", "gqa", "prefix", "prefix_cow", "long16", "long32", "tiny"])
     ap.add_argument("--partition-tokens", type=int, default=512)
-    ap.add_argument("--decode-mode", choices=["split", "whole", "shared_prefix"], default="split",
+    ap.add_argument("--window", type=int, default=4096, help="window tokens for --decode-mode window")
+    ap.add_argument("--swap", action="store_true",
+                    help="measure pa_swap_out / pa_swap_in instead (extra JSON line)")
+    ap.add_argument("--decode-mode", choices=["split", "whole", "shared_prefix", "window"],
+                    default="split",
                     help="split: pa_decode_split (persistent, partitions + merge); "
                          "whole: pa_decode (one CTA per sequence and KV head); "
                          "shared_prefix: pa_decode_shared_prefix (shared prompt blocks read once)")
@@ -592,6 +647,10 @@ def main(argv=None):
 
     import torch
     import torch.distributed as dist
+    if args.swap:
+        if rank == 0:
+            print(json.dumps(run_swap_bench(args, local_rank)), flush=True)
+        return 0
     if world > 1:
         from datetime import timedelta
         torch.cuda.set_device(local_rank)
