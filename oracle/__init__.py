@@ -13,7 +13,8 @@ Modules
     Decode attention over a block-paged KV cache, written as its definition:
     gather each sequence's keys and values through its block table, then
     softmax(scale * K q) V in float64, two-pass (max, then exp/sum).
-    Also the sliding-window form (the last ``window`` tokens only), the
+    Also the causal prefill over the paged cache (many new tokens per
+    sequence), the sliding-window form (the last ``window`` tokens only), the
     partitioned form (per-partition max/sum/accumulator and a log-sum-exp
     merge), the KV-append scatter and the block copy, as plain array
     assignments.
@@ -41,6 +42,7 @@ from .paged_attention import (  # noqa: F401
     paged_decode,
     paged_decode_one,
     paged_decode_window,
+    paged_prefill,
     partitioned_decode_one,
     kv_append,
     copy_blocks,

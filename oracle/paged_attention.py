@@ -139,6 +139,43 @@ def paged_decode_window(q, k_pool, v_pool, block_tables, context_lens, scale: fl
     return out
 
 
+def paged_prefill(q, k_pool, v_pool, block_tables, context_lens, query_lens,
+                  scale: float) -> np.ndarray:
+    """Prefill (chunked prefill) attention over the paged cache, float64.
+
+    Sequence s holds context_lens[s] tokens, of which its last query_lens[s]
+    are new; their queries are rows query_start[s] .. of ``q``
+    ``[total_new_tokens, num_q_heads, head_dim]`` (sequences back to back).
+    New token i of sequence s sits at position p = ctx_s - qlen_s + i and
+    attends to tokens 0 .. p of its sequence (causal). Prefill is the step
+    that writes a request's first KV blocks before decoding ("What is
+    PagedAttention?", How It Works: prefill allocates enough blocks for the
+    input); the attention itself is the plain causal definition.
+    """
+    q = np.asarray(q)
+    total, num_q_heads, head_dim = q.shape
+    num_kv_heads = np.asarray(k_pool).shape[1]
+    group = _group(num_q_heads, num_kv_heads)
+    out = np.zeros((total, num_q_heads, head_dim), dtype=np.float64)
+    row = 0
+    for s in range(len(context_lens)):
+        ctx = int(context_lens[s])
+        qlen = int(query_lens[s])
+        if qlen > ctx:
+            raise ValueError("query_lens[s] must not exceed context_lens[s]")
+        Ks = [gather_sequence(k_pool, block_tables[s], ctx, kvh) for kvh in range(num_kv_heads)]
+        Vs = [gather_sequence(v_pool, block_tables[s], ctx, kvh) for kvh in range(num_kv_heads)]
+        for i in range(qlen):
+            pos = ctx - qlen + i
+            for h in range(num_q_heads):
+                out[row, h] = attention_definition(q[row, h], Ks[h // group][:pos + 1],
+                                                   Vs[h // group][:pos + 1], scale)
+            row += 1
+    if row != total:
+        raise ValueError("sum of query_lens must equal q.shape[0]")
+    return out
+
+
 def partitioned_decode_one(q, k_pool, v_pool, block_tables, context_lens, scale: float,
                            seq: int, q_head: int, partition_tokens: int) -> np.ndarray:
     """Split-context route to the same result, step by step, float64.

@@ -7,6 +7,8 @@ identical keys). Tolerances: fp32 max-abs 1e-5; bf16 max-abs 2e-2 and
 mean-abs 2e-3 against the float64 oracle. Append and copy are bit-exact.
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -324,3 +326,37 @@ def test_repeated_split_calls_reuse_workspace():
         assert torch.equal(o, outs[0])
     want = _full_oracle(q, k_pool, v_pool, tables, ctx_np, w.scale)
     check_close(to_f64(outs[0]), want, w.dtype, "reused workspace")
+
+
+def test_host_validation_flag_rejects_bad_tables():
+    """PAGEDKV_VALIDATE=1 copies the tables and lengths to the host and rejects
+    an out-of-range entry before launching (the flag is read once per
+    process, so the check runs in a child)."""
+    import subprocess
+    import sys
+    import textwrap
+    code = textwrap.dedent("""
+        import sys, torch
+        sys.path.insert(0, %r)
+        sys.path.insert(0, %r)
+        from paged_kv_cache_336_b200 import binding, workloads
+        from gpu_util import setup, device_tables
+        w = workloads.random_small(3, num_seqs=3, num_q_heads=4, num_kv_heads=2, head_dim=128,
+                                   block_size=16, dtype=workloads.BF16, max_ctx=60, min_ctx=20)
+        bm, k, v = setup(w)
+        q = workloads.draw_queries(w, 3, device="cuda")
+        bt, ctx, _, _ = device_tables(bm, [0, 1, 2])
+        binding.decode(q, k, v, bt, ctx, w.scale)          # valid tables pass
+        bt[1, 0] = w.num_blocks + 3
+        try:
+            binding.decode_split(q, k, v, bt, ctx, w.scale, partition_tokens=32)
+        except binding.InvalidArgumentError as e:
+            assert "block_tables[1][0]" in str(e), e
+            print("rejected")
+    """) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+            os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PAGEDKV_VALIDATE="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert "rejected" in r.stdout

@@ -268,3 +268,37 @@ def test_window_matches_sdpa_on_the_slice(window):
     for s, n in enumerate(lens):
         t2[s, :max(0, n - window) // 16] = -1
     assert np.array_equal(oracle.paged_decode_window(q, k_pool, v_pool, t2, np.array(lens), 0.25, window), got)
+
+
+def test_prefill_single_new_token_is_decode():
+    rng = np.random.default_rng(12)
+    k_pool = rng.standard_normal((8, 2, 16, 8))
+    v_pool = rng.standard_normal((8, 2, 16, 8))
+    tables = np.array([[1, 5, 2], [7, 0, -1]])
+    lens = np.array([40, 17])
+    q = rng.standard_normal((2, 4, 8))
+    got = oracle.paged_prefill(q, k_pool, v_pool, tables, lens, [1, 1], 0.3)
+    want = oracle.paged_decode(q, k_pool, v_pool, tables, lens, 0.3)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("prior,qlen", [(0, 7), (0, 33), (21, 12), (50, 1)])
+def test_prefill_matches_sdpa_with_causal_mask(prior, qlen):
+    rng = np.random.default_rng(13 + prior + qlen)
+    ctx = prior + qlen
+    contig_k = [rng.standard_normal((ctx, 2, 16))]
+    contig_v = [rng.standard_normal((ctx, 2, 16))]
+    k_pool, v_pool, tables = _place(contig_k, contig_v, 16, 12, rng)
+    q = rng.standard_normal((qlen, 4, 16))
+    got = oracle.paged_prefill(q, k_pool, v_pool, tables, [ctx], [qlen], 0.25)
+    # SDPA over the contiguous sequence with an explicit causal mask
+    K = torch.from_numpy(contig_k[0]).permute(1, 0, 2).repeat_interleave(2, dim=0)   # [Hq, ctx, D]
+    V = torch.from_numpy(contig_v[0]).permute(1, 0, 2).repeat_interleave(2, dim=0)
+    Q = torch.from_numpy(q).permute(1, 0, 2)                                          # [Hq, qlen, D]
+    pos = torch.arange(prior, ctx).unsqueeze(1)
+    mask = torch.arange(ctx).unsqueeze(0) <= pos                                      # [qlen, ctx]
+    want = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask, scale=0.25)
+    np.testing.assert_allclose(got, want.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+    if prior == 0:
+        causal = torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=True, scale=0.25)
+        np.testing.assert_allclose(got, causal.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
