@@ -569,6 +569,63 @@ def run_reference(args, rank, world):
 
 # ---------------------------------------------------------------------------
 
+def run_prefill_bench(args, device_index):
+    """Chunked-prefill attention (pa_prefill) on a synthetic batch: every
+    sequence has `prior` tokens of earlier context and `chunk` new tokens
+    (already appended). Reports causal-attention TFLOP/s (4*D per (query,
+    key, head) pair: q.k and p.v, 2 flops per multiply-add) against the
+    measured bf16 tensor peak, and the KV bytes read per call."""
+    import torch
+    from paged_kv_cache_336_b200 import binding, workloads
+    device = torch.device("cuda", device_index)
+    torch.cuda.set_device(device)
+    B, prior, chunk, Hq, Hkv, D, bs = 16, args.prefill_prior, args.prefill_chunk, 32, 8, 128, 16
+    ctx = np.full(B, prior + chunk, dtype=np.int64)
+    w = workloads.random_small(500, num_seqs=B, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                               block_size=bs, dtype=workloads.BF16, max_ctx=prior + chunk,
+                               fixed_lens=ctx.tolist())
+    bm = binding.BlockManager(w.num_blocks, bs, w.max_blocks_per_seq, w.free_order)
+    for s_ in range(B):
+        bm.allocate(s_, int(ctx[s_]))
+    k_pool, v_pool = workloads.draw_pools(w, device)
+    tables, ctx32 = bm.export(list(range(B)))
+    bt = torch.from_numpy(tables).to(device)
+    qlen = np.full(B, chunk, dtype=np.int32)
+    q = workloads.draw_normal((B * chunk, Hq, D), workloads.BF16, 501, device)
+    out = torch.empty_like(q)
+    ws = binding.prefill_workspace(B, B * chunk, Hq, Hkv, D, bs, w.max_blocks_per_seq,
+                                   args.partition_tokens, device)
+    for _ in range(args.warmup):
+        binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, args.partition_tokens, out, ws)
+    torch.cuda.synchronize()
+    reps = max(3, min(args.steps, 200))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(reps):
+        binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, args.partition_tokens, out, ws)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / reps
+    pairs = B * int(np.sum(np.arange(prior + 1, prior + chunk + 1)))   # (query, key) pairs per head
+    flops = 4.0 * D * Hq * pairs
+    tflops = flops / (ms * 1e-3) / 1e12
+    try:
+        peak = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
+        kind = "measured (cuBLAS bf16 burst)"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    kv_bytes = B * (prior + chunk) * Hkv * D * 2 * 2
+    return {"metric": "paged chunked-prefill attention TFLOP/s (causal, bf16 in, fp32 accumulate)",
+            "value": round(tflops, 2), "unit": "TFLOP/s", "impl": "ours", "ms_per_call": round(ms, 4),
+            "config": {"workload": f"prefill: batch {B}, {prior} prior + {chunk} new tokens, "
+                                   f"{Hq}q/{Hkv}kv heads, head_dim {D}, bf16, block {bs}",
+                       "partition_tokens": args.partition_tokens},
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
+                         "peak_kind": kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                         "kv_bytes_per_call": kv_bytes,
+                         "kv_GBs": round(kv_bytes / (ms * 1e-3) / 1e9, 1)}}
+
+
 def run_swap_bench(args, device_index):
     """Swap throughput: whole blocks of the workload's pool to pinned host
     memory and back (pa_swap_out / pa_swap_in), CUDA-event timed."""
@@ -621,6 +678,10 @@ def main(argv=None):
     ap.add_argument("--window", type=int, default=4096, help="window tokens for --decode-mode window")
     ap.add_argument("--swap", action="store_true",
                     help="measure pa_swap_out / pa_swap_in instead (extra JSON line)")
+    ap.add_argument("--prefill", action="store_true",
+                    help="measure pa_prefill instead (extra JSON line)")
+    ap.add_argument("--prefill-prior", type=int, default=1024)
+    ap.add_argument("--prefill-chunk", type=int, default=1024)
     ap.add_argument("--decode-mode", choices=["split", "whole", "shared_prefix", "window"],
                     default="split",
                     help="split: pa_decode_split (persistent, partitions + merge); "
@@ -650,6 +711,10 @@ def main(argv=None):
     if args.swap:
         if rank == 0:
             print(json.dumps(run_swap_bench(args, local_rank)), flush=True)
+        return 0
+    if args.prefill:
+        if rank == 0:
+            print(json.dumps(run_prefill_bench(args, local_rank)), flush=True)
         return 0
     if world > 1:
         from datetime import timedelta

@@ -234,6 +234,37 @@ pa_status_t pa_decode_split_window(const void* q, const void* k_pool, const void
                                    void* stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_prefill - causal (chunked) prefill attention over the paged cache.
+ * Sequence s holds context_lens[s] tokens, the last query_lens[s] of them
+ * new (their K and V already written, e.g. by pa_kv_append); its queries are
+ * rows query_start .. query_start + query_lens[s] - 1 of q
+ * [total_q][num_q_heads][head_dim] (sequences back to back, total_q = sum of
+ * query_lens). New token i at position p = ctx - qlen + i attends to tokens
+ * 0..p of its sequence through its block table; out has q's layout. Prefill
+ * is the step that fills a request's first blocks ([Q] How It Works: prefill
+ * allocates enough blocks for the input).
+ *
+ * context_lens and query_lens are HOST arrays here (the host plans the
+ * tiles); block tables are device memory. bf16 only. Tiles of 64 query rows
+ * (query tokens x heads of one KV head) each read their KV once per
+ * partition of partition_tokens tokens; tiles spanning several partitions
+ * are joined by the log-sum-exp merge. workspace: at least
+ * pa_prefill_workspace_size(...) bytes, 256-byte aligned, initialised once
+ * with pa_decode_split_workspace_init.
+ * ------------------------------------------------------------------------- */
+size_t pa_prefill_workspace_size(int num_seqs, int total_q, int num_q_heads, int num_kv_heads,
+                                 int head_dim, int block_size, int max_blocks_per_seq,
+                                 int partition_tokens);
+
+pa_status_t pa_prefill(const void* q, const void* k_pool, const void* v_pool,
+                       const int32_t* block_tables, const int32_t* context_lens,
+                       const int32_t* query_lens, int num_seqs, int total_q, int num_q_heads,
+                       int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                       int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                       int partition_tokens, void* workspace, size_t workspace_bytes, void* out,
+                       uint32_t* dev_err, void* stream);
+
+/* ---------------------------------------------------------------------------
  * pa_swap_out / pa_swap_in - the data movement of swapping: whole blocks
  * (K and V, all heads; block_bytes each) between the device pools and two
  * host buffers of num_host_slots blocks each. pairs (device int64

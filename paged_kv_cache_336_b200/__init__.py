@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     decode_split,
     decode_split_window,
     decode_shared_prefix,
+    prefill,
     decode_split_workspace_size,
     kv_append,
     copy_blocks,

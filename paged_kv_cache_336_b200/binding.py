@@ -94,6 +94,9 @@ _SIGNATURES = {
                                      _I, _P, _P, _P, _P, _SZ, _P, _P, _P]),
     "pa_bm_prefix_groups": (_I, [_P, _P, _I, _I, _P, _P, _P, ctypes.POINTER(_I)]),
     "pa_bm_release_before": (_I, [_P, _I64, _I64, ctypes.POINTER(_I)]),
+    "pa_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "pa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P,
+                        _SZ, _P, _P, _P]),
     "pa_bm_swap_out": (_I, [_P, _I64, _P, _I, ctypes.POINTER(_I)]),
     "pa_bm_swap_in": (_I, [_P, _I64, _P, _I, ctypes.POINTER(_I)]),
     "pa_swap_out": (_I, [_P, _P, _P, _P, _P, _I, _SZ, _I, _I, _P, _P]),
@@ -299,6 +302,41 @@ def swap_out(k_pool, v_pool, host_k, host_v, pairs, dev_err=None, stream=None):
 def swap_in(host_k, host_v, k_pool, v_pool, pairs, dev_err=None, stream=None):
     """pa_swap_in: pairs (host slot, device block) copy whole blocks back to the pools."""
     _swap("pa_swap_in", host_k, host_v, k_pool, v_pool, pairs, k_pool, host_k, dev_err, stream)
+
+
+def prefill_workspace(num_seqs, total_q, num_q_heads, num_kv_heads, head_dim, block_size,
+                      max_blocks_per_seq, partition_tokens, device=None) -> "Workspace":
+    n = library().pa_prefill_workspace_size(num_seqs, total_q, num_q_heads, num_kv_heads, head_dim,
+                                            block_size, max_blocks_per_seq, partition_tokens)
+    if n == 0:
+        raise InvalidArgumentError(PA_ERR_INVALID_ARG, "bad workspace size arguments")
+    return Workspace(n, device)
+
+
+def prefill(q, k_pool, v_pool, block_tables, context_lens, query_lens, scale: float,
+            partition_tokens: int = 2048, out=None, workspace=None, dev_err=None, stream=None):
+    """pa_prefill: causal attention of each sequence's last query_lens[s]
+    tokens over its paged context. context_lens / query_lens: host int32
+    arrays; q, out: [sum(query_lens), num_q_heads, head_dim]."""
+    import numpy as np
+    torch = _torch()
+    _require_cuda(q, k_pool, v_pool, block_tables)
+    if out is None:
+        out = torch.empty_like(q)
+    ctx = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    qlen = np.ascontiguousarray(np.asarray(query_lens, dtype=np.int32))
+    total, Hq, D = q.shape
+    NB, Hkv, BS, _ = k_pool.shape
+    B, MBS = block_tables.shape
+    if block_tables.dtype != torch.int32 or ctx.shape != (B,) or qlen.shape != (B,):
+        raise InvalidArgumentError(PA_ERR_INVALID_ARG, "bad tables or length arrays")
+    if workspace is None:
+        workspace = prefill_workspace(B, total, Hq, Hkv, D, BS, MBS, partition_tokens, q.device)
+    _check(library().pa_prefill(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), ctx.ctypes.data, qlen.ctypes.data,
+        B, total, Hq, Hkv, D, BS, NB, MBS, float(scale), _dtype_code(q), int(partition_tokens),
+        workspace.ptr, workspace.nbytes, _ptr(out), _ptr(dev_err), _stream_ptr(stream)))
+    return out
 
 
 class Workspace:

@@ -15,6 +15,7 @@
 #include "decode_dispatch.h"
 #include "decode_kernel.cuh"
 #include "pa_internal.h"
+#include "prefill_kernel.cuh"
 #include "prefix_kernel.cuh"
 
 namespace pagedkv {
@@ -580,6 +581,155 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
   return run_decode(r, true, partition_tokens, workspace, workspace_bytes, &ex);
 }
 
+// ---- paged prefill -------------------------------------------------------------------
+// Workspace: [0,256) header | merge_lens int32 [total_q] | items PrefillItem
+// [max_items] | m, l float [total_q][Hq][pmax] | acc float [...][head_dim],
+// pmax = ceil(max_blocks_per_seq / partition blocks).
+struct PrefillLayout {
+  size_t lens_off, items_off, m_off, l_off, acc_off, total, max_items;
+  int pmax;
+};
+
+PrefillLayout prefill_layout(int num_seqs, int total_q, int num_q_heads, int num_kv_heads,
+                             int head_dim, int block_size, int max_blocks_per_seq,
+                             int partition_tokens) {
+  PrefillLayout L{};
+  const int pb = partition_tokens / block_size;
+  L.pmax = (max_blocks_per_seq + pb - 1) / pb;
+  const int G = std::max(1, num_q_heads / std::max(1, num_kv_heads));
+  const int tq = std::max(1, kPrefixRows / G);
+  const size_t tiles = static_cast<size_t>(total_q) / tq + num_seqs;
+  L.max_items = tiles * num_kv_heads * L.pmax;
+  L.lens_off = kWorkspaceHeader;
+  L.items_off = L.lens_off + align256(static_cast<size_t>(total_q) * 4);
+  const size_t rows = static_cast<size_t>(total_q) * num_q_heads * L.pmax;
+  L.m_off = L.items_off + align256(L.max_items * sizeof(PrefillItem));
+  L.l_off = L.m_off + align256(rows * 4);
+  L.acc_off = L.l_off + align256(rows * 4);
+  L.total = L.acc_off + align256(rows * static_cast<size_t>(head_dim) * 4);
+  return L;
+}
+
+pa_status_t run_prefill(const DecodeReq& r, const int32_t* ctx_host, const int32_t* qlen_host,
+                        int total_q, int partition_tokens, void* workspace, size_t workspace_bytes) {
+  DecodeInstance inst;
+  pa_status_t st = validate_and_pick(r, &inst);  // shapes, alignment, dtype, group (merge kernel)
+  if (st != PA_OK) return st;
+  if (r.dtype != PA_BF16) return fail(PA_ERR_UNSUPPORTED, "pa_prefill is bf16 only");
+  PrefixInstance pinst;
+  if (!find_prefill_bf16(r.head_dim, r.block_size, &pinst))
+    return fail(PA_ERR_UNSUPPORTED, "no prefill kernel for head_dim=%d block_size=%d", r.head_dim,
+                r.block_size);
+  if (partition_tokens <= 0 || partition_tokens % r.block_size != 0)
+    return fail(PA_ERR_INVALID_ARG, "partition_tokens (%d) must be a positive multiple of block_size",
+                partition_tokens);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PA_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (total_q < 0) return fail(PA_ERR_INVALID_ARG, "total_q < 0");
+  const int B = r.num_seqs;
+  if (B > 0 && (ctx_host == nullptr || qlen_host == nullptr))
+    return fail(PA_ERR_INVALID_ARG, "context_lens and query_lens (host) are required");
+  int64_t sum_q = 0;
+  for (int s = 0; s < B; ++s) {
+    if (qlen_host[s] < 0 || ctx_host[s] < qlen_host[s] ||
+        static_cast<int64_t>(ctx_host[s]) > static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size)
+      return fail(PA_ERR_INVALID_ARG, "sequence %d: query_len %d, context_len %d out of range", s,
+                  qlen_host[s], ctx_host[s]);
+    sum_q += qlen_host[s];
+  }
+  if (sum_q != total_q) return fail(PA_ERR_INVALID_ARG, "sum of query_lens %lld != total_q %d",
+                                    (long long)sum_q, total_q);
+  const PrefillLayout L = prefill_layout(B, total_q, r.num_q_heads, r.num_kv_heads, r.head_dim,
+                                         r.block_size, r.max_blocks_per_seq, partition_tokens);
+  if (workspace_bytes < L.total)
+    return fail(PA_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", workspace_bytes, L.total);
+  if (total_q == 0) return ok();
+
+  const int G = r.num_q_heads / r.num_kv_heads;
+  const int tq = std::max(1, kPrefixRows / G);
+  const int pb = partition_tokens / r.block_size;
+  thread_local std::vector<int32_t> lens;
+  thread_local std::vector<PrefillItem> items;
+  lens.assign(total_q, 0);
+  items.clear();
+  bool any_split = false;
+  int q_base = 0;
+  for (int s = 0; s < B; ++s) {
+    const int qlen = qlen_host[s], ctx = ctx_host[s];
+    for (int t = 0; t < qlen; t += tq) {
+      const int count = std::min(tq, qlen - t);
+      const int p0 = ctx - qlen + t;
+      const int kv_end = p0 + count;  // last position + 1
+      const int nblk = (kv_end + r.block_size - 1) / r.block_size;
+      const int nparts = (nblk + pb - 1) / pb;
+      any_split = any_split || nparts > 1;
+      for (int i = 0; i < count; ++i) lens[q_base + t + i] = kv_end;
+      for (int h = 0; h < r.num_kv_heads; ++h)
+        for (int p = 0; p < nparts; ++p)
+          items.push_back(PrefillItem{s, q_base + t, count, p0, p * pb, std::min(nblk, (p + 1) * pb),
+                                      kv_end, h, p, nparts == 1 ? 1 : 0, 0, 0});
+    }
+    q_base += qlen;
+  }
+  if (items.size() > L.max_items) return fail(PA_ERR_INVALID_ARG, "too many prefill items");
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaError_t err;
+  if ((err = cudaMemcpyAsync(ws + L.lens_off, lens.data(), lens.size() * 4, cudaMemcpyHostToDevice,
+                             r.stream)) != cudaSuccess ||
+      (err = cudaMemcpyAsync(ws + L.items_off, items.data(), items.size() * sizeof(PrefillItem),
+                             cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
+    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
+  st = prepare_kernel(pinst.kernel, pinst.smem);
+  if (st != PA_OK) return st;
+  const int rows = r.num_blocks * r.num_kv_heads * r.block_size;
+  CUtensorMap tmk, tmv;
+  st = pool_tensor_map(r.k_pool, rows, r.head_dim, r.block_size, r.dtype, &tmk);
+  if (st != PA_OK) return st;
+  st = pool_tensor_map(r.v_pool, rows, r.head_dim, r.block_size, r.dtype, &tmv);
+  if (st != PA_OK) return st;
+  PrefillArgs pf{};
+  DecodeArgs& a = pf.d;
+  a.q = r.q;
+  a.out = r.out;
+  a.block_tables = r.block_tables;
+  a.context_lens = reinterpret_cast<const int32_t*>(ws + L.lens_off);  // per query token (merge)
+  a.part_m = reinterpret_cast<float*>(ws + L.m_off);
+  a.part_l = reinterpret_cast<float*>(ws + L.l_off);
+  a.part_acc = reinterpret_cast<float*>(ws + L.acc_off);
+  a.dev_err = r.dev_err;
+  a.num_seqs = total_q;  // the merge walks (query token, head) rows
+  a.num_q_heads = r.num_q_heads;
+  a.num_kv_heads = r.num_kv_heads;
+  a.group = G;
+  a.num_blocks = r.num_blocks;
+  a.max_blocks_per_seq = r.max_blocks_per_seq;
+  a.partition_blocks = pb;
+  a.max_partitions = L.pmax;
+  a.scale_log2 = r.scale * 1.4426950408889634f;
+  pf.items = reinterpret_cast<const PrefillItem*>(ws + L.items_off);
+  void* args[] = {&tmk, &tmv, &pf};
+  err = cudaLaunchKernel(pinst.kernel, dim3(static_cast<unsigned>(items.size())), dim3(pinst.threads),
+                         args, pinst.smem, r.stream);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(err));
+  if (any_split) {
+    int bs = r.block_size;
+    void* margs[] = {&a, &bs};
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(total_q) * r.num_q_heads);
+    cfg.blockDim = dim3(128);
+    cfg.stream = r.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelExC(&cfg, inst.merge, margs);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "merge launch: %s", cudaGetErrorString(err));
+  }
+  return launch_error("prefill");
+}
+
 // ---- scratch for pa_decode_split_static ------------------------------------------
 // Callers that cannot allocate device memory get their split-decode scratch
 // (ticket counters + per-partition partials) from this fixed array instead of
@@ -740,6 +890,34 @@ pa_status_t pa_decode_split_window(const void* q, const void* k_pool, const void
   SplitExtras ex;
   ex.window = window;
   return run_decode(r, true, partition_tokens, workspace, workspace_bytes, &ex);
+}
+
+size_t pa_prefill_workspace_size(int num_seqs, int total_q, int num_q_heads, int num_kv_heads,
+                                 int head_dim, int block_size, int max_blocks_per_seq,
+                                 int partition_tokens) {
+  if (num_seqs < 0 || total_q < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || max_blocks_per_seq <= 0 || partition_tokens <= 0 ||
+      partition_tokens % block_size != 0)
+    return 0;
+  return prefill_layout(num_seqs, total_q, num_q_heads, num_kv_heads, head_dim, block_size,
+                        max_blocks_per_seq, partition_tokens)
+      .total;
+}
+
+pa_status_t pa_prefill(const void* q, const void* k_pool, const void* v_pool,
+                       const int32_t* block_tables, const int32_t* context_lens,
+                       const int32_t* query_lens, int num_seqs, int total_q, int num_q_heads,
+                       int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                       int max_blocks_per_seq, float scale, pa_dtype_t dtype,
+                       int partition_tokens, void* workspace, size_t workspace_bytes, void* out,
+                       uint32_t* dev_err, void* stream) {
+  // validate_and_pick checks the device-side shapes; context_lens here is a
+  // host array, so a placeholder non-null device pointer is not needed.
+  DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+              head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
+              static_cast<cudaStream_t>(stream)};
+  return run_prefill(r, context_lens, query_lens, total_q, partition_tokens, workspace,
+                     workspace_bytes);
 }
 
 }  // extern "C"

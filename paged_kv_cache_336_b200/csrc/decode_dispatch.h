@@ -29,5 +29,7 @@ struct PrefixInstance {
 
 // Shared-prefix pass kernels (bf16); false when (head_dim, block_size) has none.
 bool find_prefix_bf16(int head_dim, int block_size, PrefixInstance* out);
+// Paged prefill kernels (bf16); same shapes, same instance record.
+bool find_prefill_bf16(int head_dim, int block_size, PrefixInstance* out);
 
 }  // namespace pagedkv

@@ -10,6 +10,7 @@
 //    wide): each warp walks more units of an item per fill and drain.
 #include "decode_dispatch.h"
 #include "decode_kernel.cuh"
+#include "prefill_kernel.cuh"
 #include "prefix_kernel.cuh"
 
 namespace pagedkv {
@@ -63,6 +64,24 @@ bool find_prefix_bf16(int head_dim, int block_size, PrefixInstance* out) {
   if (block_size == 16 && head_dim == 128) { *out = make_prefix<16, 128>(); return true; }
   if (block_size == 32 && head_dim == 64) { *out = make_prefix<32, 64>(); return true; }
   if (block_size == 32 && head_dim == 128) { *out = make_prefix<32, 128>(); return true; }
+  return false;
+}
+
+template <int BS, int D>
+static PrefixInstance make_prefill() {
+  using Cfg = PrefixCfg<BS, D>;
+  PrefixInstance r;
+  r.kernel = reinterpret_cast<const void*>(&prefill_kernel<Cfg>);
+  r.threads = Cfg::kThreads;
+  r.smem = Cfg::kSmem;
+  return r;
+}
+
+bool find_prefill_bf16(int head_dim, int block_size, PrefixInstance* out) {
+  if (block_size == 16 && head_dim == 64) { *out = make_prefill<16, 64>(); return true; }
+  if (block_size == 16 && head_dim == 128) { *out = make_prefill<16, 128>(); return true; }
+  if (block_size == 32 && head_dim == 64) { *out = make_prefill<32, 64>(); return true; }
+  if (block_size == 32 && head_dim == 128) { *out = make_prefill<32, 128>(); return true; }
   return false;
 }
 

@@ -307,9 +307,14 @@ struct MmaWarp {
   // and the max/sum shuffles are paid once per U*16 tokens. Tokens
   // nfirst <= t < nvalid of the span (counted from its first token) take
   // part; the caller guarantees at least one.
-  template <int U>
+  //
+  // kRowLimits (causal prefill): in addition, token t counts for fragment row
+  // g only while t <= lim0 and for row g+8 only while t <= lim1; a row with
+  // no token in the span keeps its state (guards against -inf - -inf).
+  template <int U, bool kRowLimits = false>
   __device__ __forceinline__ void block_units(const uint8_t* const (&kts)[U], uint8_t* const (&vts)[U],
-                                              int nfirst, int nvalid, int lane) {
+                                              int nfirst, int nvalid, int lane, int lim0 = 0,
+                                              int lim1 = 0) {
     const int t4 = lane & 3;
     const int mj = lane >> 3;  // which 8x8 matrix this lane addresses
     const int mr = lane & 7;   // which row of it
@@ -341,7 +346,9 @@ struct MmaWarp {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int tok = n * 8 + 2 * t4 + (e & 1);
-        s[n][e] = (tok >= nfirst && tok < nvalid) ? s[n][e] * scale_log2 : -INFINITY;
+        bool in = tok >= nfirst && tok < nvalid;
+        if constexpr (kRowLimits) in = in && tok <= ((e < 2) ? lim0 : lim1);
+        s[n][e] = in ? s[n][e] * scale_log2 : -INFINITY;
       }
       mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][1]));
       mx1 = fmaxf(mx1, fmaxf(s[n][2], s[n][3]));
@@ -350,12 +357,23 @@ struct MmaWarp {
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m[0], mx0);
-    const float mn1 = fmaxf(m[1], mx1);
-    const float a0 = fast_exp2(m[0] - mn0);
-    const float a1 = fast_exp2(m[1] - mn1);
+    float mn0 = fmaxf(m[0], mx0);
+    float mn1 = fmaxf(m[1], mx1);
+    float a0, a1;
+    if constexpr (kRowLimits) {
+      // A row with nothing valid so far has mn == -inf: keep alpha 1, p 0.
+      a0 = (mn0 == -INFINITY) ? 1.f : fast_exp2(m[0] - mn0);
+      a1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m[1] - mn1);
+    } else {
+      a0 = fast_exp2(m[0] - mn0);
+      a1 = fast_exp2(m[1] - mn1);
+    }
     m[0] = mn0;
     m[1] = mn1;
+    if constexpr (kRowLimits) {
+      if (mn0 == -INFINITY) mn0 = 0.f;   // every s of the row is -inf: 2^(-inf) = 0
+      if (mn1 == -INFINITY) mn1 = 0.f;
+    }
     float r0 = 0.f, r1 = 0.f;
 #pragma unroll
     for (int n = 0; n < NTU; ++n) {
@@ -416,6 +434,27 @@ struct MmaWarp {
           mma_bf16_16816(o[2 * nd + 1], pa, b2, b3);
         }
       }
+    }
+  }
+
+  // Writes rows g and g+8 as final outputs (acc / l, bf16) to out0 / out1
+  // when valid0 / valid1; a row with l == 0 gets zeros.
+  __device__ __forceinline__ void store_final(__nv_bfloat16* out0, __nv_bfloat16* out1, bool valid0,
+                                              bool valid1, int lane) {
+    const int t4 = lane & 3;
+    float l0 = l[0], l1 = l[1];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
+    const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+#pragma unroll
+    for (int n = 0; n < ND; ++n) {
+      if (valid0)
+        *reinterpret_cast<uint32_t*>(out0 + n * 8 + 2 * t4) = pack_bf16x2(o[n][0] * i0, o[n][1] * i0);
+      if (valid1)
+        *reinterpret_cast<uint32_t*>(out1 + n * 8 + 2 * t4) = pack_bf16x2(o[n][2] * i1, o[n][3] * i1);
     }
   }
 
