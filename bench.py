@@ -593,16 +593,16 @@ def run_prefill_bench(args, device_index):
     qlen = np.full(B, chunk, dtype=np.int32)
     q = workloads.draw_normal((B * chunk, Hq, D), workloads.BF16, 501, device)
     out = torch.empty_like(q)
-    ws = binding.prefill_workspace(B, B * chunk, Hq, Hkv, D, bs, w.max_blocks_per_seq,
-                                   args.partition_tokens, device)
+    part = args.prefill_partition or -(-(prior + chunk) // bs) * bs
+    ws = binding.prefill_workspace(B, B * chunk, Hq, Hkv, D, bs, w.max_blocks_per_seq, part, device)
     for _ in range(args.warmup):
-        binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, args.partition_tokens, out, ws)
+        binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, part, out, ws)
     torch.cuda.synchronize()
     reps = max(3, min(args.steps, 200))
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
     for _ in range(reps):
-        binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, args.partition_tokens, out, ws)
+        binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, part, out, ws)
     t1.record()
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / reps
@@ -619,7 +619,8 @@ def run_prefill_bench(args, device_index):
             "value": round(tflops, 2), "unit": "TFLOP/s", "impl": "ours", "ms_per_call": round(ms, 4),
             "config": {"workload": f"prefill: batch {B}, {prior} prior + {chunk} new tokens, "
                                    f"{Hq}q/{Hkv}kv heads, head_dim {D}, bf16, block {bs}",
-                       "partition_tokens": args.partition_tokens},
+                       "partition_tokens": part,
+                       "kernel": os.environ.get("PAGEDKV_PREFILL_KERNEL", "tcgen05")},
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                          "peak_kind": kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
                          "kv_bytes_per_call": kv_bytes,
@@ -682,6 +683,8 @@ def main(argv=None):
                     help="measure pa_prefill instead (extra JSON line)")
     ap.add_argument("--prefill-prior", type=int, default=1024)
     ap.add_argument("--prefill-chunk", type=int, default=1024)
+    ap.add_argument("--prefill-partition", type=int, default=0,
+                    help="KV partition of pa_prefill in tokens; 0: the whole context (no merge)")
     ap.add_argument("--decode-mode", choices=["split", "whole", "shared_prefix", "window"],
                     default="split",
                     help="split: pa_decode_split (persistent, partitions + merge); "

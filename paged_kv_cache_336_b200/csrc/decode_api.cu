@@ -616,8 +616,12 @@ pa_status_t run_prefill(const DecodeReq& r, const int32_t* ctx_host, const int32
   pa_status_t st = validate_and_pick(r, &inst);  // shapes, alignment, dtype, group (merge kernel)
   if (st != PA_OK) return st;
   if (r.dtype != PA_BF16) return fail(PA_ERR_UNSUPPORTED, "pa_prefill is bf16 only");
+  // PAGEDKV_PREFILL_KERNEL=mma_sync selects the 64-row mma.sync kernel (kept
+  // for comparison); the default is the tcgen05 kernel.
+  const char* kname = std::getenv("PAGEDKV_PREFILL_KERNEL");
+  const bool tcgen05 = kname == nullptr || std::strcmp(kname, "mma_sync") != 0;
   PrefixInstance pinst;
-  if (!find_prefill_bf16(r.head_dim, r.block_size, &pinst))
+  if (!find_prefill_bf16(r.head_dim, r.block_size, tcgen05, &pinst))
     return fail(PA_ERR_UNSUPPORTED, "no prefill kernel for head_dim=%d block_size=%d", r.head_dim,
                 r.block_size);
   if (partition_tokens <= 0 || partition_tokens % r.block_size != 0)
@@ -646,7 +650,7 @@ pa_status_t run_prefill(const DecodeReq& r, const int32_t* ctx_host, const int32
   if (total_q == 0) return ok();
 
   const int G = r.num_q_heads / r.num_kv_heads;
-  const int tq = std::max(1, kPrefixRows / G);
+  const int tq = std::max(1, pinst.rows / G);  // query tokens per tile
   const int pb = partition_tokens / r.block_size;
   thread_local std::vector<int32_t> lens;
   thread_local std::vector<PrefillItem> items;

@@ -22,14 +22,16 @@ bool find_decode_f32(int head_dim, int block_size, int group, DecodeInstance* ou
 bool find_decode_bf16_mma(int head_dim, int block_size, bool deep, DecodeInstance* out);
 
 struct PrefixInstance {
-  const void* kernel = nullptr;  // prefix_decode_kernel<PrefixCfg<BS, D>>
+  const void* kernel = nullptr;  // prefix_decode_kernel<PrefixCfg<BS, D>> (or a prefill kernel)
   int threads = 0;
   int smem = 0;
+  int rows = 64;                 // query rows (tokens x group heads) per CTA
 };
 
 // Shared-prefix pass kernels (bf16); false when (head_dim, block_size) has none.
 bool find_prefix_bf16(int head_dim, int block_size, PrefixInstance* out);
-// Paged prefill kernels (bf16); same shapes, same instance record.
-bool find_prefill_bf16(int head_dim, int block_size, PrefixInstance* out);
+// Paged prefill kernels (bf16); same shapes, same instance record. tcgen05:
+// the 128-row tensor-memory kernel; otherwise the 64-row mma.sync kernel.
+bool find_prefill_bf16(int head_dim, int block_size, bool tcgen05, PrefixInstance* out);
 
 }  // namespace pagedkv

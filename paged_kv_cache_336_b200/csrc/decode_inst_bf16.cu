@@ -12,6 +12,7 @@
 #include "decode_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefix_kernel.cuh"
+#include "tc_prefill_kernel.cuh"
 
 namespace pagedkv {
 
@@ -77,11 +78,27 @@ static PrefixInstance make_prefill() {
   return r;
 }
 
-bool find_prefill_bf16(int head_dim, int block_size, PrefixInstance* out) {
-  if (block_size == 16 && head_dim == 64) { *out = make_prefill<16, 64>(); return true; }
-  if (block_size == 16 && head_dim == 128) { *out = make_prefill<16, 128>(); return true; }
-  if (block_size == 32 && head_dim == 64) { *out = make_prefill<32, 64>(); return true; }
-  if (block_size == 32 && head_dim == 128) { *out = make_prefill<32, 128>(); return true; }
+template <int BS, int D>
+static PrefixInstance make_tc_prefill() {
+  using Cfg = TcCfg<BS, D>;
+  PrefixInstance r;
+  r.kernel = reinterpret_cast<const void*>(&tc_prefill_kernel<Cfg>);
+  r.threads = Cfg::kThreads;
+  r.smem = Cfg::kSmem;
+  r.rows = Cfg::ROWS;
+  return r;
+}
+
+template <int BS, int D>
+static PrefixInstance pick_prefill(bool tcgen05) {
+  return tcgen05 ? make_tc_prefill<BS, D>() : make_prefill<BS, D>();
+}
+
+bool find_prefill_bf16(int head_dim, int block_size, bool tcgen05, PrefixInstance* out) {
+  if (block_size == 16 && head_dim == 64) { *out = pick_prefill<16, 64>(tcgen05); return true; }
+  if (block_size == 16 && head_dim == 128) { *out = pick_prefill<16, 128>(tcgen05); return true; }
+  if (block_size == 32 && head_dim == 64) { *out = pick_prefill<32, 64>(tcgen05); return true; }
+  if (block_size == 32 && head_dim == 128) { *out = pick_prefill<32, 128>(tcgen05); return true; }
   return false;
 }
 

@@ -2,7 +2,9 @@
 oracle: batches mixing new-prompt prefill (no prior context), chunked
 prefill on top of earlier context, single new tokens; query tiles that span
 several KV partitions (partials + merge) and ones that fit one; GQA groups
-1, 4 and 8; block sizes 16 and 32."""
+1, 4, 8 and 16; head_dim 64 and 128; block sizes 16 and 32. Both prefill
+kernels are covered: the tcgen05 one (default) and the mma.sync one
+(PAGEDKV_PREFILL_KERNEL=mma_sync)."""
 
 import numpy as np
 import pytest
@@ -16,20 +18,33 @@ from gpu_util import check_close, device_tables, setup, to_f64
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("G,bs,partition", [(1, 16, 64), (4, 16, 32), (8, 32, 64), (4, 32, 4096)])
-def test_prefill_matches_oracle(G, bs, partition):
-    rng = np.random.default_rng(70 + G + bs)
+KERNELS = ["tcgen05", "mma_sync"]
+
+
+@pytest.fixture(params=KERNELS)
+def kernel(request, monkeypatch):
+    if request.param == "mma_sync":
+        monkeypatch.setenv("PAGEDKV_PREFILL_KERNEL", "mma_sync")
+    else:
+        monkeypatch.delenv("PAGEDKV_PREFILL_KERNEL", raising=False)
+    return request.param
+
+
+@pytest.mark.parametrize("G,bs,partition,D", [(1, 16, 64, 128), (4, 16, 32, 128), (8, 32, 64, 128),
+                                              (4, 32, 4096, 128), (16, 16, 128, 128),
+                                              (2, 16, 64, 64), (8, 32, 4096, 64)])
+def test_prefill_matches_oracle(kernel, G, bs, partition, D):
     # (context length, new tokens): prompt, chunk on prior context, single token, odd sizes
     plan = [(75, 75), (300, 37), (129, 1), (64, 64), (500, 130), (17, 9)]
     ctx = np.array([c for c, _ in plan], dtype=np.int64)
     qlen = np.array([n for _, n in plan], dtype=np.int32)
     w = workloads.random_small(71 + G, num_seqs=len(plan), num_q_heads=2 * G, num_kv_heads=2,
-                               head_dim=128, block_size=bs, dtype=workloads.BF16,
+                               head_dim=D, block_size=bs, dtype=workloads.BF16,
                                max_ctx=int(ctx.max()), fixed_lens=ctx.tolist())
     bm, k_pool, v_pool = setup(w)
     bt, ctx_d, tables, ctx_np = device_tables(bm, list(range(len(plan))))
     total = int(qlen.sum())
-    q = workloads.draw_normal((total, 2 * G, 128), workloads.BF16, 77, "cuda")
+    q = workloads.draw_normal((total, 2 * G, D), workloads.BF16, 77, "cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = binding.prefill(q, k_pool, v_pool, bt, ctx_np, qlen, w.scale, partition_tokens=partition,
                           dev_err=err)
@@ -37,7 +52,93 @@ def test_prefill_matches_oracle(G, bs, partition):
     assert int(err.item()) == 0
     want = oracle.paged_prefill(to_f64(q), to_f64(k_pool), to_f64(v_pool), tables, ctx_np, qlen,
                                 w.scale)
-    check_close(to_f64(out), want, workloads.BF16, f"prefill G={G} bs={bs} part={partition}")
+    check_close(to_f64(out), want, workloads.BF16,
+                f"prefill[{kernel}] G={G} bs={bs} part={partition} D={D}")
+
+
+def _ramp_keys(k_pool, tables, ctx_np, amplitude):
+    """Overwrite every key of every sequence with amplitude * t / ctx in all
+    dimensions (t = the token's position): with all-ones queries each logit
+    grows with t, so the running max rises at every KV chunk."""
+    bs = k_pool.shape[2]
+    for s, c in enumerate(ctx_np):
+        c = int(c)
+        for t in range(c):
+            k_pool[int(tables[s, t // bs]), :, t % bs, :] = amplitude * t / c
+
+
+def test_prefill_rising_logits(kernel):
+    """Logits that grow along the context (the max moves in every chunk) and
+    span many powers of two: exercises the rescaling of the accumulator."""
+    G, bs, D = 4, 16, 128
+    plan = [(700, 700), (450, 200), (64, 64)]
+    ctx = np.array([c for c, _ in plan], dtype=np.int64)
+    qlen = np.array([n for _, n in plan], dtype=np.int32)
+    w = workloads.random_small(90, num_seqs=len(plan), num_q_heads=2 * G, num_kv_heads=2,
+                               head_dim=D, block_size=bs, dtype=workloads.BF16,
+                               max_ctx=int(ctx.max()), fixed_lens=ctx.tolist())
+    bm, k_pool, v_pool = setup(w)
+    bt, _, tables, ctx_np = device_tables(bm, list(range(len(plan))))
+    _ramp_keys(k_pool, tables, ctx_np, 3.0)  # logits from 0 to ~34 (~49 powers of two)
+    total = int(qlen.sum())
+    q = torch.ones((total, 2 * G, D), dtype=torch.bfloat16, device="cuda")
+    want = oracle.paged_prefill(to_f64(q), to_f64(k_pool), to_f64(v_pool), tables, ctx_np, qlen,
+                                w.scale)
+    for partition in (64, 4096):
+        out = binding.prefill(q, k_pool, v_pool, bt, ctx_np, qlen, w.scale,
+                              partition_tokens=partition)
+        check_close(to_f64(out), want, workloads.BF16, f"rising[{kernel}] part={partition}")
+
+
+def test_prefill_long_prompt(kernel):
+    """One long prompt (many KV chunks per tile: the stage ring wraps many
+    times) next to short ones, whole-context partitions."""
+    G, bs, D = 2, 32, 128
+    plan = [(1500, 1500), (40, 40), (1000, 3)]
+    ctx = np.array([c for c, _ in plan], dtype=np.int64)
+    qlen = np.array([n for _, n in plan], dtype=np.int32)
+    w = workloads.random_small(91, num_seqs=len(plan), num_q_heads=G, num_kv_heads=1,
+                               head_dim=D, block_size=bs, dtype=workloads.BF16,
+                               max_ctx=int(ctx.max()), fixed_lens=ctx.tolist())
+    bm, k_pool, v_pool = setup(w)
+    bt, _, tables, ctx_np = device_tables(bm, list(range(len(plan))))
+    total = int(qlen.sum())
+    q = workloads.draw_normal((total, G, D), workloads.BF16, 92, "cuda")
+    out = binding.prefill(q, k_pool, v_pool, bt, ctx_np, qlen, w.scale, partition_tokens=8192)
+    want = oracle.paged_prefill(to_f64(q), to_f64(k_pool), to_f64(v_pool), tables, ctx_np, qlen,
+                                w.scale)
+    check_close(to_f64(out), want, workloads.BF16, f"long prompt[{kernel}]")
+
+
+def test_prefill_full_size_sampled(kernel):
+    """The measured prefill configuration (16 sequences x (1024 prior + 1024
+    new tokens), 32 query / 8 KV heads, head_dim 128, block 16, 512-token
+    partitions): sampled (token, head) outputs against the oracle. The
+    output of new token i at position p is decode attention over the
+    sequence's first p + 1 tokens."""
+    from gpu_util import oracle_one
+    B, prior, chunk, Hq, Hkv, D, bs = 16, 1024, 1024, 32, 8, 128, 16
+    ctx = np.full(B, prior + chunk, dtype=np.int64)
+    w = workloads.random_small(500, num_seqs=B, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                               block_size=bs, dtype=workloads.BF16, max_ctx=prior + chunk,
+                               fixed_lens=ctx.tolist())
+    bm, k_pool, v_pool = setup(w)
+    bt, _, tables, ctx_np = device_tables(bm, list(range(B)))
+    qlen = np.full(B, chunk, dtype=np.int32)
+    q = workloads.draw_normal((B * chunk, Hq, D), workloads.BF16, 501, "cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = binding.prefill(q, k_pool, v_pool, bt, ctx_np, qlen, w.scale, partition_tokens=512,
+                          dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rng = np.random.default_rng(502)
+    picks = [(0, 0, 0), (B - 1, chunk - 1, Hq - 1), (3, 127, 5), (7, 128, 8)]
+    picks += [(int(rng.integers(B)), int(rng.integers(chunk)), int(rng.integers(Hq)))
+              for _ in range(28)]
+    got = np.stack([to_f64(out[s * chunk + i, h]) for s, i, h in picks])
+    want = np.stack([oracle_one(q[s * chunk + i:s * chunk + i + 1], k_pool, v_pool, tables[s],
+                                prior + i + 1, w.scale, 0, h) for s, i, h in picks])
+    check_close(got, want, workloads.BF16, f"full-size prefill[{kernel}]")
 
 
 def test_prefill_of_one_token_equals_decode():
