@@ -650,7 +650,7 @@ pa_status_t run_prefill(const DecodeReq& r, const int32_t* ctx_host, const int32
   if (total_q == 0) return ok();
 
   const int G = r.num_q_heads / r.num_kv_heads;
-  const int tq = std::max(1, pinst.rows / G);  // query tokens per tile
+  const int tq = pinst.tiles * std::max(1, pinst.rows / G);  // query tokens per CTA
   const int pb = partition_tokens / r.block_size;
   thread_local std::vector<int32_t> lens;
   thread_local std::vector<PrefillItem> items;

@@ -25,7 +25,8 @@ struct PrefixInstance {
   const void* kernel = nullptr;  // prefix_decode_kernel<PrefixCfg<BS, D>> (or a prefill kernel)
   int threads = 0;
   int smem = 0;
-  int rows = 64;                 // query rows (tokens x group heads) per CTA
+  int rows = 64;                 // query rows (tokens x group heads) per tile
+  int tiles = 1;                 // tiles per CTA
 };
 
 // Shared-prefix pass kernels (bf16); false when (head_dim, block_size) has none.

@@ -86,6 +86,7 @@ static PrefixInstance make_tc_prefill() {
   r.threads = Cfg::kThreads;
   r.smem = Cfg::kSmem;
   r.rows = Cfg::ROWS;
+  r.tiles = Cfg::TILES;
   return r;
 }
 

@@ -3,86 +3,121 @@
 // What is computed is the causal prefill of prefill_kernel.cuh: new token i
 // of a sequence at position p attends to tokens 0..p, read through the block
 // table ("What is PagedAttention?", How It Works). Many queries share every
-// KV tile, so the products are a dense contraction and this kernel runs them
-// as 128-row tcgen05 MMAs with fp32 accumulators in tensor memory:
+// KV tile, so the products are a dense contraction; here they run as
+// 128-row tcgen05 MMAs with fp32 accumulators in tensor memory.
 //
-//   CTA = 128 query rows (query tokens x the KV head's group heads) of one
-//   sequence, one KV head, one KV partition; Q stays in shared memory.
-//   warp 4 (producer): streams 64-token K/V chunks (four 16-token TMA units,
-//     128-byte swizzle, laid out so a chunk is one K-major / MN-major UMMA
-//     operand) into an NS-stage ring.
-//   warp 5 (MMA issuer, one thread): S_j = Q K_j^T (M=128, N=64, K=head_dim)
-//     into one of two TMEM buffers, issued one chunk ahead so the tensor core
-//     works while the softmax runs; O += P_j V_j (M=128, N=head_dim, K=64)
-//     into the TMEM accumulator once P_j is in shared memory.
-//   warps 0-3 (softmax): thread r owns row r (TMEM lane r). It reads its 64
-//     logits, applies the causal mask, and keeps a running max m used for
-//     both P and O; O is rescaled in TMEM only when the max grows by more
-//     than 2^8 (so P <= 256 and O never overflows), and P is written as bf16
-//     rows of the next MMA's A operand.
-// Each stage of the pipeline is handed over through mbarriers (TMA byte
-// counts, tcgen05.commit, warp arrivals); every wait is bounded.
+// One CTA = two tiles of 128 query rows (query tokens x the KV head's group
+// heads) of one sequence, one KV head, one KV partition. Both tiles share
+// every K/V chunk, so the tensor core has one tile's work while the other
+// tile's softmax runs:
+//   warp 8 (producer): streams K_j then V_j of each 64-token chunk (four
+//     16-token TMA units, 128-byte swizzle: a chunk is one K-major operand
+//     for S and one MN-major operand for P V) into a ring of slots, and
+//     clears the V rows past the span in the last chunk.
+//   warps 9 / 10 (MMA issuers of tile 0 / 1, one thread each), per chunk j:
+//       S_t(j+1) = Q_t K_{j+1}^T     (M=128, N=64, K=head_dim)
+//       O_t += P_t(j) V_j            (M=128, N=head_dim, K=64)
+//     They wait only for data (TMA bytes, the softmax's arrivals), never for
+//     an MMA to finish. One issuer per tile halves the serial chain of
+//     barrier waits, commits and MMA issues that one thread would run.
+//   warps 0-3 / 4-7 (softmax of tile 0 / 1): thread r owns row r (TMEM lane
+//     r). It reads its 64 logits (releasing the S buffer at once), masks
+//     causally where the chunk reaches past the row's position, and keeps a
+//     reference max m: P = 2^(x - m) goes to shared memory as bf16 rows of
+//     the A operand of P V; m moves only when the chunk's max exceeds it by
+//     more than 2^8, and then O (in TMEM) and l are scaled by 2^(m_old - m_new).
+//     A quarter of the exponentials run as a polynomial on the FMA pipe, so
+//     the MUFU unit (16 results per clock per SM) does not set the pace.
+// TMEM per tile: two 64-column S buffers (chunk parity) and head_dim O
+// columns; 512 columns for the CTA. P is double-buffered in shared memory.
+// Every hand-over is an mbarrier (TMA byte counts, tcgen05.commit, warp
+// arrivals) with one barrier per buffer, so no waiter can be lapped by two
+// phases; every wait is bounded.
 #pragma once
 
 #include "prefill_kernel.cuh"
 
 namespace pagedkv {
 
+// 2^x for x <= 8 on the FMA pipe (no MUFU): x = n + f with n = round(x)
+// and f in [-1/2, 1/2]; 2^f by a cubic (least-squares fit at Chebyshev
+// nodes with p(0) = 1: relative error below 1.5e-4, far under bf16's
+// 2^-9 rounding of P); 2^n added into the exponent bits. x is clamped at
+// -125 so the result stays a normal float (2^-125 is 0 next to the
+// chunk's largest P >= 1).
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;          // 1.5 * 2^23: rounds x to an integer in t's low bits
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(0.05592203f, f, 0.24223731f);
+  p = fmaf(p, f, 0.69312102f);
+  p = fmaf(p, f, 1.f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  return __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<uint32_t>(n) << 23));
+}
+
 template <int BS_, int D_>
 struct TcCfg {
   static constexpr int BS = BS_;
   static constexpr int D = D_;
-  static constexpr int ROWS = 128;                      // MMA M: query rows per CTA
-  static constexpr int CHUNK = 64;                      // MMA N of S: KV tokens per step
+  static constexpr int ROWS = 128;                      // MMA M: query rows per tile
+  static constexpr int TILES = 2;                       // tiles per CTA
+  static constexpr int CHUNK = 64;                      // KV tokens per step (N of S, K of P V)
   static constexpr int UR = 16;                         // TMA unit rows
   static constexpr int UPC = CHUNK / UR;                // units per chunk
   static constexpr int KCH = D * 2 / 128;               // 128-byte column chunks of a row
-  static constexpr int kQBytes = ROWS * D * 2;
-  static constexpr int kKVBytes = CHUNK * D * 2;        // K (or V) of one chunk
-  static constexpr int kStageBytes = 2 * kKVBytes;
-  static constexpr int NS = 3;
-  static constexpr int kPBytes = ROWS * CHUNK * 2;      // one P buffer
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmem = 1024 + kQBytes + NS * kStageBytes + 2 * kPBytes + kBarBytes;
-  static constexpr int kThreads = 6 * 32;
-  static constexpr uint32_t kTmemCols = 256;            // S0 [0,64) S1 [64,128) O [128,128+D)
+  static constexpr int kQBytes = ROWS * D * 2;          // one tile's Q
+  static constexpr int kSlotBytes = CHUNK * D * 2;      // K or V of one chunk
+  static constexpr int NSLOT = 6;                       // ring: K_0 V_0 K_1 V_1 ...
+  static constexpr int kPBytes = ROWS * CHUNK * 2;      // one P buffer: [ROWS][128 B]
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmem =
+      1024 + TILES * kQBytes + NSLOT * kSlotBytes + TILES * 2 * kPBytes + kBarBytes;
+  static constexpr int kSoftmaxWarps = 4 * TILES;
+  static constexpr int kThreads = (kSoftmaxWarps + 1 + TILES) * 32;
+  static constexpr uint32_t kTileCols = 256;            // S buffers [0,128), O [128, 128 + D)
+  static constexpr uint32_t kTmemCols = TILES * kTileCols;
   static constexpr uint32_t kOCol = 128;
   static constexpr float kRescaleThreshold = 8.f;       // log2 units
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(BS % UR == 0, "block size");
+  static_assert(CHUNK * 2 == 128, "a P row is one 128-byte swizzle row");
+  static_assert(32 % UPC == 0, "a chunk's units lie in one 32-unit id batch");
   static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kTmemCols <= 512, "tensor memory");
 };
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads, 1)
     tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const PrefillArgs pf) {
-  constexpr int NS = Cfg::NS;
+  constexpr int NSLOT = Cfg::NSLOT;
   constexpr int BS = Cfg::BS;
   constexpr int D = Cfg::D;
   constexpr int UR = Cfg::UR;
   constexpr int CHUNK = Cfg::CHUNK;
   constexpr int KCH = Cfg::KCH;
   constexpr int ROWS = Cfg::ROWS;
+  constexpr int SMW = Cfg::kSoftmaxWarps;
   const DecodeArgs& a = pf.d;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* qs = smem;                                    // [KCH][ROWS][128 B]
-  uint8_t* stages = qs + Cfg::kQBytes;                   // NS x {K [KCH][CHUNK][128 B], V same}
-  uint8_t* pbuf = stages + NS * Cfg::kStageBytes;        // 2 x [ROWS][128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(pbuf + 2 * Cfg::kPBytes);
-  uint64_t* full = bars;            // [NS]  TMA bytes landed
-  uint64_t* empty = bars + NS;      // [NS]  PV MMA of the stage done (commit)
-  uint64_t* s_full = bars + 2 * NS; // [2]   S MMA done (commit)
-  uint64_t* s_free = s_full + 2;    // [2]   S read by the 4 softmax warps
-  uint64_t* p_full = s_free + 2;    // [2]   P written by the 4 softmax warps
-  uint64_t* p_free = p_full + 2;    // [2]   PV MMA done reading P (commit)
-  uint64_t* o_done = p_free + 2;    // [1]   PV MMA done (commit), once per chunk
-  uint64_t* o_last = o_done + 1;    // [1]   every MMA of the CTA done (commit), once
-  uint64_t* q_full = o_last + 1;    // [1]   Q in shared memory (4 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
+  uint8_t* qs = smem;                                    // [TILES][KCH][ROWS][128 B]
+  uint8_t* slots = qs + Cfg::TILES * Cfg::kQBytes;       // [NSLOT][KCH][CHUNK][128 B]
+  uint8_t* pbuf = slots + NSLOT * Cfg::kSlotBytes;       // [TILES][2][ROWS][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(pbuf + Cfg::TILES * 2 * Cfg::kPBytes);
+  uint64_t* kv_full = bars;               // [NSLOT] TMA bytes landed
+  uint64_t* kv_empty = bars + NSLOT;      // [NSLOT] last MMA reading the slot done (commit)
+  uint64_t* s_full = bars + 2 * NSLOT;    // [tile][buffer] S MMA done (commit)
+  uint64_t* s_free = s_full + 4;          // [tile][buffer] S read (4 warp arrivals)
+  uint64_t* p_full = s_free + 4;          // [tile][buffer] P written (4 warp arrivals)
+  uint64_t* p_free = p_full + 4;          // [tile][buffer] P V MMA done (commit)
+  uint64_t* q_full = p_free + 4;          // [tile] Q in shared memory (4 warp arrivals)
+  uint64_t* o_last = q_full + 2;          // [tile] every MMA of the tile done (commit), once
+  uint64_t* v_tail = o_last + 2;          // last chunk's V tail rows cleared (producer), once
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_tail + 1);
 
   grid_dependents_launch();
   const int tid = threadIdx.x;
@@ -91,24 +126,30 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
   const PrefillItem it = pf.items[blockIdx.x];
   const int G = a.group;
   const int Hkv = a.num_kv_heads;
+  const int TQ = ROWS / G;                                   // query tokens per tile
+  const int ntiles = it.q_count > TQ ? 2 : 1;                // tile 1 idles when empty
   const int span0 = it.block_begin * BS;
   const int span_end = min(it.block_end * BS, it.kv_end);
   const int nchunks = span_end > span0 ? (span_end - span0 + CHUNK - 1) / CHUNK : 0;
+  // V rows of the last chunk past the span (when it is partial) must read as 0.
+  const int vt_last = nchunks > 0 ? span_end - (span0 + (nchunks - 1) * CHUNK) : CHUNK;
 
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], ntiles);  // one commit per tile's issuer
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
       mbar_init(&p_full[i], 4);
       mbar_init(&p_free[i], 1);
     }
-    mbar_init(o_done, 1);
-    mbar_init(o_last, 1);
-    mbar_init(q_full, 4);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 4);
+      mbar_init(&o_last[t], 1);
+    }
+    mbar_init(v_tail, 1);
     fence_barrier_init();
     tma_prefetch_descriptor(&tm_k);
     tma_prefetch_descriptor(&tm_v);
@@ -119,243 +160,307 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
   tmem_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
-    // ---- producer: K/V chunks ------------------------------------------------------
+  if (warp == SMW) {
+    // ---- producer: K_0, V_0, K_1, V_1, ... into the slot ring -----------------------
     const uint64_t policy = l2_policy(2);  // every query tile of a sequence re-reads its blocks
     const int32_t* bt = a.block_tables + static_cast<int64_t>(it.seq) * a.max_blocks_per_seq;
+    // Block ids of the span's 16-token units, 32 units per batch held one per
+    // lane, the next batch loaded a batch ahead (a chunk's units never
+    // straddle two batches).
+    const int nunits = (span_end - span0 + UR - 1) / UR;
+    auto unit_ids = [&](int batch) -> int {
+      const int u = batch * 32 + lane;
+      return u < nunits ? bt[(span0 + u * UR) / BS] : -1;
+    };
+    int ids = unit_ids(0);
+    int ids_next = unit_ids(1);
+    int batch = 0;
     int issued = 0;
-    for (int j = 0; j < nchunks; ++j) {
-      const int st = j % NS;
+    for (int i = 0; i < 2 * nchunks; ++i) {
+      const int j = i >> 1;
+      const int slot = i % NSLOT;
+      const int use = i / NSLOT;
       bool ok = true;
-      if (j >= NS) ok = mbar_wait_bounded(&empty[st], ((j / NS) - 1) & 1, a.dev_err);
+      if (use > 0) ok = mbar_wait_bounded(&kv_empty[slot], (use - 1) & 1, a.dev_err);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int c0 = span0 + j * CHUNK;
       const int nu = min(Cfg::UPC, (span_end - c0 + UR - 1) / UR);  // units holding used tokens
-      const int phys_l = (lane < nu) ? bt[(c0 + lane * UR) / BS] : -1;
+      const int u0 = j * Cfg::UPC;
+      if ((u0 >> 5) != batch) {
+        batch = u0 >> 5;
+        ids = ids_next;
+        ids_next = unit_ids(batch + 1);
+      }
       int phys_u[Cfg::UPC];
 #pragma unroll
-      for (int u = 0; u < Cfg::UPC; ++u) phys_u[u] = __shfl_sync(0xffffffffu, phys_l, u);
+      for (int u = 0; u < Cfg::UPC; ++u) phys_u[u] = __shfl_sync(0xffffffffu, ids, (u0 + u) & 31);
       if (lane == 0) {
-        uint8_t* kst = stages + st * Cfg::kStageBytes;
-        uint8_t* vst = kst + Cfg::kKVBytes;
+        const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
+        uint8_t* dst = slots + slot * Cfg::kSlotBytes;
         uint32_t bytes = 0;
 #pragma unroll
         for (int u = 0; u < Cfg::UPC; ++u)
-          if (u < nu && phys_u[u] >= 0 && phys_u[u] < a.num_blocks) bytes += 2 * KCH * UR * 128;
-        mbar_arrive_expect_tx(&full[st], bytes);
+          if (u < nu && phys_u[u] >= 0 && phys_u[u] < a.num_blocks) bytes += KCH * UR * 128;
+        mbar_arrive_expect_tx(&kv_full[slot], bytes);
 #pragma unroll
         for (int u = 0; u < Cfg::UPC; ++u) {
           if (u >= nu) continue;
           const int ph = phys_u[u];
           if (ph < 0 || ph >= a.num_blocks) {
-            report(a.dev_err, PA_DEVERR_BLOCK_ID);  // the unit keeps stale rows; the call fails
+            if (i & 1) report(a.dev_err, PA_DEVERR_BLOCK_ID);  // the unit keeps stale rows
             continue;
           }
           const int32_t y = (ph * Hkv + it.kvh) * BS + ((c0 + u * UR) % BS);
 #pragma unroll
-          for (int c = 0; c < KCH; ++c) {
-            tma_load_2d(kst + c * (CHUNK * 128) + u * (UR * 128), &tm_k, &full[st], c * 64, y, policy);
-            tma_load_2d(vst + c * (CHUNK * 128) + u * (UR * 128), &tm_v, &full[st], c * 64, y, policy);
-          }
+          for (int c = 0; c < KCH; ++c)
+            tma_load_2d(dst + c * (CHUNK * 128) + u * (UR * 128), map, &kv_full[slot], c * 64, y, policy);
         }
       }
-      issued = j + 1;
+      issued = i + 1;
+    }
+    // Clear V rows [vt_last, CHUNK) of the last chunk once its copy landed
+    // (stale or unloaded rows; 0 * NaN is NaN), then release its P V.
+    if (issued == 2 * nchunks && vt_last < CHUNK) {
+      const int i = 2 * nchunks - 1;
+      const bool landed =
+          __all_sync(0xffffffffu, mbar_wait_bounded(&kv_full[i % NSLOT], (i / NSLOT) & 1, a.dev_err));
+      if (landed) {
+        uint8_t* vst = slots + (i % NSLOT) * Cfg::kSlotBytes;
+        const int n16 = (CHUNK - vt_last) * KCH * 8;
+        for (int x = lane; x < n16; x += 32) {
+          const int row = vt_last + x / (KCH * 8);
+          const int rem = x % (KCH * 8);
+          *reinterpret_cast<uint4*>(vst + (rem >> 3) * (CHUNK * 128) + row * 128 + ((rem & 7) << 4)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(v_tail);
+      }
     }
     // Every copy issued has landed before the CTA's shared memory is released.
-    for (int j = max(0, issued - NS); j < issued; ++j)
-      mbar_wait_bounded(&full[j % NS], (j / NS) & 1, a.dev_err);
+    for (int i = max(0, issued - NSLOT); i < issued; ++i)
+      mbar_wait_bounded(&kv_full[i % NSLOT], (i / NSLOT) & 1, a.dev_err);
     __syncwarp();
-  } else if (warp == 5) {
-    // ---- MMA issuer ------------------------------------------------------------------
-    if (lane == 0 && nchunks > 0) {
+  } else if (warp > SMW) {
+    // ---- MMA issuer of tile t ----------------------------------------------------------
+    const int t = warp - SMW - 1;
+    if (lane == 0 && t < ntiles && nchunks > 0) {
       constexpr uint32_t kIdS = umma_idesc_bf16(ROWS, CHUNK, 0, 0);
       constexpr uint32_t kIdO = umma_idesc_bf16(ROWS, D, 0, 1);
-      const uint32_t qa = smem_addr(qs);
+      // Descriptors are built once; a start address moves by adding its
+      // offset in 16-byte units (the 14-bit field cannot overflow below 256 KB).
+      const uint64_t q_desc = umma_desc_sw128(smem_addr(qs + t * Cfg::kQBytes), 16, 1024);
+      const uint64_t k_desc = umma_desc_sw128(smem_addr(slots), 16, 1024);
+      const uint64_t v_desc = umma_desc_sw128(smem_addr(slots), CHUNK * 128, 1024);
+      const uint64_t p_desc = umma_desc_sw128(smem_addr(pbuf + 2 * t * Cfg::kPBytes), 16, 1024);
+      const uint32_t s_tmem = tmem + t * Cfg::kTileCols;
+      const uint32_t o_tmem = tmem + t * Cfg::kTileCols + Cfg::kOCol;
+      // S_t(j) = Q_t K_j^T into buffer j & 1, once the softmax has read
+      // S_t(j - 2) from it.
       auto issue_s = [&](int j) -> bool {
-        const int st = j % NS, b = j & 1;
-        if (!mbar_wait_bounded(&full[st], (j / NS) & 1, a.dev_err)) return false;
-        if (j >= 2 && !mbar_wait_bounded(&s_free[b], ((j >> 1) - 1) & 1, a.dev_err)) return false;
+        const int i = 2 * j, slot = i % NSLOT, b = j & 1;
+        if (!mbar_wait_bounded(&kv_full[slot], (i / NSLOT) & 1, a.dev_err)) return false;
+        if (j >= 2 && !mbar_wait_bounded(&s_free[2 * t + b], ((j >> 1) - 1) & 1, a.dev_err))
+          return false;
         tmem_fence_after_sync();
-        const uint32_t ka = smem_addr(stages + st * Cfg::kStageBytes);
+        const uint64_t kd = k_desc + static_cast<uint32_t>((slot * Cfg::kSlotBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = umma_desc_sw128(qa + (kk / 4) * (ROWS * 128) + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd = umma_desc_sw128(ka + (kk / 4) * (CHUNK * 128) + (kk % 4) * 32, 16, 1024);
-          umma_bf16(tmem + b * CHUNK, ad, bd, kIdS, kk > 0);
-        }
-        umma_commit(&s_full[b]);
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(s_tmem + b * CHUNK, q_desc + (((kk / 4) * (ROWS * 128) + (kk % 4) * 32) >> 4),
+                    kd + (((kk / 4) * (CHUNK * 128) + (kk % 4) * 32) >> 4), kIdS, kk > 0);
+        umma_commit(&s_full[2 * t + b]);
+        umma_commit(&kv_empty[slot]);
         return true;
       };
-      bool ok = mbar_wait_bounded(q_full, 0, a.dev_err) && issue_s(0);
+      bool ok = mbar_wait_bounded(&q_full[t], 0, a.dev_err) && issue_s(0);
       for (int j = 0; j < nchunks && ok; ++j) {
-        // S of the next chunk goes to the tensor core before this chunk's P is ready.
+        // The next chunk's S goes to the tensor core before this chunk's P V.
         if (j + 1 < nchunks && !issue_s(j + 1)) break;
-        const int st = j % NS, b = j & 1;
-        if (!mbar_wait_bounded(&p_full[b], (j >> 1) & 1, a.dev_err)) break;
+        const int i = 2 * j + 1, slot = i % NSLOT, b = j & 1;
+        ok = mbar_wait_bounded(&kv_full[slot], (i / NSLOT) & 1, a.dev_err);
+        if (ok && j == nchunks - 1 && vt_last < CHUNK) ok = mbar_wait_bounded(v_tail, 0, a.dev_err);
+        ok = ok && mbar_wait_bounded(&p_full[2 * t + b], (j >> 1) & 1, a.dev_err);
+        if (!ok) break;
         tmem_fence_after_sync();
-        const uint32_t pa = smem_addr(pbuf + b * Cfg::kPBytes);
-        const uint32_t va = smem_addr(stages + st * Cfg::kStageBytes + Cfg::kKVBytes);
+        const uint64_t vd = v_desc + static_cast<uint32_t>((slot * Cfg::kSlotBytes) >> 4);
+        const uint64_t pd = p_desc + static_cast<uint32_t>((b * Cfg::kPBytes) >> 4);
 #pragma unroll
-        for (int t = 0; t < CHUNK / 16; ++t) {
-          const uint64_t ad = umma_desc_sw128(pa + t * 32, 16, 1024);
-          const uint64_t bd = umma_desc_sw128(va + t * (16 * 128), CHUNK * 128, 1024);
-          umma_bf16(tmem + Cfg::kOCol, ad, bd, kIdO, j > 0 || t > 0);
-        }
-        umma_commit(&empty[st]);
-        umma_commit(&p_free[b]);
-        umma_commit(o_done);
+        for (int k = 0; k < CHUNK / 16; ++k)
+          umma_bf16(o_tmem, pd + ((k * 32) >> 4), vd + ((k * 16 * 128) >> 4), kIdO, j > 0 || k > 0);
+        umma_commit(&p_free[2 * t + b]);
+        umma_commit(&kv_empty[slot]);
       }
       // o_last completes once every MMA issued above has; TMEM is freed after it.
-      umma_commit(o_last);
-      mbar_wait_bounded(o_last, 0, a.dev_err);
+      umma_commit(&o_last[t]);
+      mbar_wait_bounded(&o_last[t], 0, a.dev_err);
     }
     __syncwarp();
   } else {
-    // ---- softmax warps: thread r owns query row r (TMEM lane r) -----------------------------
-    const int r = tid;
-    const int jq = r / G;
-    const bool valid = jq < it.q_count;
-    const int lim = valid ? it.p0 + jq : -1;  // last token this row attends to
-    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+    // ---- softmax warps: tile t = warp / 4, thread r owns row r (TMEM lane r) --------
+    const int t = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const int jq = t * TQ + r / G;                       // query token within the item
+    const bool valid = (r / G) < TQ && jq < it.q_count;
+    const int lim = valid ? it.p0 + jq : -1;             // last token this row attends to
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + t * Cfg::kTileCols;
+    const bool active = t < ntiles;
     {
-      const int64_t t = it.q_begin + (valid ? jq : 0);
+      const int64_t tok = it.q_begin + (valid ? jq : 0);
       const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
       const uint4* src = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const __nv_bfloat16*>(a.q) + (t * a.num_q_heads + h) * D);
+          reinterpret_cast<const __nv_bfloat16*>(a.q) + (tok * a.num_q_heads + h) * D);
+      uint8_t* qt = qs + t * Cfg::kQBytes;
+      if (active) {
 #pragma unroll
-      for (int c = 0; c < D * 2 / 16; ++c) {
-        const uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-        const int cc = c >> 3, w = c & 7;
-        *reinterpret_cast<uint4*>(qs + cc * (ROWS * 128) + r * 128 + ((w ^ (r & 7)) << 4)) = v;
+        for (int c = 0; c < D * 2 / 16; ++c) {
+          const uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+          const int cc = c >> 3, w = c & 7;
+          *reinterpret_cast<uint4*>(qt + cc * (ROWS * 128) + r * 128 + ((w ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(q_full);
+      if (active && lane == 0) mbar_arrive(&q_full[t]);
     }
+    const float sl2 = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;  // warp-uniform
-    for (int j = 0; j < nchunks; ++j) {
-      const int st = j % NS, b = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[b], (j >> 1) & 1, a.dev_err));
+    for (int j = 0; j < nchunks && active; ++j) {
+      const int b = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[2 * t + b], (j >> 1) & 1, a.dev_err));
       if (!ok) break;
       tmem_fence_after_sync();
       float sv[CHUNK];
-      {
-        float t32[32];
-        tmem_ld32(tmem + lane_base + b * CHUNK, t32);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[i] = t32[i];
-        tmem_ld32(tmem + lane_base + b * CHUNK + 32, t32);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[32 + i] = t32[i];
-      }
+      tmem_ld64(trow + b * CHUNK, sv);
       tmem_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
+      if (lane == 0) mbar_arrive(&s_free[2 * t + b]);
       const int c0 = span0 + j * CHUNK;
-      float mx = -INFINITY;
+      // Scaled logits: x = s * scale * log2(e). Only chunks that reach past
+      // the row's position or the span's end need the mask.
+      const bool whole = c0 + CHUNK <= span_end && c0 + CHUNK - 1 <= lim && sl2 > 0.f;
+      float mx;
+      if (whole) {
+        float m8[8];
 #pragma unroll
-      for (int i = 0; i < CHUNK; ++i) {
-        const int tok = c0 + i;
-        const bool in = tok < span_end && tok <= lim;  // causal: up to the row's own position
-        sv[i] = in ? sv[i] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sv[i]);
+        for (int i = 0; i < 8; ++i) m8[i] = sv[i];
+#pragma unroll
+        for (int i = 8; i < CHUNK; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i]);
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+      } else {
+        mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < CHUNK; ++i) {
+          const int tk = c0 + i;
+          const bool in = tk < span_end && tk <= lim;
+          sv[i] = in ? sv[i] * sl2 : -INFINITY;
+          mx = fmaxf(mx, sv[i]);
+        }
       }
-      // The reference max moves only when the chunk's max exceeds it by more
-      // than the threshold; O and l are then scaled by 2^(old - new).
       const bool raise = mx > m_used + Cfg::kRescaleThreshold;
       const bool rescale_o = raise && m_used != -INFINITY;
       if (__any_sync(0xffffffffu, rescale_o)) {
         // O must hold every earlier P V product before it is scaled.
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (j - 1) & 1, a.dev_err));
+        const int pb = 2 * t + ((j - 1) & 1);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&p_free[pb], ((j - 1) >> 1) & 1, a.dev_err));
         if (!ok) break;
         tmem_fence_after_sync();
         const float alpha = rescale_o ? fast_exp2(m_used - mx) : 1.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o32[32];
-          tmem_ld32(tmem + lane_base + Cfg::kOCol + c * 32, o32);
+          tmem_ld32(trow + Cfg::kOCol + c * 32, o32);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o32[i] *= alpha;
-          tmem_st32(tmem + lane_base + Cfg::kOCol + c * 32, o32);
+          tmem_st32(trow + Cfg::kOCol + c * 32, o32);
         }
         tmem_fence_before_sync();
         l *= alpha;
       }
       if (raise) m_used = mx;
-      // P = 2^(s - m_used) <= 2^8 as bf16: row r of the A operand of P V.
+      // P = 2^(x - m_used) <= 2^8, as bf16: row r of the A operand of P V
+      // (128-byte swizzled rows). Its buffer last fed P V of chunk j - 2.
       if (j >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&p_free[b], ((j >> 1) - 1) & 1, a.dev_err));
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait_bounded(&p_free[2 * t + b], ((j >> 1) - 1) & 1, a.dev_err));
         if (!ok) break;
       }
-      uint8_t* prow = pbuf + b * Cfg::kPBytes + r * 128;
-      float rs = 0.f;
+      uint32_t pk[CHUNK / 2];
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (whole) {
+        const float nm = -m_used;
 #pragma unroll
-      for (int w8 = 0; w8 < CHUNK / 8; ++w8) {
-        float p[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float x = sv[w8 * 8 + i];
-          p[i] = (x == -INFINITY) ? 0.f : fast_exp2(x - m_used);
-          rs += p[i];
+        for (int i = 0; i < CHUNK; i += 2) {
+          // pairs 3, 7, 11, ... on the FMA pipe, the rest on MUFU
+          const bool poly = (i & 6) == 6;
+          const float x0 = fmaf(sv[i], sl2, nm), x1 = fmaf(sv[i + 1], sl2, nm);
+          const float p0 = poly ? exp2_fma(x0) : fast_exp2(x0);
+          const float p1 = poly ? exp2_fma(x1) : fast_exp2(x1);
+          s4[(i >> 1) & 3] += p0 + p1;
+          pk[i >> 1] = pack_bf16x2(p0, p1);
         }
-        const uint4 pk = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
-                                    pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
-        *reinterpret_cast<uint4*>(prow + ((w8 ^ (r & 7)) << 4)) = pk;
+      } else {
+        const float mu = (m_used == -INFINITY) ? 0.f : m_used;  // a row with nothing yet: all p = 0
+#pragma unroll
+        for (int i = 0; i < CHUNK; i += 2) {
+          const float p0 = fast_exp2(sv[i] - mu);
+          const float p1 = fast_exp2(sv[i + 1] - mu);
+          s4[(i >> 1) & 3] += p0 + p1;
+          pk[i >> 1] = pack_bf16x2(p0, p1);
+        }
       }
-      l += rs;
-      // Rows of V past the span hold stale or unloaded data (0 * NaN is NaN): clear them.
-      const int vt = span_end - c0;
-      if (vt < CHUNK) {
-        uint8_t* vst = stages + st * Cfg::kStageBytes + Cfg::kKVBytes;
-        const int n16 = (CHUNK - vt) * KCH * 8;
-        for (int x = r; x < n16; x += ROWS) {
-          const int row = vt + x / (KCH * 8);
-          const int rem = x % (KCH * 8);
-          *reinterpret_cast<uint4*>(vst + (rem >> 3) * (CHUNK * 128) + row * 128 + ((rem & 7) << 4)) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
+      l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      {
+        uint8_t* prow = pbuf + (2 * t + b) * Cfg::kPBytes + r * 128;
+#pragma unroll
+        for (int w8 = 0; w8 < CHUNK / 8; ++w8)
+          *reinterpret_cast<uint4*>(prow + ((w8 ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * w8], pk[4 * w8 + 1], pk[4 * w8 + 2], pk[4 * w8 + 3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[b]);
+      if (lane == 0) mbar_arrive(&p_full[2 * t + b]);
     }
     // ---- epilogue: O from TMEM, normalised (single partition) or as a partial --------------
-    if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_last, 0, a.dev_err));
-    if (ok) {
-      tmem_fence_after_sync();
-      const int64_t t = it.q_begin + (valid ? jq : 0);
-      const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
-      const int64_t row = t * a.num_q_heads + h;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+    if (active) {
+      if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_last[t], 0, a.dev_err));
+      if (ok) {
+        tmem_fence_after_sync();
+        const int64_t tok = it.q_begin + (valid ? jq : 0);
+        const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
+        const int64_t row = tok * a.num_q_heads + h;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float o32[32];
-        if (nchunks > 0) {
-          tmem_ld32(tmem + lane_base + Cfg::kOCol + c * 32, o32);
-        } else {
+        for (int c = 0; c < D / 32; ++c) {
+          float o32[32];
+          if (nchunks > 0) {
+            tmem_ld32(trow + Cfg::kOCol + c * 32, o32);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o32[i] = 0.f;
+            for (int i = 0; i < 32; ++i) o32[i] = 0.f;
+          }
+          if (!valid) continue;
+          if (it.final_out) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * D + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16x2(o32[8 * i] * inv, o32[8 * i + 1] * inv),
+                                  pack_bf16x2(o32[8 * i + 2] * inv, o32[8 * i + 3] * inv),
+                                  pack_bf16x2(o32[8 * i + 4] * inv, o32[8 * i + 5] * inv),
+                                  pack_bf16x2(o32[8 * i + 6] * inv, o32[8 * i + 7] * inv));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(a.part_acc + (row * a.max_partitions + it.part) * D + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(o32[4 * i], o32[4 * i + 1], o32[4 * i + 2], o32[4 * i + 3]);
+          }
         }
-        if (!valid) continue;
-        if (it.final_out) {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * D + c * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pack_bf16x2(o32[8 * i] * inv, o32[8 * i + 1] * inv),
-                                pack_bf16x2(o32[8 * i + 2] * inv, o32[8 * i + 3] * inv),
-                                pack_bf16x2(o32[8 * i + 4] * inv, o32[8 * i + 5] * inv),
-                                pack_bf16x2(o32[8 * i + 6] * inv, o32[8 * i + 7] * inv));
-        } else {
-          float4* dst = reinterpret_cast<float4*>(a.part_acc + (row * a.max_partitions + it.part) * D + c * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(o32[4 * i], o32[4 * i + 1], o32[4 * i + 2], o32[4 * i + 3]);
+        if (valid && !it.final_out) {
+          a.part_m[row * a.max_partitions + it.part] = m_used;
+          a.part_l[row * a.max_partitions + it.part] = l;
         }
-      }
-      if (valid && !it.final_out) {
-        a.part_m[row * a.max_partitions + it.part] = m_used;
-        a.part_l[row * a.max_partitions + it.part] = l;
       }
     }
   }
