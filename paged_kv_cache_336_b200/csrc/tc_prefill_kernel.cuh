@@ -14,25 +14,26 @@
 //     16-token TMA units, 128-byte swizzle: a chunk is one K-major operand
 //     for S and one MN-major operand for P V) into a ring of slots, and
 //     clears the V rows past the span in the last chunk.
-//   warps 9 / 10 (MMA issuers of tile 0 / 1, one thread each), per chunk j:
+//   warps 9 / 10 (MMA issuers of tile 0 / 1), per chunk j:
 //       S_t(j+1) = Q_t K_{j+1}^T     (M=128, N=64, K=head_dim)
-//       O_t += P_t(j) V_j            (M=128, N=head_dim, K=64)
-//     They wait only for data (TMA bytes, the softmax's arrivals), never for
-//     an MMA to finish. One issuer per tile halves the serial chain of
-//     barrier waits, commits and MMA issues that one thread would run.
+//       O_t += P_t(j) V_j            (M=128, N=head_dim, K=64, P read from TMEM)
+//     The only MMA completion an issuer waits for is the P V of two chunks
+//     back, before S overwrites the buffer holding that P.
 //   warps 0-3 / 4-7 (softmax of tile 0 / 1): thread r owns row r (TMEM lane
-//     r). It reads its 64 logits (releasing the S buffer at once), masks
-//     causally where the chunk reaches past the row's position, and keeps a
-//     reference max m: P = 2^(x - m) goes to shared memory as bf16 rows of
-//     the A operand of P V; m moves only when the chunk's max exceeds it by
-//     more than 2^8, and then O (in TMEM) and l are scaled by 2^(m_old - m_new).
+//     r). It reads its 64 logits, masks causally where the chunk reaches
+//     past the row's position, and keeps a reference max m: P = 2^(x - m)
+//     is written back as packed bf16 over the logits it came from (the A
+//     operand of P V); m moves only when the chunk's max exceeds it by more
+//     than 2^8, and then O (in TMEM) and l are scaled by 2^(m_old - m_new).
 //     A quarter of the exponentials run as a polynomial on the FMA pipe, so
 //     the MUFU unit (16 results per clock per SM) does not set the pace.
-// TMEM per tile: two 64-column S buffers (chunk parity) and head_dim O
-// columns; 512 columns for the CTA. P is double-buffered in shared memory.
-// Every hand-over is an mbarrier (TMA byte counts, tcgen05.commit, warp
-// arrivals) with one barrier per buffer, so no waiter can be lapped by two
-// phases; every wait is bounded.
+// TMEM per tile: two 64-column S / P buffers (chunk parity) and head_dim O
+// columns; 512 columns for the CTA. The tensor core reads its shared-memory
+// operands at about 128 bytes per clock per SM, so P stays out of shared
+// memory: per chunk the MMAs read Q and K (S) and V (P V) only. Every
+// hand-over is an mbarrier (TMA byte counts, tcgen05.commit, warp arrivals)
+// with one barrier per buffer, so no waiter can be lapped by two phases;
+// every wait is bounded.
 #pragma once
 
 #include "prefill_kernel.cuh"
@@ -68,11 +69,9 @@ struct TcCfg {
   static constexpr int KCH = D * 2 / 128;               // 128-byte column chunks of a row
   static constexpr int kQBytes = ROWS * D * 2;          // one tile's Q
   static constexpr int kSlotBytes = CHUNK * D * 2;      // K or V of one chunk
-  static constexpr int NSLOT = 6;                       // ring: K_0 V_0 K_1 V_1 ...
-  static constexpr int kPBytes = ROWS * CHUNK * 2;      // one P buffer: [ROWS][128 B]
+  static constexpr int NSLOT = 8;                       // ring: K_0 V_0 K_1 V_1 ...
   static constexpr int kBarBytes = 512;
-  static constexpr int kSmem =
-      1024 + TILES * kQBytes + NSLOT * kSlotBytes + TILES * 2 * kPBytes + kBarBytes;
+  static constexpr int kSmem = 1024 + TILES * kQBytes + NSLOT * kSlotBytes + kBarBytes;
   static constexpr int kSoftmaxWarps = 4 * TILES;
   static constexpr int kThreads = (kSoftmaxWarps + 1 + TILES) * 32;
   static constexpr uint32_t kTileCols = 256;            // S buffers [0,128), O [128, 128 + D)
@@ -81,7 +80,6 @@ struct TcCfg {
   static constexpr float kRescaleThreshold = 8.f;       // log2 units
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(BS % UR == 0, "block size");
-  static_assert(CHUNK * 2 == 128, "a P row is one 128-byte swizzle row");
   static_assert(32 % UPC == 0, "a chunk's units lie in one 32-unit id batch");
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kTmemCols <= 512, "tensor memory");
@@ -106,13 +104,11 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* qs = smem;                                    // [TILES][KCH][ROWS][128 B]
   uint8_t* slots = qs + Cfg::TILES * Cfg::kQBytes;       // [NSLOT][KCH][CHUNK][128 B]
-  uint8_t* pbuf = slots + NSLOT * Cfg::kSlotBytes;       // [TILES][2][ROWS][128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(pbuf + Cfg::TILES * 2 * Cfg::kPBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(slots + NSLOT * Cfg::kSlotBytes);
   uint64_t* kv_full = bars;               // [NSLOT] TMA bytes landed
   uint64_t* kv_empty = bars + NSLOT;      // [NSLOT] last MMA reading the slot done (commit)
   uint64_t* s_full = bars + 2 * NSLOT;    // [tile][buffer] S MMA done (commit)
-  uint64_t* s_free = s_full + 4;          // [tile][buffer] S read (4 warp arrivals)
-  uint64_t* p_full = s_free + 4;          // [tile][buffer] P written (4 warp arrivals)
+  uint64_t* p_full = s_full + 4;          // [tile][buffer] P written (4 warp arrivals)
   uint64_t* p_free = p_full + 4;          // [tile][buffer] P V MMA done (commit)
   uint64_t* q_full = p_free + 4;          // [tile] Q in shared memory (4 warp arrivals)
   uint64_t* o_last = q_full + 2;          // [tile] every MMA of the tile done (commit), once
@@ -141,7 +137,6 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
       mbar_init(&p_full[i], 4);
       mbar_init(&p_free[i], 1);
     }
@@ -194,7 +189,9 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       int phys_u[Cfg::UPC];
 #pragma unroll
       for (int u = 0; u < Cfg::UPC; ++u) phys_u[u] = __shfl_sync(0xffffffffu, ids, (u0 + u) & 31);
-      if (lane == 0) {
+      // Every value above is warp-uniform; one elected lane of the converged
+      // warp issues the copies.
+      if (elect_one()) {
         const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
         uint8_t* dst = slots + slot * Cfg::kSlotBytes;
         uint32_t bytes = 0;
@@ -216,6 +213,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
             tma_load_2d(dst + c * (CHUNK * 128) + u * (UR * 128), map, &kv_full[slot], c * 64, y, policy);
         }
       }
+      __syncwarp();
       issued = i + 1;
     }
     // Clear V rows [vt_last, CHUNK) of the last chunk once its copy landed
@@ -243,9 +241,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       mbar_wait_bounded(&kv_full[i % NSLOT], (i / NSLOT) & 1, a.dev_err);
     __syncwarp();
   } else if (warp > SMW) {
-    // ---- MMA issuer of tile t ----------------------------------------------------------
+    // ---- MMA issuer of tile t: the whole warp runs the loop (waits are warp-wide,
+    // values warp-uniform); one elected lane issues each group of MMAs and commits.
     const int t = warp - SMW - 1;
-    if (lane == 0 && t < ntiles && nchunks > 0) {
+    if (t < ntiles && nchunks > 0) {
       constexpr uint32_t kIdS = umma_idesc_bf16(ROWS, CHUNK, 0, 0);
       constexpr uint32_t kIdO = umma_idesc_bf16(ROWS, D, 0, 1);
       // Descriptors are built once; a start address moves by adding its
@@ -253,49 +252,58 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       const uint64_t q_desc = umma_desc_sw128(smem_addr(qs + t * Cfg::kQBytes), 16, 1024);
       const uint64_t k_desc = umma_desc_sw128(smem_addr(slots), 16, 1024);
       const uint64_t v_desc = umma_desc_sw128(smem_addr(slots), CHUNK * 128, 1024);
-      const uint64_t p_desc = umma_desc_sw128(smem_addr(pbuf + 2 * t * Cfg::kPBytes), 16, 1024);
       const uint32_t s_tmem = tmem + t * Cfg::kTileCols;
       const uint32_t o_tmem = tmem + t * Cfg::kTileCols + Cfg::kOCol;
-      // S_t(j) = Q_t K_j^T into buffer j & 1, once the softmax has read
-      // S_t(j - 2) from it.
+      auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, a.dev_err));
+      };
+      // S_t(j) = Q_t K_j^T into buffer j & 1, once P V of chunk j - 2 has
+      // read the P that the buffer holds.
       auto issue_s = [&](int j) -> bool {
         const int i = 2 * j, slot = i % NSLOT, b = j & 1;
-        if (!mbar_wait_bounded(&kv_full[slot], (i / NSLOT) & 1, a.dev_err)) return false;
-        if (j >= 2 && !mbar_wait_bounded(&s_free[2 * t + b], ((j >> 1) - 1) & 1, a.dev_err))
-          return false;
+        if (!wait(&kv_full[slot], (i / NSLOT) & 1)) return false;
+        if (j >= 2 && !wait(&p_free[2 * t + b], ((j >> 1) - 1) & 1)) return false;
         tmem_fence_after_sync();
         const uint64_t kd = k_desc + static_cast<uint32_t>((slot * Cfg::kSlotBytes) >> 4);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16(s_tmem + b * CHUNK, q_desc + (((kk / 4) * (ROWS * 128) + (kk % 4) * 32) >> 4),
-                    kd + (((kk / 4) * (CHUNK * 128) + (kk % 4) * 32) >> 4), kIdS, kk > 0);
-        umma_commit(&s_full[2 * t + b]);
-        umma_commit(&kv_empty[slot]);
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_bf16(s_tmem + b * CHUNK, q_desc + (((kk / 4) * (ROWS * 128) + (kk % 4) * 32) >> 4),
+                      kd + (((kk / 4) * (CHUNK * 128) + (kk % 4) * 32) >> 4), kIdS, kk > 0);
+          umma_commit(&s_full[2 * t + b]);
+          umma_commit(&kv_empty[slot]);
+        }
+        __syncwarp();
         return true;
       };
-      bool ok = mbar_wait_bounded(&q_full[t], 0, a.dev_err) && issue_s(0);
+      bool ok = wait(&q_full[t], 0) && issue_s(0);
       for (int j = 0; j < nchunks && ok; ++j) {
         // The next chunk's S goes to the tensor core before this chunk's P V.
         if (j + 1 < nchunks && !issue_s(j + 1)) break;
         const int i = 2 * j + 1, slot = i % NSLOT, b = j & 1;
-        ok = mbar_wait_bounded(&kv_full[slot], (i / NSLOT) & 1, a.dev_err);
-        if (ok && j == nchunks - 1 && vt_last < CHUNK) ok = mbar_wait_bounded(v_tail, 0, a.dev_err);
-        ok = ok && mbar_wait_bounded(&p_full[2 * t + b], (j >> 1) & 1, a.dev_err);
+        ok = wait(&kv_full[slot], (i / NSLOT) & 1);
+        if (ok && j == nchunks - 1 && vt_last < CHUNK) ok = wait(v_tail, 0);
+        ok = ok && wait(&p_full[2 * t + b], (j >> 1) & 1);
         if (!ok) break;
         tmem_fence_after_sync();
         const uint64_t vd = v_desc + static_cast<uint32_t>((slot * Cfg::kSlotBytes) >> 4);
-        const uint64_t pd = p_desc + static_cast<uint32_t>((b * Cfg::kPBytes) >> 4);
+        const uint32_t pa = s_tmem + b * CHUNK;  // P over S: 8 columns per K = 16 step
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < CHUNK / 16; ++k)
-          umma_bf16(o_tmem, pd + ((k * 32) >> 4), vd + ((k * 16 * 128) >> 4), kIdO, j > 0 || k > 0);
-        umma_commit(&p_free[2 * t + b]);
-        umma_commit(&kv_empty[slot]);
+          for (int k = 0; k < CHUNK / 16; ++k)
+            umma_bf16_ts(o_tmem, pa + k * 8, vd + ((k * 16 * 128) >> 4), kIdO, j > 0 || k > 0);
+          umma_commit(&p_free[2 * t + b]);
+          umma_commit(&kv_empty[slot]);
+        }
+        __syncwarp();
       }
       // o_last completes once every MMA issued above has; TMEM is freed after it.
-      umma_commit(&o_last[t]);
-      mbar_wait_bounded(&o_last[t], 0, a.dev_err);
+      // elect.sync picks the same lane of the fully active warp every time,
+      // so the MMAs above and this commit share one issuing thread.
+      if (elect_one()) umma_commit(&o_last[t]);
+      __syncwarp();
+      wait(&o_last[t], 0);
     }
-    __syncwarp();
   } else {
     // ---- softmax warps: tile t = warp / 4, thread r owns row r (TMEM lane r) --------
     const int t = warp >> 2;
@@ -333,9 +341,6 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       tmem_fence_after_sync();
       float sv[CHUNK];
       tmem_ld64(trow + b * CHUNK, sv);
-      tmem_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[2 * t + b]);
       const int c0 = span0 + j * CHUNK;
       // Scaled logits: x = s * scale * log2(e). Only chunks that reach past
       // the row's position or the span's end need the mask.
@@ -380,13 +385,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         l *= alpha;
       }
       if (raise) m_used = mx;
-      // P = 2^(x - m_used) <= 2^8, as bf16: row r of the A operand of P V
-      // (128-byte swizzled rows). Its buffer last fed P V of chunk j - 2.
-      if (j >= 2) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait_bounded(&p_free[2 * t + b], ((j >> 1) - 1) & 1, a.dev_err));
-        if (!ok) break;
-      }
+      // P = 2^(x - m_used) <= 2^8, as packed bf16 pairs over the logits.
       uint32_t pk[CHUNK / 2];
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
       if (whole) {
@@ -412,14 +411,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         }
       }
       l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      {
-        uint8_t* prow = pbuf + (2 * t + b) * Cfg::kPBytes + r * 128;
-#pragma unroll
-        for (int w8 = 0; w8 < CHUNK / 8; ++w8)
-          *reinterpret_cast<uint4*>(prow + ((w8 ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * w8], pk[4 * w8 + 1], pk[4 * w8 + 2], pk[4 * w8 + 3]);
-      }
-      fence_proxy_async_smem();
+      tmem_st32_bits(trow + b * CHUNK, pk);
+      tmem_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[2 * t + b]);
     }
