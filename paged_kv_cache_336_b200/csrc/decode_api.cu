@@ -102,6 +102,53 @@ pa_status_t pool_tensor_map(const void* base, int rows, int head_dim, int block_
   return PA_OK;
 }
 
+// q [total_q][num_q_heads][head_dim] (bf16) as a 3-D tensor (head_dim,
+// heads, tokens); one box = 64 columns x `group` heads x `tokens` tokens,
+// 128-byte swizzle: the query rows of one KV head for a run of tokens.
+struct QKey {
+  const void* q;
+  int total_q, heads, head_dim, group, tokens;
+};
+
+struct QCache {
+  static constexpr int kSlots = 8;
+  QKey key[kSlots];
+  CUtensorMap map[kSlots];
+  int used = 0, next = 0;
+};
+
+pa_status_t q_tensor_map(const void* q, int total_q, int num_q_heads, int head_dim, int group,
+                         int tokens, CUtensorMap* out) {
+  thread_local QCache cache;
+  for (int i = 0; i < cache.used; ++i) {
+    const QKey& k = cache.key[i];
+    if (k.q == q && k.total_q == total_q && k.heads == num_q_heads && k.head_dim == head_dim &&
+        k.group == group && k.tokens == tokens) {
+      *out = cache.map[i];
+      return PA_OK;
+    }
+  }
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                        static_cast<cuuint64_t>(total_q)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                           static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(tokens)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMap m;
+  std::memset(&m, 0, sizeof(m));
+  CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", static_cast<int>(r));
+  const int slot = cache.used < QCache::kSlots ? cache.used++ : (cache.next++ % QCache::kSlots);
+  cache.key[slot] = QKey{q, total_q, num_q_heads, head_dim, group, tokens};
+  cache.map[slot] = m;
+  *out = m;
+  return PA_OK;
+}
+
 struct DecodeReq {
   const void* q;
   const void* k_pool;
@@ -712,9 +759,15 @@ pa_status_t run_prefill(const DecodeReq& r, const int32_t* ctx_host, const int32
   a.max_partitions = L.pmax;
   a.scale_log2 = r.scale * 1.4426950408889634f;
   pf.items = reinterpret_cast<const PrefillItem*>(ws + L.items_off);
-  void* args[] = {&tmk, &tmv, &pf};
+  CUtensorMap tmq;
+  void* args3[] = {&tmk, &tmv, &pf};
+  void* args4[] = {&tmk, &tmv, &tmq, &pf};
+  if (pinst.q_map) {
+    st = q_tensor_map(r.q, total_q, r.num_q_heads, r.head_dim, G, std::max(1, pinst.rows / G), &tmq);
+    if (st != PA_OK) return st;
+  }
   err = cudaLaunchKernel(pinst.kernel, dim3(static_cast<unsigned>(items.size())), dim3(pinst.threads),
-                         args, pinst.smem, r.stream);
+                         pinst.q_map ? args4 : args3, pinst.smem, r.stream);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(err));
   if (any_split) {
     int bs = r.block_size;

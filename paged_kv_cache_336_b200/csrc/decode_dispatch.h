@@ -27,6 +27,7 @@ struct PrefixInstance {
   int smem = 0;
   int rows = 64;                 // query rows (tokens x group heads) per tile
   int tiles = 1;                 // tiles per CTA
+  bool q_map = false;            // takes a 3-D tensor map of q after the pool maps
 };
 
 // Shared-prefix pass kernels (bf16); false when (head_dim, block_size) has none.

@@ -78,15 +78,20 @@ static PrefixInstance make_prefill() {
   return r;
 }
 
+// tcgen05 prefill: two 128-row tiles per CTA sharing each K/V chunk (measured
+// faster than one tile per CTA at two CTAs per SM).
+constexpr int kTcPrefillTiles = 2;
+
 template <int BS, int D>
 static PrefixInstance make_tc_prefill() {
-  using Cfg = TcCfg<BS, D>;
+  using Cfg = TcCfg<BS, D, kTcPrefillTiles>;
   PrefixInstance r;
   r.kernel = reinterpret_cast<const void*>(&tc_prefill_kernel<Cfg>);
   r.threads = Cfg::kThreads;
   r.smem = Cfg::kSmem;
   r.rows = Cfg::ROWS;
   r.tiles = Cfg::TILES;
+  r.q_map = true;
   return r;
 }
 

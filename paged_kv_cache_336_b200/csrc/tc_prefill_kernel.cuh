@@ -10,7 +10,10 @@
 // heads) of one sequence, one KV head, one KV partition. Both tiles share
 // every K/V chunk, so the tensor core has one tile's work while the other
 // tile's softmax runs:
-//   warp 8 (producer): streams K_j then V_j of each 64-token chunk (four
+//   warp 8 (producer): loads each tile's Q (one 3-D TMA box per 64 columns:
+//     tokens x group heads x 64, landing as 128-byte swizzled rows in
+//     token-major, head-minor order), then streams K_j then V_j of each
+//     64-token chunk (four
 //     16-token TMA units, 128-byte swizzle: a chunk is one K-major operand
 //     for S and one MN-major operand for P V) into a ring of slots, and
 //     clears the V rows past the span in the last chunk.
@@ -57,19 +60,23 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<uint32_t>(n) << 23));
 }
 
-template <int BS_, int D_>
+template <int BS_, int D_, int TILES_>
 struct TcCfg {
   static constexpr int BS = BS_;
   static constexpr int D = D_;
   static constexpr int ROWS = 128;                      // MMA M: query rows per tile
-  static constexpr int TILES = 2;                       // tiles per CTA
+  static constexpr int TILES = TILES_;                  // tiles per CTA (1 or 2)
   static constexpr int CHUNK = 64;                      // KV tokens per step (N of S, K of P V)
   static constexpr int UR = 16;                         // TMA unit rows
   static constexpr int UPC = CHUNK / UR;                // units per chunk
   static constexpr int KCH = D * 2 / 128;               // 128-byte column chunks of a row
   static constexpr int kQBytes = ROWS * D * 2;          // one tile's Q
   static constexpr int kSlotBytes = CHUNK * D * 2;      // K or V of one chunk
-  static constexpr int NSLOT = 8;                       // ring: K_0 V_0 K_1 V_1 ...
+  // ring: K_0 V_0 K_1 V_1 ...; one-tile CTAs run two per SM (TMEM and
+  // shared memory for two), so one CTA's prologue and epilogue overlap the
+  // other's main loop.
+  static constexpr int NSLOT = TILES == 2 ? 8 : 4;
+  static constexpr int kMinBlocks = TILES == 2 ? 1 : 2;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmem = 1024 + TILES * kQBytes + NSLOT * kSlotBytes + kBarBytes;
   static constexpr int kSoftmaxWarps = 4 * TILES;
@@ -82,13 +89,16 @@ struct TcCfg {
   static_assert(BS % UR == 0, "block size");
   static_assert(32 % UPC == 0, "a chunk's units lie in one 32-unit id batch");
   static_assert(kSmem <= 227 * 1024, "shared memory");
-  static_assert(kTmemCols <= 512, "tensor memory");
+  static_assert(kTmemCols * kMinBlocks <= 512, "tensor memory");
+  static_assert(kSmem * kMinBlocks <= 228 * 1024, "shared memory per SM");
+  static_assert(TILES == 1 || TILES == 2, "tiles");
 };
 
 template <class Cfg>
-__global__ void __launch_bounds__(Cfg::kThreads, 1)
+__global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const PrefillArgs pf) {
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_q, const PrefillArgs pf) {
   constexpr int NSLOT = Cfg::NSLOT;
   constexpr int BS = Cfg::BS;
   constexpr int D = Cfg::D;
@@ -110,7 +120,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
   uint64_t* s_full = bars + 2 * NSLOT;    // [tile][buffer] S MMA done (commit)
   uint64_t* p_full = s_full + 4;          // [tile][buffer] P written (4 warp arrivals)
   uint64_t* p_free = p_full + 4;          // [tile][buffer] P V MMA done (commit)
-  uint64_t* q_full = p_free + 4;          // [tile] Q in shared memory (4 warp arrivals)
+  uint64_t* q_full = p_free + 4;          // [tile] Q in shared memory (TMA bytes)
   uint64_t* o_last = q_full + 2;          // [tile] every MMA of the tile done (commit), once
   uint64_t* v_tail = o_last + 2;          // last chunk's V tail rows cleared (producer), once
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_tail + 1);
@@ -123,7 +133,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
   const int G = a.group;
   const int Hkv = a.num_kv_heads;
   const int TQ = ROWS / G;                                   // query tokens per tile
-  const int ntiles = it.q_count > TQ ? 2 : 1;                // tile 1 idles when empty
+  const int ntiles = (Cfg::TILES == 2 && it.q_count > TQ) ? 2 : 1;  // tile 1 idles when empty
   const int span0 = it.block_begin * BS;
   const int span_end = min(it.block_end * BS, it.kv_end);
   const int nchunks = span_end > span0 ? (span_end - span0 + CHUNK - 1) / CHUNK : 0;
@@ -141,13 +151,14 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       mbar_init(&p_free[i], 1);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&q_full[t], 4);
+      mbar_init(&q_full[t], 1);
       mbar_init(&o_last[t], 1);
     }
     mbar_init(v_tail, 1);
     fence_barrier_init();
     tma_prefetch_descriptor(&tm_k);
     tma_prefetch_descriptor(&tm_v);
+    tma_prefetch_descriptor(&tm_q);
   }
   if (warp == 0) tmem_alloc(tmem_slot, Cfg::kTmemCols);
   tmem_fence_before_sync();
@@ -167,6 +178,17 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
       const int u = batch * 32 + lane;
       return u < nunits ? bt[(span0 + u * UR) / BS] : -1;
     };
+    // Q of each tile first: rows past the query tokens of the array read as 0
+    // (the box's out-of-range fill), rows past the item's tokens are masked.
+    if (elect_one()) {
+      for (int t = 0; t < ntiles; ++t) {
+        mbar_arrive_expect_tx(&q_full[t], KCH * TQ * G * 128);
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(qs + t * Cfg::kQBytes + c * (ROWS * 128), &tm_q, &q_full[t], c * 64,
+                      it.kvh * G, it.q_begin + t * TQ);
+      }
+    }
+    __syncwarp();
     int ids = unit_ids(0);
     int ids_next = unit_ids(1);
     int batch = 0;
@@ -313,24 +335,6 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
     const int lim = valid ? it.p0 + jq : -1;             // last token this row attends to
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + t * Cfg::kTileCols;
     const bool active = t < ntiles;
-    {
-      const int64_t tok = it.q_begin + (valid ? jq : 0);
-      const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
-      const uint4* src = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const __nv_bfloat16*>(a.q) + (tok * a.num_q_heads + h) * D);
-      uint8_t* qt = qs + t * Cfg::kQBytes;
-      if (active) {
-#pragma unroll
-        for (int c = 0; c < D * 2 / 16; ++c) {
-          const uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-          const int cc = c >> 3, w = c & 7;
-          *reinterpret_cast<uint4*>(qt + cc * (ROWS * 128) + r * 128 + ((w ^ (r & 7)) << 4)) = v;
-        }
-        fence_proxy_async_smem();
-      }
-      __syncwarp();
-      if (active && lane == 0) mbar_arrive(&q_full[t]);
-    }
     const float sl2 = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;  // warp-uniform
