@@ -43,21 +43,54 @@
 
 namespace pagedkv {
 
-// 2^x for x <= 8 on the FMA pipe (no MUFU): x = n + f with n = round(x)
-// and f in [-1/2, 1/2]; 2^f by a cubic (least-squares fit at Chebyshev
-// nodes with p(0) = 1: relative error below 1.5e-4, far under bf16's
-// 2^-9 rounding of P); 2^n added into the exponent bits. x is clamped at
-// -125 so the result stays a normal float (2^-125 is 0 next to the
-// chunk's largest P >= 1).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;          // 1.5 * 2^23: rounds x to an integer in t's low bits
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0.05592203f, f, 0.24223731f);
-  p = fmaf(p, f, 0.69312102f);
-  p = fmaf(p, f, 1.f);
-  const int n = __float_as_int(t) - 0x4B400000;
-  return __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<uint32_t>(n) << 23));
+// ---- packed fp32 pairs (Blackwell f32x2 arithmetic) --------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of x <= 8 on the FMA pipe (no MUFU): x = n + f with
+// n = round(x) and f in [-1/2, 1/2]; 2^f by a cubic (least-squares fit at
+// Chebyshev nodes with p(0) = 1: relative error below 1.5e-4, far under
+// bf16's 2^-9 rounding of P); 2^n is added into the exponent bits. With
+// t = x + 1.5 * 2^23 (which rounds x to an integer in t's low mantissa
+// bits), the bits of t shifted left by 23 are n << 23, because the low 9
+// bits of 1.5 * 2^23's pattern are zero. x is clamped at -125 so the result
+// stays a normal float (2^-125 is 0 next to a chunk's largest P >= 1).
+__device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float& p0, float& p1) {
+  float a, b;
+  f2_unpack(x2, a, b);
+  x2 = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t t = f2_add(x2, f2_pack(12582912.f, 12582912.f));
+  const uint64_t u = f2_add(t, f2_pack(-12582912.f, -12582912.f));   // round(x)
+  const uint64_t f = f2_fma(u, f2_pack(-1.f, -1.f), x2);              // x - round(x)
+  uint64_t p = f2_fma(f2_pack(0.05592203f, 0.05592203f), f, f2_pack(0.24223731f, 0.24223731f));
+  p = f2_fma(p, f, f2_pack(0.69312102f, 0.69312102f));
+  p = f2_fma(p, f, f2_pack(1.f, 1.f));
+  float ta, tb, pa, pb;
+  f2_unpack(t, ta, tb);
+  f2_unpack(p, pa, pb);
+  p0 = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ta) << 23));
+  p1 = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(tb) << 23));
 }
 
 template <int BS_, int D_, int TILES_>
@@ -353,11 +386,11 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       if (whole) {
         float m8[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = sv[i];
-#pragma unroll
-        for (int i = 8; i < CHUNK; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i]);
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+        for (int k = 0; k < 8; ++k) {
+          const float* v = sv + 8 * k;
+          m8[k] = fmax3(fmax3(v[0], v[1], v[2]), fmax3(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+        }
+        mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
       } else {
         mx = -INFINITY;
 #pragma unroll
@@ -393,17 +426,28 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       uint32_t pk[CHUNK / 2];
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
       if (whole) {
-        const float nm = -m_used;
+        const uint64_t sl2_2 = f2_pack(sl2, sl2);
+        const uint64_t nm2 = f2_pack(-m_used, -m_used);
+        uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int i = 0; i < CHUNK; i += 2) {
-          // pairs 3, 7, 11, ... on the FMA pipe, the rest on MUFU
-          const bool poly = (i & 6) == 6;
-          const float x0 = fmaf(sv[i], sl2, nm), x1 = fmaf(sv[i + 1], sl2, nm);
-          const float p0 = poly ? exp2_fma(x0) : fast_exp2(x0);
-          const float p1 = poly ? exp2_fma(x1) : fast_exp2(x1);
-          s4[(i >> 1) & 3] += p0 + p1;
+          const uint64_t x2 = f2_fma(f2_pack(sv[i], sv[i + 1]), sl2_2, nm2);
+          float p0, p1;
+          if ((i & 6) == 6) {  // pairs 3, 7, 11, ... on the FMA pipe, the rest on MUFU
+            exp2_fma_pair(x2, p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(p0, p1));
           pk[i >> 1] = pack_bf16x2(p0, p1);
         }
+        float a0, a1, b0, b1;
+        f2_unpack(acc2[0], a0, a1);
+        f2_unpack(acc2[1], b0, b1);
+        s4[0] = a0; s4[1] = a1; s4[2] = b0; s4[3] = b1;
       } else {
         const float mu = (m_used == -INFINITY) ? 0.f : m_used;  // a row with nothing yet: all p = 0
 #pragma unroll
