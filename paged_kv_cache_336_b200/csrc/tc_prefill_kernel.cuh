@@ -28,8 +28,10 @@
 //     is written back as packed bf16 over the logits it came from (the A
 //     operand of P V); m moves only when the chunk's max exceeds it by more
 //     than 2^8, and then O (in TMEM) and l are scaled by 2^(m_old - m_new).
-//     A quarter of the exponentials run as a polynomial on the FMA pipe, so
-//     the MUFU unit (16 results per clock per SM) does not set the pace.
+//     The unmasked path runs on packed fp32 pairs (f32x2 FMA/add) and a
+//     three-input max. The softmax is bound by issue slots, not by MUFU:
+//     moving a share of the exponentials to an FMA-pipe polynomial measured
+//     slower at every share tried (1/4, 3/8, 1/2).
 // TMEM per tile: two 64-column S / P buffers (chunk parity) and head_dim O
 // columns; 512 columns for the CTA. The tensor core reads its shared-memory
 // operands at about 128 bytes per clock per SM, so P stays out of shared
@@ -66,31 +68,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// 2^x for a pair of x <= 8 on the FMA pipe (no MUFU): x = n + f with
-// n = round(x) and f in [-1/2, 1/2]; 2^f by a cubic (least-squares fit at
-// Chebyshev nodes with p(0) = 1: relative error below 1.5e-4, far under
-// bf16's 2^-9 rounding of P); 2^n is added into the exponent bits. With
-// t = x + 1.5 * 2^23 (which rounds x to an integer in t's low mantissa
-// bits), the bits of t shifted left by 23 are n << 23, because the low 9
-// bits of 1.5 * 2^23's pattern are zero. x is clamped at -125 so the result
-// stays a normal float (2^-125 is 0 next to a chunk's largest P >= 1).
-__device__ __forceinline__ void exp2_fma_pair(uint64_t x2, float& p0, float& p1) {
-  float a, b;
-  f2_unpack(x2, a, b);
-  x2 = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
-  const uint64_t t = f2_add(x2, f2_pack(12582912.f, 12582912.f));
-  const uint64_t u = f2_add(t, f2_pack(-12582912.f, -12582912.f));   // round(x)
-  const uint64_t f = f2_fma(u, f2_pack(-1.f, -1.f), x2);              // x - round(x)
-  uint64_t p = f2_fma(f2_pack(0.05592203f, 0.05592203f), f, f2_pack(0.24223731f, 0.24223731f));
-  p = f2_fma(p, f, f2_pack(0.69312102f, 0.69312102f));
-  p = f2_fma(p, f, f2_pack(1.f, 1.f));
-  float ta, tb, pa, pb;
-  f2_unpack(t, ta, tb);
-  f2_unpack(p, pa, pb);
-  p0 = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ta) << 23));
-  p1 = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(tb) << 23));
 }
 
 template <int BS_, int D_, int TILES_>
@@ -331,9 +308,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
         __syncwarp();
         return true;
       };
+      // Issuing whichever of S and P V became ready first measured the same
+      // as this fixed order (S of the next chunk, then P V of this one).
       bool ok = wait(&q_full[t], 0) && issue_s(0);
       for (int j = 0; j < nchunks && ok; ++j) {
-        // The next chunk's S goes to the tensor core before this chunk's P V.
         if (j + 1 < nchunks && !issue_s(j + 1)) break;
         const int i = 2 * j + 1, slot = i % NSLOT, b = j & 1;
         ok = wait(&kv_full[slot], (i / NSLOT) & 1);
@@ -432,15 +410,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
 #pragma unroll
         for (int i = 0; i < CHUNK; i += 2) {
           const uint64_t x2 = f2_fma(f2_pack(sv[i], sv[i + 1]), sl2_2, nm2);
-          float p0, p1;
-          if ((i & 6) == 6) {  // pairs 3, 7, 11, ... on the FMA pipe, the rest on MUFU
-            exp2_fma_pair(x2, p0, p1);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p0 = fast_exp2(x0);
-            p1 = fast_exp2(x1);
-          }
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
           acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(p0, p1));
           pk[i >> 1] = pack_bf16x2(p0, p1);
         }
