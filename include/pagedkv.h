@@ -445,6 +445,18 @@ pa_status_t pa_bm_stats(pa_bm_t bm, pa_bm_stats_t* stats);
  * A block-manager failure (PA_ERR_NO_FREE_BLOCKS / PA_ERR_INVALID_ARG)
  * returns before anything is enqueued, state unchanged. A CUDA error after
  * the manager step leaves the manager with the step applied.
+ *
+ * Pipelining (optional): with the three fields at the end of the struct set
+ * (pa_step_pipeline_create), the uploads run on `copy_stream`: they wait
+ * for `compute_done` (this set's previous step, decode and download, is
+ * finished with the device staging) and the kernels on `stream` wait for
+ * `upload_done`. The host staging of a set is rewritten only after that
+ * set's previous uploads completed (the call first waits on `upload_done`).
+ * A caller that alternates two buffer sets with synchronize = 0 overlaps a
+ * step's uploads and host work with the previous step's kernels. It keeps
+ * q_host, k_new_host and v_new_host unchanged until the step's uploads are
+ * done, and reads out_host after synchronising `stream`. Pool updates stay
+ * ordered on `stream`. With the fields NULL everything runs on `stream`.
  * ========================================================================= */
 typedef struct {
   /* shape and cache */
@@ -470,7 +482,18 @@ typedef struct {
   int64_t* h_pairs;         /* [max_seqs][2] */
   int32_t* h_tables;        /* [max_seqs][max_blocks_per_seq] */
   int32_t* h_context_lens;  /* [max_seqs] */
+  /* pipelining (optional, NULL = off; see above) */
+  void* upload_done;        /* cudaEvent_t recorded on copy_stream after the uploads */
+  void* compute_done;       /* cudaEvent_t recorded on `stream` after the decode */
+  void* copy_stream;        /* cudaStream_t for the uploads and the download */
 } pa_step_buffers_t;
+
+/* Creates the two events of a buffer set's pipelining fields (timing
+ * disabled) and stores copy_stream; the caller owns the stream.
+ * pa_step_pipeline_destroy destroys the events and clears the three fields.
+ * Setup-time calls, not for the hot path. */
+pa_status_t pa_step_pipeline_create(pa_step_buffers_t* buf, void* copy_stream);
+pa_status_t pa_step_pipeline_destroy(pa_step_buffers_t* buf);
 
 /* Number of host->device and device->host bytes one pa_decode_step call of
  * n sequences moves when it makes `num_copies` copy-on-write copies. */

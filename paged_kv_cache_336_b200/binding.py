@@ -75,6 +75,7 @@ class StepBuffers(ctypes.Structure):
         ("d_q", _P), ("d_k_new", _P), ("d_v_new", _P), ("d_out", _P),
         ("d_slots", _P), ("d_pairs", _P), ("d_tables", _P), ("d_context_lens", _P),
         ("h_slots", _P), ("h_pairs", _P), ("h_tables", _P), ("h_context_lens", _P),
+        ("upload_done", _P), ("compute_done", _P), ("copy_stream", _P),
     ]
 
 # name -> (restype, argtypes); mirrors include/pagedkv.h
@@ -124,6 +125,8 @@ _SIGNATURES = {
     "pa_decode_step_d2h_bytes": (_SZ, [ctypes.POINTER(StepBuffers), _I]),
     "pa_decode_step": (_I, [_P, ctypes.POINTER(StepBuffers), _P, _I, _P, _P, _P, _P,
                             ctypes.POINTER(_I), _I, _P, _P]),
+    "pa_step_pipeline_create": (_I, [ctypes.POINTER(StepBuffers), _P]),
+    "pa_step_pipeline_destroy": (_I, [ctypes.POINTER(StepBuffers)]),
 }
 
 
@@ -596,7 +599,9 @@ class DecodeStepper:
     decode, download (and, by default, stream synchronisation)."""
 
     def __init__(self, bm: "BlockManager", k_pool, v_pool, num_q_heads: int, scale: float,
-                 max_seqs: int, partition_tokens: int = 512):
+                 max_seqs: int, partition_tokens: int = 512, copy_stream=None):
+        """copy_stream: a torch.cuda.Stream for the uploads (pipelined steps,
+        see pa_step_pipeline_create); None runs everything on the step's stream."""
         torch = _torch()
         _require_cuda(k_pool, v_pool)
         NB, Hkv, BS, D = k_pool.shape
@@ -631,6 +636,17 @@ class DecodeStepper:
         b.h_slots, b.h_pairs = _ptr(self.h_slots), _ptr(self.h_pairs)
         b.h_tables, b.h_context_lens = _ptr(self.h_tables), _ptr(self.h_ctx)
         self.buffers = b
+        self.copy_stream = copy_stream
+        if copy_stream is not None:
+            _check(library().pa_step_pipeline_create(ctypes.byref(self.buffers),
+                                                     _stream_ptr(copy_stream)))
+
+    def __del__(self):
+        try:
+            if getattr(self, "copy_stream", None) is not None:
+                library().pa_step_pipeline_destroy(ctypes.byref(self.buffers))
+        except Exception:
+            pass
 
     def h2d_bytes(self, n: int, num_copies: int) -> int:
         return int(library().pa_decode_step_h2d_bytes(ctypes.byref(self.buffers), n, num_copies))

@@ -60,25 +60,49 @@ pa_status_t pa_decode_step(pa_bm_t bm, const pa_step_buffers_t* b, const int64_t
       b->h_tables == nullptr || b->h_context_lens == nullptr)
     return fail(PA_ERR_INVALID_ARG, "NULL staging buffer");
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  const bool piped = b->copy_stream != nullptr;
+  if (piped && (b->upload_done == nullptr || b->compute_done == nullptr))
+    return fail(PA_ERR_INVALID_ARG, "copy_stream set without upload_done / compute_done events");
+  cudaStream_t cs = piped ? static_cast<cudaStream_t>(b->copy_stream) : stream;
+  cudaEvent_t upload_done = static_cast<cudaEvent_t>(b->upload_done);
+  cudaEvent_t compute_done = static_cast<cudaEvent_t>(b->compute_done);
+
+  // 0. this set's host staging is rewritten below: its previous uploads
+  // must have read it
+  pa_status_t st;
+  if (upload_done != nullptr &&
+      (st = cuda_check(cudaEventSynchronize(upload_done), "wait for previous uploads")) != PA_OK)
+    return st;
 
   // 1. block manager: one slot per sequence, copies where a tail is shared
   int ncow = 0;
-  pa_status_t st = pa_bm_append_slots(bm, seq_ids, n, b->h_slots, b->h_pairs, &ncow);
+  st = pa_bm_append_slots(bm, seq_ids, n, b->h_slots, b->h_pairs, &ncow);
   if (st != PA_OK) return st;
   st = pa_bm_export(bm, seq_ids, n, b->h_tables, b->h_context_lens, -1);
   if (st != PA_OK) return st;
   if (num_copies) *num_copies = ncow;
 
-  // 2. uploads
-  if ((st = cuda_check(cudaMemcpyAsync(b->d_q, q_host, q_bytes(b, n), cudaMemcpyHostToDevice, stream), "upload q")) != PA_OK) return st;
-  if ((st = cuda_check(cudaMemcpyAsync(b->d_k_new, k_new_host, kv_bytes(b, n), cudaMemcpyHostToDevice, stream), "upload k_new")) != PA_OK) return st;
-  if ((st = cuda_check(cudaMemcpyAsync(b->d_v_new, v_new_host, kv_bytes(b, n), cudaMemcpyHostToDevice, stream), "upload v_new")) != PA_OK) return st;
-  if ((st = cuda_check(cudaMemcpyAsync(b->d_slots, b->h_slots, static_cast<size_t>(n) * 8, cudaMemcpyHostToDevice, stream), "upload slots")) != PA_OK) return st;
-  if ((st = cuda_check(cudaMemcpyAsync(b->d_tables, b->h_tables, static_cast<size_t>(n) * b->max_blocks_per_seq * 4, cudaMemcpyHostToDevice, stream), "upload tables")) != PA_OK) return st;
-  if ((st = cuda_check(cudaMemcpyAsync(b->d_context_lens, b->h_context_lens, static_cast<size_t>(n) * 4, cudaMemcpyHostToDevice, stream), "upload lengths")) != PA_OK) return st;
-  if (ncow > 0 &&
-      (st = cuda_check(cudaMemcpyAsync(b->d_pairs, b->h_pairs, static_cast<size_t>(ncow) * 16, cudaMemcpyHostToDevice, stream), "upload copy pairs")) != PA_OK)
+  // 2. uploads (on the copy stream once this set's device staging is no longer
+  // read by its previous step: compute_done was recorded after that step's
+  // download; waiting on a never-recorded event returns at once)
+  if (piped && (st = cuda_check(cudaStreamWaitEvent(cs, compute_done, 0), "order uploads")) != PA_OK)
     return st;
+  if ((st = cuda_check(cudaMemcpyAsync(b->d_q, q_host, q_bytes(b, n), cudaMemcpyHostToDevice, cs), "upload q")) != PA_OK) return st;
+  if ((st = cuda_check(cudaMemcpyAsync(b->d_k_new, k_new_host, kv_bytes(b, n), cudaMemcpyHostToDevice, cs), "upload k_new")) != PA_OK) return st;
+  if ((st = cuda_check(cudaMemcpyAsync(b->d_v_new, v_new_host, kv_bytes(b, n), cudaMemcpyHostToDevice, cs), "upload v_new")) != PA_OK) return st;
+  if ((st = cuda_check(cudaMemcpyAsync(b->d_slots, b->h_slots, static_cast<size_t>(n) * 8, cudaMemcpyHostToDevice, cs), "upload slots")) != PA_OK) return st;
+  if ((st = cuda_check(cudaMemcpyAsync(b->d_tables, b->h_tables, static_cast<size_t>(n) * b->max_blocks_per_seq * 4, cudaMemcpyHostToDevice, cs), "upload tables")) != PA_OK) return st;
+  if ((st = cuda_check(cudaMemcpyAsync(b->d_context_lens, b->h_context_lens, static_cast<size_t>(n) * 4, cudaMemcpyHostToDevice, cs), "upload lengths")) != PA_OK) return st;
+  if (ncow > 0 &&
+      (st = cuda_check(cudaMemcpyAsync(b->d_pairs, b->h_pairs, static_cast<size_t>(ncow) * 16, cudaMemcpyHostToDevice, cs), "upload copy pairs")) != PA_OK)
+    return st;
+
+  if (piped) {
+    if ((st = cuda_check(cudaEventRecord(upload_done, cs), "record uploads")) != PA_OK) return st;
+    if ((st = cuda_check(cudaStreamWaitEvent(stream, upload_done, 0), "order uploads")) != PA_OK) return st;
+  } else if (upload_done != nullptr) {
+    if ((st = cuda_check(cudaEventRecord(upload_done, stream), "record uploads")) != PA_OK) return st;
+  }
 
   // 3. kernels: copy-on-write copies before the append writes into them
   const size_t block_bytes = static_cast<size_t>(b->num_kv_heads) * b->block_size * b->head_dim * elt(b->dtype);
@@ -95,9 +119,34 @@ pa_status_t pa_decode_step(pa_bm_t bm, const pa_step_buffers_t* b, const int64_t
                        b->d_out, dev_err, stream);
   if (st != PA_OK) return st;
 
-  // 4. download
+  // 4. download, on `stream` behind the decode; then mark this set's device
+  // staging free for its next uploads
   if ((st = cuda_check(cudaMemcpyAsync(out_host, b->d_out, q_bytes(b, n), cudaMemcpyDeviceToHost, stream), "download out")) != PA_OK) return st;
+  if (piped && (st = cuda_check(cudaEventRecord(compute_done, stream), "record step")) != PA_OK) return st;
   if (synchronize && (st = cuda_check(cudaStreamSynchronize(stream), "synchronize")) != PA_OK) return st;
+  return ok();
+}
+
+pa_status_t pa_step_pipeline_create(pa_step_buffers_t* b, void* copy_stream) {
+  if (b == nullptr || copy_stream == nullptr) return fail(PA_ERR_INVALID_ARG, "buffers or copy_stream is NULL");
+  cudaEvent_t e1 = nullptr, e2 = nullptr;
+  pa_status_t st = cuda_check(cudaEventCreateWithFlags(&e1, cudaEventDisableTiming), "create event");
+  if (st != PA_OK) return st;
+  if ((st = cuda_check(cudaEventCreateWithFlags(&e2, cudaEventDisableTiming), "create event")) != PA_OK) {
+    cudaEventDestroy(e1);
+    return st;
+  }
+  b->upload_done = e1;
+  b->compute_done = e2;
+  b->copy_stream = copy_stream;
+  return ok();
+}
+
+pa_status_t pa_step_pipeline_destroy(pa_step_buffers_t* b) {
+  if (b == nullptr) return fail(PA_ERR_INVALID_ARG, "buffers is NULL");
+  if (b->upload_done) cudaEventDestroy(static_cast<cudaEvent_t>(b->upload_done));
+  if (b->compute_done) cudaEventDestroy(static_cast<cudaEvent_t>(b->compute_done));
+  b->upload_done = b->compute_done = b->copy_stream = nullptr;
   return ok();
 }
 

@@ -32,7 +32,9 @@ def kernel(request, monkeypatch):
 
 @pytest.mark.parametrize("G,bs,partition,D", [(1, 16, 64, 128), (4, 16, 32, 128), (8, 32, 64, 128),
                                               (4, 32, 4096, 128), (16, 16, 128, 128),
-                                              (2, 16, 64, 64), (8, 32, 4096, 64)])
+                                              (2, 16, 64, 64), (8, 32, 4096, 64),
+                                              # groups that do not divide a 128-row tile
+                                              (6, 16, 64, 128), (3, 32, 4096, 64)])
 def test_prefill_matches_oracle(kernel, G, bs, partition, D):
     # (context length, new tokens): prompt, chunk on prior context, single token, odd sizes
     plan = [(75, 75), (300, 37), (129, 1), (64, 64), (500, 130), (17, 9)]

@@ -63,3 +63,61 @@ def test_decode_step_matches_oracle(dtype, Hq, Hkv, bs):
     assert int(err.item()) == 0
     assert total_cow == 2          # sequences 2 and 0 copy; 1 is the last holder
     assert np.array_equal(to_f64(k_pool), k_ref) and np.array_equal(to_f64(v_pool), v_ref)
+
+
+def _step_setup(seed, NB=60, bs=16, MBS=12, Hq=8, Hkv=2, D=128):
+    order = np.random.default_rng(seed).permutation(NB).astype(np.int32)
+    bm = binding.BlockManager(NB, bs, MBS, order)
+    bm.allocate(0, 2 * bs + 5)
+    bm.allocate(3, 3 * bs)
+    bm.allocate(4, 1)
+    bm.fork(0, 1)
+    bm.fork(0, 2)
+    w = workloads.random_small(seed, num_seqs=1, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                               block_size=bs, dtype=workloads.BF16, max_ctx=1)
+    w.num_blocks = NB
+    k_pool, v_pool = workloads.draw_pools(w, "cuda")
+    return bm, w, k_pool, v_pool
+
+
+def test_pipelined_steps_equal_synchronous_steps():
+    """Two buffer sets alternated with synchronize = 0, uploads on a copy
+    stream (pa_step_pipeline_create): every step's output, the copy counts
+    and the final pools are bit-identical to one-at-a-time synchronous steps
+    from the same start."""
+    Hq, D, steps = 8, 128, 10
+    seqs = np.array([2, 0, 3, 4, 1], dtype=np.int64)
+    scale = 1.0 / np.sqrt(D)
+    runs = []
+    for piped in (False, True):
+        bm, w, k_pool, v_pool = _step_setup(33)
+        inputs = []
+        for step in range(steps):
+            q = workloads.draw_queries(w, len(seqs), step=step).pin_memory()
+            kn, vn = workloads.draw_new_kv(w, len(seqs), step=step)
+            inputs.append((q, kn.pin_memory(), vn.pin_memory()))
+        outs = [torch.empty_like(inputs[0][0]).pin_memory() for _ in range(steps)]
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        if piped:
+            copy_stream = torch.cuda.Stream()
+            sets = [binding.DecodeStepper(bm, k_pool, v_pool, Hq, scale, max_seqs=8,
+                                          partition_tokens=16, copy_stream=copy_stream)
+                    for _ in range(2)]
+        else:
+            sets = [binding.DecodeStepper(bm, k_pool, v_pool, Hq, scale, max_seqs=8,
+                                          partition_tokens=16)]
+        stream = torch.cuda.current_stream()
+        cows = []
+        for step in range(steps):
+            q, kn, vn = inputs[step]
+            cows.append(sets[step % len(sets)].step(seqs, q, kn, vn, outs[step],
+                                                    synchronize=not piped, dev_err=err,
+                                                    stream=stream))
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        runs.append((cows, [o.clone() for o in outs], k_pool.clone().cpu(), v_pool.clone().cpu()))
+    (c0, o0, k0, v0), (c1, o1, k1, v1) = runs
+    assert c0 == c1 and sum(c0) > 0
+    for step in range(steps):
+        assert torch.equal(o0[step], o1[step]), f"step {step}"
+    assert torch.equal(k0, k1) and torch.equal(v0, v1)
