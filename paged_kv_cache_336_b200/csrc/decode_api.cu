@@ -464,9 +464,17 @@ constexpr int kMaxPrefixParts = 16;
 constexpr int kPrefixRows = 64;  // query rows per prefix CTA (4 warps x 16)
 
 struct PrefixLayout {
-  size_t skip_off, base_off, members_off, items_off;
+  size_t skip_off, base_off, members_off, items_off, qtiles_off, qpack_off;
   SplitExtras ex;
-  size_t max_items;
+  size_t max_items, max_qtiles;
+};
+
+constexpr int kTcPrefixRows = 128;  // query rows per tcgen05 prefix tile
+
+// Q rows of one tcgen05 prefix tile: members [member_begin, + count) of the
+// packed member list, heads kvh * group .. + group.
+struct QPackTile {
+  int32_t member_begin, count, kvh, pad;
 };
 
 PrefixLayout prefix_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
@@ -475,17 +483,49 @@ PrefixLayout prefix_layout(int num_seqs, int num_q_heads, int num_kv_heads, int 
   const int pb = partition_tokens / block_size;
   L.ex.pmax = kMaxPrefixParts + (max_blocks_per_seq + pb - 1) / pb + 1;
   const size_t B = static_cast<size_t>(num_seqs);
+  const size_t G = static_cast<size_t>(std::max(1, num_q_heads / std::max(1, num_kv_heads)));
   L.max_items = B * static_cast<size_t>(num_kv_heads) * kMaxPrefixParts;
+  // row tiles: each group's members in runs of 128 / G, per KV head
+  L.max_qtiles = (B + (B * G + kTcPrefixRows - 1) / kTcPrefixRows) * static_cast<size_t>(num_kv_heads);
   L.skip_off = kWorkspaceHeader;
   L.base_off = L.skip_off + align256(B * 4);
   L.members_off = L.base_off + align256(B * 4);
   L.items_off = L.members_off + align256(B * 4);
+  L.qtiles_off = L.items_off + align256(L.max_items * std::max(sizeof(PrefixItem), sizeof(PrefillItem)));
+  L.qpack_off = L.qtiles_off + align256(L.max_qtiles * sizeof(QPackTile));
+  const size_t qpack_bytes = L.max_qtiles * kTcPrefixRows * static_cast<size_t>(head_dim) * 2;
   const size_t rows = B * num_q_heads * L.ex.pmax;
-  L.ex.m_off = L.items_off + align256(L.max_items * sizeof(PrefixItem));
+  L.ex.m_off = L.qpack_off + align256(qpack_bytes);
   L.ex.l_off = L.ex.m_off + align256(rows * 4);
   L.ex.acc_off = L.ex.l_off + align256(rows * 4);
   L.ex.total = L.ex.acc_off + align256(rows * static_cast<size_t>(head_dim) * 4);
   return L;
+}
+
+// Packs the query rows of each tcgen05 prefix tile contiguously ([tile][token
+// = member][head][head_dim], rows past the tile's members zero) so that one
+// 3-D TMA box loads a tile's Q. One CTA per tile, one thread per row.
+__global__ void __launch_bounds__(kTcPrefixRows) q_pack_kernel(const __nv_bfloat16* __restrict__ q,
+                                                               const int32_t* __restrict__ members,
+                                                               const QPackTile* __restrict__ tiles,
+                                                               int group, int num_q_heads, int head_dim,
+                                                               int tokens, __nv_bfloat16* __restrict__ qpack) {
+  grid_dependents_launch();  // the prefix kernel may start; it waits before reading qpack
+  const QPackTile tl = tiles[blockIdx.x];
+  const int r = threadIdx.x;
+  const int m = r / group, g = r % group;
+  if (m >= tokens) return;
+  uint4* dst = reinterpret_cast<uint4*>(
+      qpack + ((static_cast<int64_t>(blockIdx.x) * tokens + m) * group + g) * head_dim);
+  const int n16 = head_dim / 8;
+  if (m < tl.count) {
+    const int64_t s = members[tl.member_begin + m];
+    const uint4* src = reinterpret_cast<const uint4*>(
+        q + (s * num_q_heads + static_cast<int64_t>(tl.kvh) * group + g) * head_dim);
+    for (int i = 0; i < n16; ++i) dst[i] = src[i];
+  } else {
+    for (int i = 0; i < n16; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
 }
 
 pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_groups,
@@ -495,8 +535,17 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
   pa_status_t st = validate_and_pick(r, &inst);
   if (st != PA_OK) return st;
   if (r.dtype != PA_BF16) return fail(PA_ERR_UNSUPPORTED, "pa_decode_shared_prefix is bf16 only");
+  // PAGEDKV_PREFIX_KERNEL=tcgen05 selects the tcgen05 pass (the prefill kernel
+  // with one 128-row tile per CTA, Q packed by a small kernel). Its prefix
+  // kernel is faster than the 64-row mma.sync pass (37.6 vs 41.3 us on the
+  // 8 x 4008-token, 16-branch workload), but the whole call measured slower
+  // (70.3 vs 69.0 us): two 100 KB CTAs per SM leave no room for the suffix
+  // kernel that runs alongside. The default stays mma.sync.
+  const char* kname = std::getenv("PAGEDKV_PREFIX_KERNEL");
+  const bool tc = kname != nullptr && std::strcmp(kname, "tcgen05") == 0;
   PrefixInstance pinst;
-  if (!find_prefix_bf16(r.head_dim, r.block_size, &pinst))
+  if (!(tc ? find_tc_prefix_bf16(r.head_dim, r.block_size, &pinst)
+           : find_prefix_bf16(r.head_dim, r.block_size, &pinst)))
     return fail(PA_ERR_UNSUPPORTED, "no shared-prefix kernel for head_dim=%d block_size=%d",
                 r.head_dim, r.block_size);
   if (partition_tokens <= 0 || partition_tokens % r.block_size != 0)
@@ -516,14 +565,19 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
     return fail(PA_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", workspace_bytes, L.ex.total);
   if (B == 0) return ok();
 
+  const int chunk_rows = tc ? kTcPrefixRows : kPrefixRows;
   thread_local std::vector<int32_t> skip, base, mem;
   thread_local std::vector<PrefixItem> items;
+  thread_local std::vector<PrefillItem> tc_items;
+  thread_local std::vector<QPackTile> qtiles;
   thread_local std::vector<char> seen;
   skip.assign(B, 0);
   base.assign(B, 0);
   seen.assign(B, 0);
   mem.clear();
   items.clear();
+  tc_items.clear();
+  qtiles.clear();
   // groups: validate, and find the prefix partition size
   int64_t total_blocks = 0;
   int max_blocks = 0;
@@ -539,7 +593,7 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
       if (m < 0 || m >= B || seen[m]) return fail(PA_ERR_INVALID_ARG, "group member %d invalid or repeated", m);
       seen[m] = 1;
     }
-    const int chunks = ((b1 - b0) * G + kPrefixRows - 1) / kPrefixRows;
+    const int chunks = ((b1 - b0) * G + chunk_rows - 1) / chunk_rows;
     many_chunks = many_chunks || chunks > 1;
     total_blocks += static_cast<int64_t>(blocks[g]) * chunks * r.num_kv_heads;
     max_blocks = std::max(max_blocks, blocks[g]);
@@ -547,13 +601,28 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
   DeviceInfo dinfo;
   st = device_info(&dinfo);
   if (st != PA_OK) return st;
-  // Partition so that there are about three items per SM (one wave at three
-  // CTAs per SM), at most kMaxPrefixParts per group, and at least four blocks
-  // each; fewer partitions mean fewer partials for the merge.
-  int pbp = static_cast<int>((total_blocks + 3LL * dinfo.sms - 1) / (3LL * dinfo.sms));
+  // Partition so that the items fill about one wave (the kernel's CTAs per
+  // SM x SMs), at most kMaxPrefixParts per group, and at least four blocks
+  // each; fewer partitions mean fewer partials for the merge. Rounding up the
+  // partitions of each group can overflow the wave, so the size grows until
+  // the items fit (a second, nearly empty wave costs a whole item's time).
+  const int per_sm = tc ? 2 : 3;
+  const int64_t slots = static_cast<int64_t>(per_sm) * dinfo.sms;
+  int pbp = static_cast<int>((total_blocks + slots - 1) / slots);
   pbp = std::max(pbp, (max_blocks + kMaxPrefixParts - 1) / kMaxPrefixParts);
   pbp = std::max(pbp, 4);
-  const int per_chunk = std::max(1, kPrefixRows / G);
+  auto count_items = [&](int part_blocks) {
+    int64_t n = 0;
+    for (int g = 0; g < num_groups; ++g) {
+      const int members_g = offs[g + 1] - offs[g];
+      if (members_g == 0) continue;
+      const int chunks = (members_g * G + chunk_rows - 1) / chunk_rows;
+      n += static_cast<int64_t>((blocks[g] + part_blocks - 1) / part_blocks) * chunks * r.num_kv_heads;
+    }
+    return n;
+  };
+  while (pbp < max_blocks && count_items(pbp) > slots) ++pbp;
+  const int per_chunk = std::max(1, chunk_rows / G);
   for (int g = 0; g < num_groups; ++g) {
     const int b0 = offs[g], b1 = offs[g + 1];
     if (b1 - b0 == 0) continue;
@@ -566,12 +635,24 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
     }
     for (int c = first; c < first + (b1 - b0); c += per_chunk) {
       const int cnt = std::min(per_chunk, first + (b1 - b0) - c);
-      for (int h = 0; h < r.num_kv_heads; ++h)
-        for (int p = 0; p < nparts; ++p)
-          items.push_back(PrefixItem{members[b0], c, cnt, p * pbp, std::min(blocks[g], (p + 1) * pbp), h, p, 0});
+      for (int h = 0; h < r.num_kv_heads; ++h) {
+        // tcgen05: the tile's Q rows are packed at token index tile * per_chunk;
+        // no causal limit (every row sees the whole shared span: p0 past it)
+        const int tile = static_cast<int>(qtiles.size());
+        if (tc) qtiles.push_back(QPackTile{c, cnt, h, 0});
+        for (int p = 0; p < nparts; ++p) {
+          const int bb = p * pbp, be = std::min(blocks[g], (p + 1) * pbp);
+          if (tc)
+            tc_items.push_back(PrefillItem{members[b0], tile * per_chunk, cnt, be * r.block_size, bb, be,
+                                           be * r.block_size, h, p, 0, 0, c});
+          else
+            items.push_back(PrefixItem{members[b0], c, cnt, bb, be, h, p, 0});
+        }
+      }
     }
   }
-  if (items.size() > L.max_items) return fail(PA_ERR_INVALID_ARG, "too many prefix items");
+  if (items.size() > L.max_items || tc_items.size() > L.max_items || qtiles.size() > L.max_qtiles)
+    return fail(PA_ERR_INVALID_ARG, "too many prefix items");
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaError_t err;
@@ -585,11 +666,68 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
       (err = cudaMemcpyAsync(ws + L.items_off, items.data(), items.size() * sizeof(PrefixItem),
                              cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
     return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
+  if (!tc_items.empty() &&
+      ((err = cudaMemcpyAsync(ws + L.items_off, tc_items.data(), tc_items.size() * sizeof(PrefillItem),
+                              cudaMemcpyHostToDevice, r.stream)) != cudaSuccess ||
+       (err = cudaMemcpyAsync(ws + L.qtiles_off, qtiles.data(), qtiles.size() * sizeof(QPackTile),
+                              cudaMemcpyHostToDevice, r.stream)) != cudaSuccess))
+    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
 
   SplitExtras ex = L.ex;
   ex.seq_skip_blocks = reinterpret_cast<const int32_t*>(ws + L.skip_off);
   ex.seq_part_base = reinterpret_cast<const int32_t*>(ws + L.base_off);
 
+  if (!tc_items.empty()) {
+    auto* qpack = reinterpret_cast<__nv_bfloat16*>(ws + L.qpack_off);
+    q_pack_kernel<<<static_cast<unsigned>(qtiles.size()), kTcPrefixRows, 0, r.stream>>>(
+        static_cast<const __nv_bfloat16*>(r.q), reinterpret_cast<const int32_t*>(ws + L.members_off),
+        reinterpret_cast<const QPackTile*>(ws + L.qtiles_off), G, r.num_q_heads, r.head_dim, per_chunk,
+        qpack);
+    if ((err = cudaGetLastError()) != cudaSuccess) return fail(PA_ERR_CUDA, "q pack launch: %s", cudaGetErrorString(err));
+    st = prepare_kernel(pinst.kernel, pinst.smem);
+    if (st != PA_OK) return st;
+    const int rows = r.num_blocks * r.num_kv_heads * r.block_size;
+    CUtensorMap tmk, tmv, tmq;
+    st = pool_tensor_map(r.k_pool, rows, r.head_dim, r.block_size, r.dtype, &tmk);
+    if (st != PA_OK) return st;
+    st = pool_tensor_map(r.v_pool, rows, r.head_dim, r.block_size, r.dtype, &tmv);
+    if (st != PA_OK) return st;
+    st = q_tensor_map(qpack, static_cast<int>(qtiles.size()) * per_chunk, G, r.head_dim, G, per_chunk, &tmq);
+    if (st != PA_OK) return st;
+    PrefillArgs pf{};
+    DecodeArgs& a = pf.d;
+    a.q = r.q;
+    a.block_tables = r.block_tables;
+    a.context_lens = r.context_lens;
+    a.part_m = reinterpret_cast<float*>(ws + ex.m_off);
+    a.part_l = reinterpret_cast<float*>(ws + ex.l_off);
+    a.part_acc = reinterpret_cast<float*>(ws + ex.acc_off);
+    a.dev_err = r.dev_err;
+    a.num_seqs = B;
+    a.num_q_heads = r.num_q_heads;
+    a.num_kv_heads = r.num_kv_heads;
+    a.group = G;
+    a.num_blocks = r.num_blocks;
+    a.max_blocks_per_seq = r.max_blocks_per_seq;
+    a.max_partitions = ex.pmax;
+    a.scale_log2 = r.scale * 1.4426950408889634f;
+    pf.items = reinterpret_cast<const PrefillItem*>(ws + L.items_off);
+    pf.out_tokens = reinterpret_cast<const int32_t*>(ws + L.members_off);
+    void* args[] = {&tmk, &tmv, &tmq, &pf};
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(tc_items.size()));
+    cfg.blockDim = dim3(pinst.threads);
+    cfg.dynamicSmemBytes = pinst.smem;
+    cfg.stream = r.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelExC(&cfg, pinst.kernel, args);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "prefix launch: %s", cudaGetErrorString(err));
+    ex.after_prefix_kernel = true;
+  }
   if (!items.empty()) {
     st = prepare_kernel(pinst.kernel, pinst.smem);
     if (st != PA_OK) return st;
@@ -718,7 +856,7 @@ pa_status_t run_prefill(const DecodeReq& r, const int32_t* ctx_host, const int32
       for (int h = 0; h < r.num_kv_heads; ++h)
         for (int p = 0; p < nparts; ++p)
           items.push_back(PrefillItem{s, q_base + t, count, p0, p * pb, std::min(nblk, (p + 1) * pb),
-                                      kv_end, h, p, nparts == 1 ? 1 : 0, 0, 0});
+                                      kv_end, h, p, nparts == 1 ? 1 : 0, h * G, -1});
     }
     q_base += qlen;
   }
@@ -759,6 +897,7 @@ pa_status_t run_prefill(const DecodeReq& r, const int32_t* ctx_host, const int32
   a.max_partitions = L.pmax;
   a.scale_log2 = r.scale * 1.4426950408889634f;
   pf.items = reinterpret_cast<const PrefillItem*>(ws + L.items_off);
+  pf.out_tokens = nullptr;
   CUtensorMap tmq;
   void* args3[] = {&tmk, &tmv, &pf};
   void* args4[] = {&tmk, &tmv, &tmq, &pf};

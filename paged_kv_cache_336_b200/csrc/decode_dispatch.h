@@ -35,5 +35,7 @@ bool find_prefix_bf16(int head_dim, int block_size, PrefixInstance* out);
 // Paged prefill kernels (bf16); same shapes, same instance record. tcgen05:
 // the 128-row tensor-memory kernel; otherwise the 64-row mma.sync kernel.
 bool find_prefill_bf16(int head_dim, int block_size, bool tcgen05, PrefixInstance* out);
+// tcgen05 shared-prefix pass: the prefill kernel with one 128-row tile per CTA.
+bool find_tc_prefix_bf16(int head_dim, int block_size, PrefixInstance* out);
 
 }  // namespace pagedkv

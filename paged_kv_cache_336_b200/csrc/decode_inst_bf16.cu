@@ -82,9 +82,9 @@ static PrefixInstance make_prefill() {
 // faster than one tile per CTA at two CTAs per SM).
 constexpr int kTcPrefillTiles = 2;
 
-template <int BS, int D>
+template <int BS, int D, int TILES = kTcPrefillTiles>
 static PrefixInstance make_tc_prefill() {
-  using Cfg = TcCfg<BS, D, kTcPrefillTiles>;
+  using Cfg = TcCfg<BS, D, TILES>;
   PrefixInstance r;
   r.kernel = reinterpret_cast<const void*>(&tc_prefill_kernel<Cfg>);
   r.threads = Cfg::kThreads;
@@ -105,6 +105,14 @@ bool find_prefill_bf16(int head_dim, int block_size, bool tcgen05, PrefixInstanc
   if (block_size == 16 && head_dim == 128) { *out = pick_prefill<16, 128>(tcgen05); return true; }
   if (block_size == 32 && head_dim == 64) { *out = pick_prefill<32, 64>(tcgen05); return true; }
   if (block_size == 32 && head_dim == 128) { *out = pick_prefill<32, 128>(tcgen05); return true; }
+  return false;
+}
+
+bool find_tc_prefix_bf16(int head_dim, int block_size, PrefixInstance* out) {
+  if (block_size == 16 && head_dim == 64) { *out = make_tc_prefill<16, 64, 1>(); return true; }
+  if (block_size == 16 && head_dim == 128) { *out = make_tc_prefill<16, 128, 1>(); return true; }
+  if (block_size == 32 && head_dim == 64) { *out = make_tc_prefill<32, 64, 1>(); return true; }
+  if (block_size == 32 && head_dim == 128) { *out = make_tc_prefill<32, 128, 1>(); return true; }
   return false;
 }
 

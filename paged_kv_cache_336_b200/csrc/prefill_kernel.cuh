@@ -33,12 +33,14 @@ struct PrefillItem {
   int32_t kvh;
   int32_t part;         // partial slot (KV partition index)
   int32_t final_out;    // 1: the tile has a single partition, write outputs directly
-  int32_t pad0, pad1;
+  int32_t q_head0;      // tcgen05 kernel: first head of the Q box (kvh * group; 0 for packed Q)
+  int32_t out_begin;    // tcgen05 kernel: >= 0: output row j is out_tokens[out_begin + j]
 };
 
 struct PrefillArgs {
   DecodeArgs d;              // q, block tables, partials, out, sizes, scale, dev_err
   const PrefillItem* items;  // [gridDim.x]
+  const int32_t* out_tokens; // output token (or sequence) of each item row; see out_begin
 };
 
 template <class Cfg>

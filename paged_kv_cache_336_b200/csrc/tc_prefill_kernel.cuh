@@ -190,12 +190,15 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     };
     // Q of each tile first: rows past the query tokens of the array read as 0
     // (the box's out-of-range fill), rows past the item's tokens are masked.
+    // When Q was packed by a preceding kernel (launched as its programmatic
+    // dependent), wait for that grid here; K/V prefetch is not held back.
+    grid_dependency_wait();
     if (elect_one()) {
       for (int t = 0; t < ntiles; ++t) {
         mbar_arrive_expect_tx(&q_full[t], KCH * TQ * G * 128);
         for (int c = 0; c < KCH; ++c)
           tma_load_3d(qs + t * Cfg::kQBytes + c * (ROWS * 128), &tm_q, &q_full[t], c * 64,
-                      it.kvh * G, it.q_begin + t * TQ);
+                      it.q_head0, it.q_begin + t * TQ);
       }
     }
     __syncwarp();
@@ -442,7 +445,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_last[t], 0, a.dev_err));
       if (ok) {
         tmem_fence_after_sync();
-        const int64_t tok = it.q_begin + (valid ? jq : 0);
+        const int64_t tok = !valid ? it.q_begin
+                            : it.out_begin >= 0 ? pf.out_tokens[it.out_begin + jq] : it.q_begin + jq;
         const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
         const int64_t row = tok * a.num_q_heads + h;
         const float inv = l > 0.f ? 1.f / l : 0.f;

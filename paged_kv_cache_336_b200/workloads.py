@@ -138,7 +138,9 @@ def _prefix_common(name: str, prompt_len: int, tail_max: int, seed: int,
     ctx = np.full(nseq, prompt_len, dtype=np.int64)
     prompt_blocks = -(-prompt_len // bs)
     private = sum(-(-(prompt_len % bs + t + 1) // bs) + 1 for t in tails)
-    nb = int(math.ceil(1.1 * (prompts * prompt_blocks + private)))
+    # + 4 blocks (64 tokens) per sequence: room for the bench's cycled decode
+    # states and its end-to-end steps
+    nb = int(math.ceil(1.1 * (prompts * prompt_blocks + private))) + 4 * nseq
     return Workload(
         name=name, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=bs,
         dtype=BF16, num_blocks=nb,

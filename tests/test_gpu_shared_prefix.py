@@ -3,8 +3,10 @@
 Forked sequences share their prompt's blocks; the shared-prefix route reads
 them once per KV head for the whole group and must still return plain decode
 attention. Small cases are compared with the full float64 oracle (several
-groups, a group wider than one 64-row CTA, sequences in no group, block
+groups, a group wider than one CTA's rows, sequences in no group, block
 sizes 16 and 32); the full-size prefix-sharing workloads with sampled rows.
+Both prefix-pass kernels are covered: the mma.sync one (default, 64 query
+rows per CTA) and the tcgen05 one (PAGEDKV_PREFIX_KERNEL=tcgen05, 128).
 """
 
 import numpy as np
@@ -20,8 +22,18 @@ from gpu_util import (build_tables, check_close, device_tables, oracle_one, samp
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("G,bs,branches", [(1, 16, 5), (4, 16, 16), (8, 32, 12), (4, 32, 3)])
-def test_shared_prefix_small_matches_oracle(G, bs, branches):
+@pytest.fixture(params=["mma_sync", "tcgen05"])
+def kernel(request, monkeypatch):
+    if request.param == "tcgen05":
+        monkeypatch.setenv("PAGEDKV_PREFIX_KERNEL", "tcgen05")
+    else:
+        monkeypatch.delenv("PAGEDKV_PREFIX_KERNEL", raising=False)
+    return request.param
+
+
+@pytest.mark.parametrize("G,bs,branches", [(1, 16, 5), (4, 16, 16), (8, 32, 12), (4, 32, 3),
+                                           (16, 16, 20), (6, 32, 7)])
+def test_shared_prefix_small_matches_oracle(kernel, G, bs, branches):
     Hkv, D = 2, 128
     rng = np.random.default_rng(40 + G + bs)
     NB = 400
@@ -73,7 +85,7 @@ def test_shared_prefix_small_matches_oracle(G, bs, branches):
 
 
 @pytest.mark.parametrize("name", ["prefix", "prefix_cow"])
-def test_shared_prefix_full_size(name):
+def test_shared_prefix_full_size(kernel, name):
     w = workloads.WORKLOADS[name]()
     bm, k_pool, v_pool = setup(w)
     slots, pairs = bm.append_slots_arrays(w.step_seqs)
