@@ -40,6 +40,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -151,7 +152,10 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.device_index = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        # raw samples go to PAGEDKV_CLOCKS_DIR (default: the system temp dir);
+        # the JSON line carries their summary
+        out_dir = os.environ.get("PAGEDKV_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"clocks_rank{device_index}.csv")
 
     def start(self):
         try:
