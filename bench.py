@@ -695,10 +695,32 @@ def run_swap_bench(args, device_index):
         ms = t0.elapsed_time(t1) / reps
         nbytes = 2 * nslots * block_bytes
         res[name] = {"GB/s": round(nbytes / (ms * 1e-3) / 1e9, 2), "ms": round(ms, 4), "bytes": nbytes}
+    # Roofline: the host link, measured as plain contiguous pinned-memory copies
+    # of the same byte count (copy engine, one direction at a time).
+    dev_buf = torch.empty(2 * host_k.numel(), dtype=host_k.dtype, device=device)
+    host_buf = torch.empty(2 * host_k.numel(), dtype=host_k.dtype).pin_memory()
+    link = {}
+    for name, dst, src in (("d2h", host_buf, dev_buf), ("h2d", dev_buf, host_buf)):
+        for _ in range(3):
+            dst.copy_(src, non_blocking=True)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(10):
+            dst.copy_(src, non_blocking=True)
+        t1.record()
+        torch.cuda.synchronize()
+        link[name] = dev_buf.numel() * dev_buf.element_size() / (t0.elapsed_time(t1) / 10 * 1e-3) / 1e9
+    res["swap_out"]["frac_of_measured_d2h"] = round(res["swap_out"]["GB/s"] / link["d2h"], 4)
+    res["swap_in"]["frac_of_measured_h2d"] = round(res["swap_in"]["GB/s"] / link["h2d"], 4)
     return {"metric": "swap of whole KV blocks between HBM and pinned host memory (K and V)",
             "unit": "GB/s", "value": res["swap_out"]["GB/s"], "impl": "ours",
             "config": {"workload": workload_label(w), "blocks": nslots,
-                       "block_bytes_each_pool": block_bytes}, **res}
+                       "block_bytes_each_pool": block_bytes},
+            "roofline": {"bound": "host link", "unit": "GB/s",
+                         "measured_d2h": round(link["d2h"], 2), "measured_h2d": round(link["h2d"], 2),
+                         "peak_kind": "measured: contiguous pinned-memory copies of the same bytes"},
+            **res}
 
 
 def main(argv=None):
