@@ -245,12 +245,16 @@ pa_status_t pa_decode_split_window(const void* q, const void* k_pool, const void
  * allocates enough blocks for the input).
  *
  * context_lens and query_lens are HOST arrays here (the host plans the
- * tiles); block tables are device memory. bf16 only. Tiles of 64 query rows
- * (query tokens x heads of one KV head) each read their KV once per
- * partition of partition_tokens tokens; tiles spanning several partitions
- * are joined by the log-sum-exp merge. workspace: at least
- * pa_prefill_workspace_size(...) bytes, 256-byte aligned, initialised once
- * with pa_decode_split_workspace_init.
+ * tiles); block tables are device memory. bf16, head_dim 64 or 128, block
+ * size 16 or 32. Each CTA takes two tiles of 128 query rows (query tokens x
+ * heads of one KV head; tcgen05 tensor cores, accumulators in tensor
+ * memory; PAGEDKV_PREFILL_KERNEL=mma_sync selects 64-row mma.sync tiles)
+ * and reads their KV once per partition of partition_tokens tokens; tiles
+ * spanning several partitions are joined by the log-sum-exp merge. q and
+ * out must be 16-byte aligned; with total_q = 0 they may be NULL and the
+ * call enqueues nothing. workspace: at least pa_prefill_workspace_size(...)
+ * bytes, 256-byte aligned, initialised once with
+ * pa_decode_split_workspace_init.
  * ------------------------------------------------------------------------- */
 size_t pa_prefill_workspace_size(int num_seqs, int total_q, int num_q_heads, int num_kv_heads,
                                  int head_dim, int block_size, int max_blocks_per_seq,

@@ -795,8 +795,15 @@ PrefillLayout prefill_layout(int num_seqs, int total_q, int num_q_heads, int num
   return L;
 }
 
-pa_status_t run_prefill(const DecodeReq& r, const int32_t* ctx_host, const int32_t* qlen_host,
+pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const int32_t* qlen_host,
                         int total_q, int partition_tokens, void* workspace, size_t workspace_bytes) {
+  // With no new tokens q and out are never touched and may be NULL; every
+  // other argument is still checked.
+  DecodeReq r = r_in;
+  if (total_q == 0) {
+    if (r.q == nullptr) r.q = r.k_pool;
+    if (r.out == nullptr) r.out = const_cast<void*>(r.k_pool);  // never written
+  }
   DecodeInstance inst;
   pa_status_t st = validate_and_pick(r, &inst);  // shapes, alignment, dtype, group (merge kernel)
   if (st != PA_OK) return st;

@@ -163,3 +163,32 @@ def test_prefill_rejects_bad_lengths():
         binding.prefill(q, k, k, bt, [10, 3], [2, 4], 0.1)        # query_len > context_len
     with pytest.raises(binding.InvalidArgumentError):
         binding.prefill(q, k, k, bt, [10, 30], [2, 2], 0.1)       # sum of query_lens != 5
+
+
+def test_prefill_with_empty_sequences(kernel):
+    """Sequences with earlier context but no new tokens (query_len 0) sit in
+    the batch beside ordinary ones; a batch with no new tokens at all
+    returns at once."""
+    G, bs, D = 4, 16, 128
+    plan = [(90, 0), (200, 33), (0, 0), (47, 47), (130, 0)]
+    ctx = np.array([c for c, _ in plan], dtype=np.int64)
+    qlen = np.array([n for _, n in plan], dtype=np.int32)
+    w = workloads.random_small(95, num_seqs=len(plan), num_q_heads=2 * G, num_kv_heads=2,
+                               head_dim=D, block_size=bs, dtype=workloads.BF16,
+                               max_ctx=int(ctx.max()), fixed_lens=ctx.tolist())
+    bm, k_pool, v_pool = setup(w)
+    bt, _, tables, ctx_np = device_tables(bm, list(range(len(plan))))
+    total = int(qlen.sum())
+    q = workloads.draw_normal((total, 2 * G, D), workloads.BF16, 96, "cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = binding.prefill(q, k_pool, v_pool, bt, ctx_np, qlen, w.scale, partition_tokens=64,
+                          dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    want = oracle.paged_prefill(to_f64(q), to_f64(k_pool), to_f64(v_pool), tables, ctx_np, qlen,
+                                w.scale)
+    check_close(to_f64(out), want, workloads.BF16, f"empty sequences[{kernel}]")
+    q0 = torch.empty((0, 2 * G, D), dtype=torch.bfloat16, device="cuda")
+    out0 = binding.prefill(q0, k_pool, v_pool, bt, ctx_np, np.zeros(len(plan), np.int32), w.scale,
+                           partition_tokens=64)
+    assert out0.shape == (0, 2 * G, D)
