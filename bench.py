@@ -476,8 +476,10 @@ def run_e2e(args, ds, rank, world, device):
                            partition_tokens=ds.partition_tokens)
 
     def timed(pipelined: bool):
-        h2d = d2h = 0
-        total = 0
+        # bookkeeping stays out of the timed loop: every step appends one token
+        # to each sequence, so step i decodes lengths ctx0 + i + 1
+        ctx0 = np.array([ds.bm.context_len(int(x)) for x in seqs], dtype=np.int64)
+        ncows = []
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -485,14 +487,15 @@ def run_e2e(args, ds, rank, world, device):
         for i in range(steps):
             j = i % ring
             st = piped[i % 2] if pipelined else sync
-            ncow = st.step(seqs, hq[j], hk[j], hv[j], hout[i % 2], synchronize=not pipelined,
-                           stream=stream)
-            h2d += st.h2d_bytes(n, ncow)
-            d2h += st.d2h_bytes(n)
-            ctx = st.h_ctx[:n].numpy().astype(np.int64)
-            total += decode_bytes(w, ctx) + append_bytes(w, n) + copy_bytes(w, ncow)
+            ncows.append(st.step(seqs, hq[j], hk[j], hv[j], hout[i % 2],
+                                 synchronize=not pipelined, stream=stream))
         torch.cuda.synchronize()
         elapsed = time.perf_counter() - t_start
+        assert np.array_equal(np.array([ds.bm.context_len(int(x)) for x in seqs]), ctx0 + steps)
+        total = sum(decode_bytes(w, ctx0 + i + 1) + append_bytes(w, n) + copy_bytes(w, c)
+                    for i, c in enumerate(ncows))
+        h2d = sum(sync.h2d_bytes(n, c) for c in ncows)
+        d2h = steps * sync.d2h_bytes(n)
         elapsed, total, _ = reduce_over_ranks(elapsed, total, steps * n, device)
         return total / elapsed / 1e9, elapsed / steps * 1e3, h2d / steps, d2h / steps
 
