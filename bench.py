@@ -447,7 +447,7 @@ def run_e2e(args, ds, rank, world, device):
     """Same metric through the public API from pinned host buffers: one
     pa_decode_step call per step (host block-manager step, H2D of the step's
     inputs, copies + append + split decode, D2H of out). Measured two ways:
-    pipelined (two staging sets alternated, uploads on a copy stream, no
+    pipelined (two staging sets alternated, uploads and downloads on their own streams, no
     per-step host synchronisation; the value reported) and one step at a
     time with a stream synchronisation after each (reported beside it)."""
     import torch
@@ -469,8 +469,10 @@ def run_e2e(args, ds, rank, world, device):
     hout = [torch.empty(hq[0].shape, dtype=hq[0].dtype).pin_memory() for _ in range(2)]
     stream = torch.cuda.current_stream()
     copy_stream = torch.cuda.Stream()
+    download_stream = torch.cuda.Stream()
     piped = [b.DecodeStepper(ds.bm, ds.k_pool, ds.v_pool, w.num_q_heads, w.scale, max_seqs=n,
-                             partition_tokens=ds.partition_tokens, copy_stream=copy_stream)
+                             partition_tokens=ds.partition_tokens, copy_stream=copy_stream,
+                             download_stream=download_stream)
              for _ in range(2)]
     sync = b.DecodeStepper(ds.bm, ds.k_pool, ds.v_pool, w.num_q_heads, w.scale, max_seqs=n,
                            partition_tokens=ds.partition_tokens)
@@ -506,8 +508,8 @@ def run_e2e(args, ds, rank, world, device):
             "steps": steps, "ms_per_step": round(ms, 4),
             "path": "pa_decode_step (C ABI) per step: host block manager step + pinned H2D "
                     "of the step's inputs + copies/append/split decode + D2H out; two staging "
-                    "sets alternated, uploads on a copy stream overlapping the previous step's "
-                    "kernels, one synchronisation at the end",
+                    "sets alternated, uploads and downloads on their own streams overlapping the "
+                    "neighbouring steps' kernels, one synchronisation at the end",
             "one_step_at_a_time": {"value": round(g_sync, 2), "unit": "GB/s",
                                    "ms_per_step": round(ms_sync, 4),
                                    "path": "the same call with a stream synchronisation after "

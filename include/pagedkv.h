@@ -450,17 +450,27 @@ pa_status_t pa_bm_stats(pa_bm_t bm, pa_bm_stats_t* stats);
  * returns before anything is enqueued, state unchanged. A CUDA error after
  * the manager step leaves the manager with the step applied.
  *
- * Pipelining (optional): with the three fields at the end of the struct set
- * (pa_step_pipeline_create), the uploads run on `copy_stream`: they wait
- * for `compute_done` (this set's previous step, decode and download, is
- * finished with the device staging) and the kernels on `stream` wait for
- * `upload_done`. The host staging of a set is rewritten only after that
- * set's previous uploads completed (the call first waits on `upload_done`).
- * A caller that alternates two buffer sets with synchronize = 0 overlaps a
- * step's uploads and host work with the previous step's kernels. It keeps
+ * Packed staging (optional): when the four small arrays are laid out back
+ * to back on both sides, in the order slots [max_seqs] | pairs
+ * [max_seqs][2] | context_lens [max_seqs] | tables [max_seqs][...], one
+ * upload carries them (max_seqs * 28 + n * max_blocks_per_seq * 4 bytes);
+ * pa_decode_step_h2d_bytes counts that copy.
+ *
+ * Pipelining (optional): with the fields at the end of the struct set
+ * (pa_step_pipeline_create), the uploads run on `copy_stream` and the
+ * download on `download_stream`:
+ *   uploads   wait for download_done (this set's previous step has finished
+ *             with its device staging), then record upload_done;
+ *   kernels   on `stream` wait for upload_done, then record compute_done;
+ *   download  waits for compute_done, then records download_done.
+ * The host staging of a set is rewritten only after that set's previous
+ * uploads completed (the call first waits on upload_done). A caller that
+ * alternates two buffer sets with synchronize = 0 overlaps a step's uploads,
+ * download and host work with the kernels of its neighbours. It keeps
  * q_host, k_new_host and v_new_host unchanged until the step's uploads are
- * done, and reads out_host after synchronising `stream`. Pool updates stay
- * ordered on `stream`. With the fields NULL everything runs on `stream`.
+ * done, and reads out_host after synchronising `download_stream`. Pool
+ * updates stay ordered on `stream`. With the fields NULL everything runs on
+ * `stream`.
  * ========================================================================= */
 typedef struct {
   /* shape and cache */
@@ -489,14 +499,17 @@ typedef struct {
   /* pipelining (optional, NULL = off; see above) */
   void* upload_done;        /* cudaEvent_t recorded on copy_stream after the uploads */
   void* compute_done;       /* cudaEvent_t recorded on `stream` after the decode */
-  void* copy_stream;        /* cudaStream_t for the uploads and the download */
+  void* copy_stream;        /* cudaStream_t for the uploads */
+  void* download_done;      /* cudaEvent_t recorded on download_stream after the download */
+  void* download_stream;    /* cudaStream_t for the download */
 } pa_step_buffers_t;
 
-/* Creates the two events of a buffer set's pipelining fields (timing
- * disabled) and stores copy_stream; the caller owns the stream.
- * pa_step_pipeline_destroy destroys the events and clears the three fields.
+/* Creates the three events of a buffer set's pipelining fields (timing
+ * disabled) and stores the two streams; the caller owns the streams.
+ * pa_step_pipeline_destroy destroys the events and clears the fields.
  * Setup-time calls, not for the hot path. */
-pa_status_t pa_step_pipeline_create(pa_step_buffers_t* buf, void* copy_stream);
+pa_status_t pa_step_pipeline_create(pa_step_buffers_t* buf, void* copy_stream,
+                                    void* download_stream);
 pa_status_t pa_step_pipeline_destroy(pa_step_buffers_t* buf);
 
 /* Number of host->device and device->host bytes one pa_decode_step call of

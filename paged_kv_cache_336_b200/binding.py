@@ -76,6 +76,7 @@ class StepBuffers(ctypes.Structure):
         ("d_slots", _P), ("d_pairs", _P), ("d_tables", _P), ("d_context_lens", _P),
         ("h_slots", _P), ("h_pairs", _P), ("h_tables", _P), ("h_context_lens", _P),
         ("upload_done", _P), ("compute_done", _P), ("copy_stream", _P),
+        ("download_done", _P), ("download_stream", _P),
     ]
 
 # name -> (restype, argtypes); mirrors include/pagedkv.h
@@ -125,7 +126,7 @@ _SIGNATURES = {
     "pa_decode_step_d2h_bytes": (_SZ, [ctypes.POINTER(StepBuffers), _I]),
     "pa_decode_step": (_I, [_P, ctypes.POINTER(StepBuffers), _P, _I, _P, _P, _P, _P,
                             ctypes.POINTER(_I), _I, _P, _P]),
-    "pa_step_pipeline_create": (_I, [ctypes.POINTER(StepBuffers), _P]),
+    "pa_step_pipeline_create": (_I, [ctypes.POINTER(StepBuffers), _P, _P]),
     "pa_step_pipeline_destroy": (_I, [ctypes.POINTER(StepBuffers)]),
 }
 
@@ -599,9 +600,11 @@ class DecodeStepper:
     decode, download (and, by default, stream synchronisation)."""
 
     def __init__(self, bm: "BlockManager", k_pool, v_pool, num_q_heads: int, scale: float,
-                 max_seqs: int, partition_tokens: int = 512, copy_stream=None):
+                 max_seqs: int, partition_tokens: int = 512, copy_stream=None,
+                 download_stream=None):
         """copy_stream: a torch.cuda.Stream for the uploads (pipelined steps,
-        see pa_step_pipeline_create); None runs everything on the step's stream."""
+        see pa_step_pipeline_create), download_stream one for the download
+        (made here when not given); None runs everything on the step's stream."""
         torch = _torch()
         _require_cuda(k_pool, v_pool)
         NB, Hkv, BS, D = k_pool.shape
@@ -615,14 +618,19 @@ class DecodeStepper:
         self.d_out = torch.empty_like(self.d_q)
         self.d_k_new = torch.empty(max_seqs, Hkv, D, dtype=self.dtype, device=dev)
         self.d_v_new = torch.empty_like(self.d_k_new)
-        self.d_slots = torch.empty(max_seqs, dtype=torch.int64, device=dev)
-        self.d_pairs = torch.empty(max_seqs, 2, dtype=torch.int64, device=dev)
-        self.d_tables = torch.empty(max_seqs, mbs, dtype=torch.int32, device=dev)
-        self.d_ctx = torch.empty(max_seqs, dtype=torch.int32, device=dev)
-        self.h_slots = torch.empty(max_seqs, dtype=torch.int64).pin_memory()
-        self.h_pairs = torch.empty(max_seqs, 2, dtype=torch.int64).pin_memory()
-        self.h_tables = torch.empty(max_seqs, mbs, dtype=torch.int32).pin_memory()
-        self.h_ctx = torch.empty(max_seqs, dtype=torch.int32).pin_memory()
+        # the four small staging arrays back to back (slots | pairs | lengths |
+        # tables) on both sides, so one upload carries them
+        nbytes = max_seqs * (8 + 16 + 4) + max_seqs * mbs * 4
+        self.d_pack = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.h_pack = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+
+        def views(buf):
+            o1, o2, o3 = max_seqs * 8, max_seqs * 24, max_seqs * 28
+            return (buf[:o1].view(torch.int64), buf[o1:o2].view(torch.int64).view(max_seqs, 2),
+                    buf[o2:o3].view(torch.int32), buf[o3:].view(torch.int32).view(max_seqs, mbs))
+
+        self.d_slots, self.d_pairs, self.d_ctx, self.d_tables = views(self.d_pack)
+        self.h_slots, self.h_pairs, self.h_ctx, self.h_tables = views(self.h_pack)
         b = StepBuffers()
         b.max_seqs, b.num_q_heads, b.num_kv_heads, b.head_dim = max_seqs, num_q_heads, Hkv, D
         b.block_size, b.num_blocks, b.max_blocks_per_seq = BS, NB, mbs
@@ -638,8 +646,10 @@ class DecodeStepper:
         self.buffers = b
         self.copy_stream = copy_stream
         if copy_stream is not None:
+            self.download_stream = download_stream or torch.cuda.Stream(device=dev)
             _check(library().pa_step_pipeline_create(ctypes.byref(self.buffers),
-                                                     _stream_ptr(copy_stream)))
+                                                     _stream_ptr(copy_stream),
+                                                     _stream_ptr(self.download_stream)))
 
     def __del__(self):
         try:

@@ -262,6 +262,34 @@ pa_status_t device_info(DeviceInfo* info) {
   return PA_OK;
 }
 
+// Resident CTAs per SM of `kernel` at `threads` x `smem`, queried once per
+// (device, kernel, threads, smem): the query costs microseconds of host time
+// per call otherwise.
+pa_status_t occupancy(const void* kernel, int threads, int smem, int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice failed");
+  struct Entry {
+    int dev;
+    const void* k;
+    int threads, smem, occ;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& e : cache) {
+    if (e.dev == dev && e.k == kernel && e.threads == threads && e.smem == smem) {
+      *out = e.occ;
+      return PA_OK;
+    }
+  }
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem) != cudaSuccess || occ <= 0)
+    return fail(PA_ERR_CUDA, "occupancy query failed (smem %d)", smem);
+  cache.push_back(Entry{dev, kernel, threads, smem, occ});
+  *out = occ;
+  return PA_OK;
+}
+
 // Raises the kernel's dynamic shared memory limit when needed (per device).
 pa_status_t prepare_kernel(const void* kernel, int smem) {
   static std::mutex mu;
@@ -390,9 +418,8 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
     st = device_info(&dinfo);
     if (st != PA_OK) return st;
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, inst.kernel, inst.threads, smem) != cudaSuccess ||
-        occ <= 0)
-      return fail(PA_ERR_CUDA, "occupancy query failed for %s (smem %d)", inst.name, smem);
+    st = occupancy(inst.kernel, inst.threads, smem, &occ);
+    if (st != PA_OK) return st;
     const int64_t max_items = static_cast<int64_t>(r.num_seqs) * r.num_kv_heads * L.pmax;
     const int64_t ctas = std::min<int64_t>(max_items, static_cast<int64_t>(dinfo.sms) * occ);
     grid = dim3(static_cast<unsigned>(ctas > 0 ? ctas : 1));

@@ -270,7 +270,7 @@ def test_decode_step_rejects_before_touching_the_device():
     assert lib.pa_decode_step(bm2._h, ctypes.byref(b), ids.ctypes.data, 1, *args) == \
         binding.PA_ERR_NO_FREE_BLOCKS
     assert bm2.context_len(7) == 8 and bm2.free_queue_list() == []
-    assert ctypes.sizeof(binding.StepBuffers) == 192
+    assert ctypes.sizeof(binding.StepBuffers) == 208
     # a copy stream without its events is rejected before the manager step
     b.copy_stream = FAKE
     assert lib.pa_decode_step(bm2._h, ctypes.byref(b), ids.ctypes.data, 1, *args) == \
