@@ -25,9 +25,9 @@ Policy choices the pages leave open (each is the plainest reading):
 * Free blocks form a FIFO queue, seeded from ``initial_free_order``
   (identity when omitted). Allocation pops from the front; a ``free`` call
   pushes the blocks it reclaims to the back in ascending block-ID order.
-* A copy-on-write copies the whole block (all heads, all slots); the pages
-  say both "valid entries" and "the contents of the shared block", and the
-  whole block is a superset of the valid entries.
+* A copy-on-write copies the whole block (all heads, all slots). One page
+  says the copy covers the block's valid entries, another that it covers the
+  shared block's contents; the whole block covers both.
 * ``append_slots`` processes sequences in the order given. A shared partial
   tail is copied by each writer while its count is above one; the last
   holder (count one) writes in place.
