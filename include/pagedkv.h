@@ -250,7 +250,11 @@ pa_status_t pa_decode_split_window(const void* q, const void* k_pool, const void
  * heads of one KV head; tcgen05 tensor cores, accumulators in tensor
  * memory; PAGEDKV_PREFILL_KERNEL=mma_sync selects 64-row mma.sync tiles)
  * and reads their KV once per partition of partition_tokens tokens; tiles
- * spanning several partitions are joined by the log-sum-exp merge. q and
+ * spanning several partitions are joined by the log-sum-exp merge. With
+ * more (tile pair, partition) items than resident CTAs the tcgen05 kernel
+ * runs persistently: the host hands each item to the CTA with the least
+ * estimated work so far, and a CTA loads its next item's Q and K/V while it
+ * finishes the current one (PAGEDKV_PREFILL_CTAS=n caps that grid). q and
  * out must be 16-byte aligned; with total_q = 0 they may be NULL and the
  * call enqueues nothing. workspace: at least pa_prefill_workspace_size(...)
  * bytes, 256-byte aligned, initialised once with

@@ -9,7 +9,10 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <queue>
+#include <utility>
 #include <vector>
 
 #include "decode_dispatch.h"
@@ -795,10 +798,11 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
 
 // ---- paged prefill -------------------------------------------------------------------
 // Workspace: [0,256) header | merge_lens int32 [total_q] | items PrefillItem
-// [max_items] | m, l float [total_q][Hq][pmax] | acc float [...][head_dim],
+// [max_items] | schedule offsets int32 [max_items + 1] | m, l float
+// [total_q][Hq][pmax] | acc float [...][head_dim],
 // pmax = ceil(max_blocks_per_seq / partition blocks).
 struct PrefillLayout {
-  size_t lens_off, items_off, m_off, l_off, acc_off, total, max_items;
+  size_t lens_off, items_off, sched_off, m_off, l_off, acc_off, total, max_items;
   int pmax;
 };
 
@@ -815,7 +819,8 @@ PrefillLayout prefill_layout(int num_seqs, int total_q, int num_q_heads, int num
   L.lens_off = kWorkspaceHeader;
   L.items_off = L.lens_off + align256(static_cast<size_t>(total_q) * 4);
   const size_t rows = static_cast<size_t>(total_q) * num_q_heads * L.pmax;
-  L.m_off = L.items_off + align256(L.max_items * sizeof(PrefillItem));
+  L.sched_off = L.items_off + align256(L.max_items * sizeof(PrefillItem));
+  L.m_off = L.sched_off + align256((L.max_items + 1) * 4);
   L.l_off = L.m_off + align256(rows * 4);
   L.acc_off = L.l_off + align256(rows * 4);
   L.total = L.acc_off + align256(rows * static_cast<size_t>(head_dim) * 4);
@@ -877,9 +882,11 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
   items.clear();
   bool any_split = false;
   int q_base = 0;
+  // Items in sequence order, each sequence's query tiles last-first (the
+  // longest spans first), so that the work handed out last is short.
   for (int s = 0; s < B; ++s) {
     const int qlen = qlen_host[s], ctx = ctx_host[s];
-    for (int t = 0; t < qlen; t += tq) {
+    for (int t = qlen > 0 ? (qlen - 1) / tq * tq : -1; t >= 0; t -= tq) {
       const int count = std::min(tq, qlen - t);
       const int p0 = ctx - qlen + t;
       const int kv_end = p0 + count;  // last position + 1
@@ -895,16 +902,70 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
     q_base += qlen;
   }
   if (items.size() > L.max_items) return fail(PA_ERR_INVALID_ARG, "too many prefill items");
+  st = prepare_kernel(pinst.kernel, pinst.smem);
+  if (st != PA_OK) return st;
+
+  // The tcgen05 kernel runs persistently when there are more items than
+  // resident CTAs: each item goes, in list order, to the CTA with the least
+  // estimated work so far (cost ~ KV chunks x active tiles, plus a constant
+  // per item), and each CTA's items are stored together. A CTA starts the
+  // next item's loads while it finishes the current one.
+  thread_local std::vector<PrefillItem> sched_items;
+  thread_local std::vector<int32_t> sched_offs, owner;
+  unsigned grid = static_cast<unsigned>(items.size());
+  const PrefillItem* upload_items = items.data();
+  bool persistent = false;
+  if (pinst.q_map) {
+    DeviceInfo di;
+    int occ = 0;
+    if ((st = device_info(&di)) != PA_OK) return st;
+    if ((st = occupancy(pinst.kernel, pinst.threads, pinst.smem, &occ)) != PA_OK) return st;
+    size_t ctas = static_cast<size_t>(di.sms) * occ;
+    // PAGEDKV_PREFILL_CTAS=n caps the persistent grid (tests use it to give
+    // every CTA many items at small sizes).
+    if (const char* cap = std::getenv("PAGEDKV_PREFILL_CTAS")) {
+      const long n = std::strtol(cap, nullptr, 10);
+      if (n > 0) ctas = std::min(ctas, static_cast<size_t>(n));
+    }
+    if (items.size() > ctas) {
+      persistent = true;
+      grid = static_cast<unsigned>(ctas);
+      const int tile_tokens = std::max(1, pinst.rows / G);
+      using Load = std::pair<int64_t, int32_t>;
+      std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+      for (unsigned b = 0; b < grid; ++b) heap.push(Load{0, static_cast<int32_t>(b)});
+      owner.resize(items.size());
+      sched_offs.assign(grid + 1, 0);
+      for (size_t i = 0; i < items.size(); ++i) {
+        const PrefillItem& it = items[i];
+        const int64_t span = std::max(0, std::min(it.block_end * r.block_size, it.kv_end) -
+                                             it.block_begin * r.block_size);
+        const int64_t cost = span * (it.q_count > tile_tokens ? 21 : 15) / 64 + 20;
+        Load ld = heap.top();
+        heap.pop();
+        owner[i] = ld.second;
+        ++sched_offs[ld.second + 1];
+        heap.push(Load{ld.first + cost, ld.second});
+      }
+      for (unsigned b = 0; b < grid; ++b) sched_offs[b + 1] += sched_offs[b];
+      sched_items.resize(items.size());
+      thread_local std::vector<int32_t> fill;
+      fill.assign(sched_offs.begin(), sched_offs.end() - 1);
+      for (size_t i = 0; i < items.size(); ++i) sched_items[fill[owner[i]]++] = items[i];
+      upload_items = sched_items.data();
+    }
+  }
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaError_t err;
   if ((err = cudaMemcpyAsync(ws + L.lens_off, lens.data(), lens.size() * 4, cudaMemcpyHostToDevice,
                              r.stream)) != cudaSuccess ||
-      (err = cudaMemcpyAsync(ws + L.items_off, items.data(), items.size() * sizeof(PrefillItem),
-                             cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
+      (err = cudaMemcpyAsync(ws + L.items_off, upload_items, items.size() * sizeof(PrefillItem),
+                             cudaMemcpyHostToDevice, r.stream)) != cudaSuccess ||
+      (persistent &&
+       (err = cudaMemcpyAsync(ws + L.sched_off, sched_offs.data(), sched_offs.size() * 4,
+                              cudaMemcpyHostToDevice, r.stream)) != cudaSuccess))
     return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
-  st = prepare_kernel(pinst.kernel, pinst.smem);
-  if (st != PA_OK) return st;
   const int rows = r.num_blocks * r.num_kv_heads * r.block_size;
   CUtensorMap tmk, tmv;
   st = pool_tensor_map(r.k_pool, rows, r.head_dim, r.block_size, r.dtype, &tmk);
@@ -932,6 +993,7 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
   a.scale_log2 = r.scale * 1.4426950408889634f;
   pf.items = reinterpret_cast<const PrefillItem*>(ws + L.items_off);
   pf.out_tokens = nullptr;
+  pf.sched_off = persistent ? reinterpret_cast<const int32_t*>(ws + L.sched_off) : nullptr;
   CUtensorMap tmq;
   void* args3[] = {&tmk, &tmv, &pf};
   void* args4[] = {&tmk, &tmv, &tmq, &pf};
@@ -939,8 +1001,8 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
     st = q_tensor_map(r.q, total_q, r.num_q_heads, r.head_dim, G, std::max(1, pinst.rows / G), &tmq);
     if (st != PA_OK) return st;
   }
-  err = cudaLaunchKernel(pinst.kernel, dim3(static_cast<unsigned>(items.size())), dim3(pinst.threads),
-                         pinst.q_map ? args4 : args3, pinst.smem, r.stream);
+  err = cudaLaunchKernel(pinst.kernel, dim3(grid), dim3(pinst.threads), pinst.q_map ? args4 : args3,
+                         pinst.smem, r.stream);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(err));
   if (any_split) {
     int bs = r.block_size;

@@ -39,8 +39,11 @@ struct PrefillItem {
 
 struct PrefillArgs {
   DecodeArgs d;              // q, block tables, partials, out, sizes, scale, dev_err
-  const PrefillItem* items;  // [gridDim.x]
+  const PrefillItem* items;  // [gridDim.x], or [sched_off[gridDim.x]] with a schedule
   const int32_t* out_tokens; // output token (or sequence) of each item row; see out_begin
+  // tcgen05 kernel: NULL, one item per CTA (item blockIdx.x); else CTA b runs
+  // items [sched_off[b], sched_off[b + 1]) in order (a persistent launch).
+  const int32_t* sched_off;
 };
 
 template <class Cfg>

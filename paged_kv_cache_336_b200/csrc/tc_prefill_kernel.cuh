@@ -6,22 +6,26 @@
 // KV tile, so the products are a dense contraction; here they run as
 // 128-row tcgen05 MMAs with fp32 accumulators in tensor memory.
 //
-// One CTA = two tiles of 128 query rows (query tokens x the KV head's group
+// An item = two tiles of 128 query rows (query tokens x the KV head's group
 // heads) of one sequence, one KV head, one KV partition. Both tiles share
 // every K/V chunk, so the tensor core has one tile's work while the other
-// tile's softmax runs:
-//   warp 8 (producer): loads each tile's Q (one 3-D TMA box per 64 columns:
-//     tokens x group heads x 64, landing as 128-byte swizzled rows in
-//     token-major, head-minor order), then streams K_j then V_j of each
-//     64-token chunk (four
+// tile's softmax runs. A CTA runs one item, or (persistent launch) a list of
+// items back to back: the ring, the S buffers and every barrier carry on
+// across items, so the next item's loads and first S overlap the end of the
+// current one and its epilogue.
+//   warp 8 (producer): streams K_j then V_j of each 64-token chunk (four
 //     16-token TMA units, 128-byte swizzle: a chunk is one K-major operand
 //     for S and one MN-major operand for P V) into a ring of slots, and
 //     clears the V rows past the span in the last chunk.
-//   warps 9 / 10 (MMA issuers of tile 0 / 1), per chunk j:
+//   warps 9 / 10 (MMA issuers of tile 0 / 1) load the tile's Q (one 3-D TMA
+//     box per 64 columns: tokens x group heads x 64, landing as 128-byte
+//     swizzled rows in token-major, head-minor order; the next item's as
+//     soon as the current item's last S is done), and per chunk j issue:
 //       S_t(j+1) = Q_t K_{j+1}^T     (M=128, N=64, K=head_dim)
 //       O_t += P_t(j) V_j            (M=128, N=head_dim, K=64, P read from TMEM)
-//     The only MMA completion an issuer waits for is the P V of two chunks
-//     back, before S overwrites the buffer holding that P.
+//     The MMA completions an issuer waits for: the P V of two chunks back,
+//     before S overwrites the buffer holding that P; the item's last S,
+//     before the next Q overwrites this one.
 //   warps 0-3 / 4-7 (softmax of tile 0 / 1): thread r owns row r (TMEM lane
 //     r). It reads its 64 logits, masks causally where the chunk reaches
 //     past the row's position, and keeps a reference max m: P = 2^(x - m)
@@ -37,8 +41,9 @@
 // operands at about 128 bytes per clock per SM, so P stays out of shared
 // memory: per chunk the MMAs read Q and K (S) and V (P V) only. Every
 // hand-over is an mbarrier (TMA byte counts, tcgen05.commit, warp arrivals)
-// with one barrier per buffer, so no waiter can be lapped by two phases;
-// every wait is bounded.
+// with one barrier per buffer, so no waiter can be lapped by two phases (the
+// producer clears a partial chunk's V only after both issuers are past the
+// previous clear); every wait is bounded.
 #pragma once
 
 #include "prefill_kernel.cuh"
@@ -104,6 +109,28 @@ struct TcCfg {
   static_assert(TILES == 1 || TILES == 2, "tiles");
 };
 
+// One work item as every role of the CTA sees it.
+struct TcItem {
+  PrefillItem it;
+  int ntiles;    // tiles holding query rows (1 or 2)
+  int span0;     // first KV token of the partition
+  int span_end;  // KV tokens [span0, span_end) are streamed
+  int nchunks;   // CHUNK-token steps over the span
+  int vt_last;   // valid rows of the last chunk
+};
+
+template <class Cfg>
+__device__ __forceinline__ TcItem tc_item(const PrefillArgs& pf, int idx, int tq) {
+  TcItem x;
+  x.it = pf.items[idx];
+  x.ntiles = (Cfg::TILES == 2 && x.it.q_count > tq) ? 2 : 1;
+  x.span0 = x.it.block_begin * Cfg::BS;
+  x.span_end = min(x.it.block_end * Cfg::BS, x.it.kv_end);
+  x.nchunks = x.span_end > x.span0 ? (x.span_end - x.span0 + Cfg::CHUNK - 1) / Cfg::CHUNK : 0;
+  x.vt_last = x.nchunks > 0 ? x.span_end - (x.span0 + (x.nchunks - 1) * Cfg::CHUNK) : Cfg::CHUNK;
+  return x;
+}
+
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -126,34 +153,33 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
   uint8_t* slots = qs + Cfg::TILES * Cfg::kQBytes;       // [NSLOT][KCH][CHUNK][128 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(slots + NSLOT * Cfg::kSlotBytes);
   uint64_t* kv_full = bars;               // [NSLOT] TMA bytes landed
-  uint64_t* kv_empty = bars + NSLOT;      // [NSLOT] last MMA reading the slot done (commit)
+  uint64_t* kv_empty = bars + NSLOT;      // [NSLOT] both tiles done with the slot
   uint64_t* s_full = bars + 2 * NSLOT;    // [tile][buffer] S MMA done (commit)
   uint64_t* p_full = s_full + 4;          // [tile][buffer] P written (4 warp arrivals)
   uint64_t* p_free = p_full + 4;          // [tile][buffer] P V MMA done (commit)
   uint64_t* q_full = p_free + 4;          // [tile] Q in shared memory (TMA bytes)
-  uint64_t* o_last = q_full + 2;          // [tile] every MMA of the tile done (commit), once
-  uint64_t* v_tail = o_last + 2;          // last chunk's V tail rows cleared (producer), once
+  uint64_t* q_free = q_full + 2;          // [tile] the item's last S MMA done (commit)
+  uint64_t* o_last = q_free + 2;          // [tile] every MMA of the item done (commit)
+  uint64_t* o_empty = o_last + 2;         // [tile] O read out of TMEM (4 warp arrivals)
+  uint64_t* mma_done = o_empty + 2;       // [tile] every MMA of the CTA done (commit), once
+  uint64_t* v_tail = mma_done + 2;        // a last chunk's V tail rows cleared (producer)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_tail + 1);
 
   grid_dependents_launch();
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const PrefillItem it = pf.items[blockIdx.x];
   const int G = a.group;
   const int Hkv = a.num_kv_heads;
-  const int TQ = ROWS / G;                                   // query tokens per tile
-  const int ntiles = (Cfg::TILES == 2 && it.q_count > TQ) ? 2 : 1;  // tile 1 idles when empty
-  const int span0 = it.block_begin * BS;
-  const int span_end = min(it.block_end * BS, it.kv_end);
-  const int nchunks = span_end > span0 ? (span_end - span0 + CHUNK - 1) / CHUNK : 0;
-  // V rows of the last chunk past the span (when it is partial) must read as 0.
-  const int vt_last = nchunks > 0 ? span_end - (span0 + (nchunks - 1) * CHUNK) : CHUNK;
+  const int TQ = ROWS / G;  // query tokens per tile
+  // This CTA's items, in order.
+  const int k_begin = pf.sched_off ? pf.sched_off[blockIdx.x] : static_cast<int>(blockIdx.x);
+  const int k_end = pf.sched_off ? pf.sched_off[blockIdx.x + 1] : k_begin + 1;
 
   if (tid == 0) {
     for (int i = 0; i < NSLOT; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], ntiles);  // one commit per tile's issuer
+      mbar_init(&kv_empty[i], Cfg::TILES);  // one arrival per tile's issuer, idle or not
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
@@ -162,7 +188,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&q_full[t], 1);
+      mbar_init(&q_free[t], 1);
       mbar_init(&o_last[t], 1);
+      mbar_init(&o_empty[t], 4);
+      mbar_init(&mma_done[t], 1);
     }
     mbar_init(v_tail, 1);
     fence_barrier_init();
@@ -176,128 +205,175 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
   tmem_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
+  // Every role walks the same items and keeps its own running counts; a
+  // barrier's phase parity follows from them:
+  //   g  - K/V loads before the item (ring slot g % NSLOT, use g / NSLOT);
+  //   cb - chunks of tile t before the item (S / P buffer cb & 1);
+  //   nt - items tile t took part in (q_full, q_free, o_last, o_empty);
+  //   tails - items with a partial last chunk (v_tail).
   if (warp == SMW) {
-    // ---- producer: K_0, V_0, K_1, V_1, ... into the slot ring -----------------------
+    // ---- producer: K_0, V_0, K_1, V_1, ... of every item into the slot ring ----------
     const uint64_t policy = l2_policy(2);  // every query tile of a sequence re-reads its blocks
-    const int32_t* bt = a.block_tables + static_cast<int64_t>(it.seq) * a.max_blocks_per_seq;
-    // Block ids of the span's 16-token units, 32 units per batch held one per
-    // lane, the next batch loaded a batch ahead (a chunk's units never
-    // straddle two batches).
-    const int nunits = (span_end - span0 + UR - 1) / UR;
-    auto unit_ids = [&](int batch) -> int {
-      const int u = batch * 32 + lane;
-      return u < nunits ? bt[(span0 + u * UR) / BS] : -1;
-    };
-    // Q of each tile first: rows past the query tokens of the array read as 0
-    // (the box's out-of-range fill), rows past the item's tokens are masked.
-    // When Q was packed by a preceding kernel (launched as its programmatic
-    // dependent), wait for that grid here; K/V prefetch is not held back.
-    grid_dependency_wait();
-    if (elect_one()) {
-      for (int t = 0; t < ntiles; ++t) {
-        mbar_arrive_expect_tx(&q_full[t], KCH * TQ * G * 128);
-        for (int c = 0; c < KCH; ++c)
-          tma_load_3d(qs + t * Cfg::kQBytes + c * (ROWS * 128), &tm_q, &q_full[t], c * 64,
-                      it.q_head0, it.q_begin + t * TQ);
-      }
-    }
-    __syncwarp();
-    int ids = unit_ids(0);
-    int ids_next = unit_ids(1);
-    int batch = 0;
-    int issued = 0;
-    for (int i = 0; i < 2 * nchunks; ++i) {
-      const int j = i >> 1;
-      const int slot = i % NSLOT;
-      const int use = i / NSLOT;
-      bool ok = true;
-      if (use > 0) ok = mbar_wait_bounded(&kv_empty[slot], (use - 1) & 1, a.dev_err);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const int c0 = span0 + j * CHUNK;
-      const int nu = min(Cfg::UPC, (span_end - c0 + UR - 1) / UR);  // units holding used tokens
-      const int u0 = j * Cfg::UPC;
-      if ((u0 >> 5) != batch) {
-        batch = u0 >> 5;
-        ids = ids_next;
-        ids_next = unit_ids(batch + 1);
-      }
-      int phys_u[Cfg::UPC];
-#pragma unroll
-      for (int u = 0; u < Cfg::UPC; ++u) phys_u[u] = __shfl_sync(0xffffffffu, ids, (u0 + u) & 31);
-      // Every value above is warp-uniform; one elected lane of the converged
-      // warp issues the copies.
-      if (elect_one()) {
-        const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
-        uint8_t* dst = slots + slot * Cfg::kSlotBytes;
-        uint32_t bytes = 0;
-#pragma unroll
-        for (int u = 0; u < Cfg::UPC; ++u)
-          if (u < nu && phys_u[u] >= 0 && phys_u[u] < a.num_blocks) bytes += KCH * UR * 128;
-        mbar_arrive_expect_tx(&kv_full[slot], bytes);
-#pragma unroll
-        for (int u = 0; u < Cfg::UPC; ++u) {
-          if (u >= nu) continue;
-          const int ph = phys_u[u];
-          if (ph < 0 || ph >= a.num_blocks) {
-            if (i & 1) report(a.dev_err, PA_DEVERR_BLOCK_ID);  // the unit keeps stale rows
-            continue;
-          }
-          const int32_t y = (ph * Hkv + it.kvh) * BS + ((c0 + u * UR) % BS);
-#pragma unroll
-          for (int c = 0; c < KCH; ++c)
-            tma_load_2d(dst + c * (CHUNK * 128) + u * (UR * 128), map, &kv_full[slot], c * 64, y, policy);
+    int g = 0;
+    int prev_tail = -1;  // ring index of the previous partial chunk's V
+    bool ok = true;
+    for (int idx = k_begin; idx < k_end && ok; ++idx) {
+      const TcItem x = tc_item<Cfg>(pf, idx, TQ);
+      if (x.nchunks == 0) continue;
+      const int32_t* bt = a.block_tables + static_cast<int64_t>(x.it.seq) * a.max_blocks_per_seq;
+      // Block ids of the span's 16-token units, 32 units per batch held one per
+      // lane, the next batch loaded a batch ahead (a chunk's units never
+      // straddle two batches).
+      const int nunits = (x.span_end - x.span0 + UR - 1) / UR;
+      auto unit_ids = [&](int batch) -> int {
+        const int u = batch * 32 + lane;
+        return u < nunits ? bt[(x.span0 + u * UR) / BS] : -1;
+      };
+      int ids = unit_ids(0);
+      int ids_next = unit_ids(1);
+      int batch = 0;
+      for (int i = 0; i < 2 * x.nchunks; ++i) {
+        const int j = i >> 1;
+        const int gi = g + i;
+        const int slot = gi % NSLOT;
+        const int use = gi / NSLOT;
+        if (use > 0) ok = mbar_wait_bounded(&kv_empty[slot], (use - 1) & 1, a.dev_err);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          g = gi;  // loads issued so far
+          break;
         }
+        const int c0 = x.span0 + j * CHUNK;
+        const int nu = min(Cfg::UPC, (x.span_end - c0 + UR - 1) / UR);  // units holding used tokens
+        const int u0 = j * Cfg::UPC;
+        if ((u0 >> 5) != batch) {
+          batch = u0 >> 5;
+          ids = ids_next;
+          ids_next = unit_ids(batch + 1);
+        }
+        int phys_u[Cfg::UPC];
+#pragma unroll
+        for (int u = 0; u < Cfg::UPC; ++u) phys_u[u] = __shfl_sync(0xffffffffu, ids, (u0 + u) & 31);
+        // Every value above is warp-uniform; one elected lane of the converged
+        // warp issues the copies.
+        if (elect_one()) {
+          const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
+          uint8_t* dst = slots + slot * Cfg::kSlotBytes;
+          uint32_t bytes = 0;
+#pragma unroll
+          for (int u = 0; u < Cfg::UPC; ++u)
+            if (u < nu && phys_u[u] >= 0 && phys_u[u] < a.num_blocks) bytes += KCH * UR * 128;
+          mbar_arrive_expect_tx(&kv_full[slot], bytes);
+#pragma unroll
+          for (int u = 0; u < Cfg::UPC; ++u) {
+            if (u >= nu) continue;
+            const int ph = phys_u[u];
+            if (ph < 0 || ph >= a.num_blocks) {
+              if (i & 1) report(a.dev_err, PA_DEVERR_BLOCK_ID);  // the unit keeps stale rows
+              continue;
+            }
+            const int32_t y = (ph * Hkv + x.it.kvh) * BS + ((c0 + u * UR) % BS);
+#pragma unroll
+            for (int c = 0; c < KCH; ++c)
+              tma_load_2d(dst + c * (CHUNK * 128) + u * (UR * 128), map, &kv_full[slot], c * 64, y, policy);
+          }
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      issued = i + 1;
-    }
-    // Clear V rows [vt_last, CHUNK) of the last chunk once its copy landed
-    // (stale or unloaded rows; 0 * NaN is NaN), then release its P V.
-    if (issued == 2 * nchunks && vt_last < CHUNK) {
-      const int i = 2 * nchunks - 1;
-      const bool landed =
-          __all_sync(0xffffffffu, mbar_wait_bounded(&kv_full[i % NSLOT], (i / NSLOT) & 1, a.dev_err));
-      if (landed) {
-        uint8_t* vst = slots + (i % NSLOT) * Cfg::kSlotBytes;
-        const int n16 = (CHUNK - vt_last) * KCH * 8;
-        for (int x = lane; x < n16; x += 32) {
-          const int row = vt_last + x / (KCH * 8);
-          const int rem = x % (KCH * 8);
+      if (!ok) break;
+      // Clear V rows [vt_last, CHUNK) of a partial last chunk once its copy
+      // landed (stale or unloaded rows; 0 * NaN is NaN), then release its P V.
+      // The previous clear must have been waited for by both issuers first
+      // (its slot released), so v_tail never runs two phases ahead of a waiter.
+      if (x.vt_last < CHUNK) {
+        const int gi = g + 2 * x.nchunks - 1;
+        bool ready = mbar_wait_bounded(&kv_full[gi % NSLOT], (gi / NSLOT) & 1, a.dev_err);
+        if (ready && prev_tail >= 0 && gi - prev_tail < NSLOT)
+          ready = mbar_wait_bounded(&kv_empty[prev_tail % NSLOT], (prev_tail / NSLOT) & 1, a.dev_err);
+        if (!__all_sync(0xffffffffu, ready)) {
+          ok = false;
+          g += 2 * x.nchunks;
+          break;
+        }
+        uint8_t* vst = slots + (gi % NSLOT) * Cfg::kSlotBytes;
+        const int n16 = (CHUNK - x.vt_last) * KCH * 8;
+        for (int e = lane; e < n16; e += 32) {
+          const int row = x.vt_last + e / (KCH * 8);
+          const int rem = e % (KCH * 8);
           *reinterpret_cast<uint4*>(vst + (rem >> 3) * (CHUNK * 128) + row * 128 + ((rem & 7) << 4)) =
               make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(v_tail);
+        prev_tail = gi;
       }
+      g += 2 * x.nchunks;
     }
     // Every copy issued has landed before the CTA's shared memory is released.
-    for (int i = max(0, issued - NSLOT); i < issued; ++i)
-      mbar_wait_bounded(&kv_full[i % NSLOT], (i / NSLOT) & 1, a.dev_err);
+    for (int gi = max(0, g - NSLOT); gi < g; ++gi)
+      mbar_wait_bounded(&kv_full[gi % NSLOT], (gi / NSLOT) & 1, a.dev_err);
     __syncwarp();
   } else if (warp > SMW) {
     // ---- MMA issuer of tile t: the whole warp runs the loop (waits are warp-wide,
-    // values warp-uniform); one elected lane issues each group of MMAs and commits.
+    // values warp-uniform); one elected lane issues each group of MMAs and commits,
+    // and loads the tile's Q (the next item's as soon as this item's last S is done).
     const int t = warp - SMW - 1;
-    if (t < ntiles && nchunks > 0) {
-      constexpr uint32_t kIdS = umma_idesc_bf16(ROWS, CHUNK, 0, 0);
-      constexpr uint32_t kIdO = umma_idesc_bf16(ROWS, D, 0, 1);
-      // Descriptors are built once; a start address moves by adding its
-      // offset in 16-byte units (the 14-bit field cannot overflow below 256 KB).
-      const uint64_t q_desc = umma_desc_sw128(smem_addr(qs + t * Cfg::kQBytes), 16, 1024);
-      const uint64_t k_desc = umma_desc_sw128(smem_addr(slots), 16, 1024);
-      const uint64_t v_desc = umma_desc_sw128(smem_addr(slots), CHUNK * 128, 1024);
-      const uint32_t s_tmem = tmem + t * Cfg::kTileCols;
-      const uint32_t o_tmem = tmem + t * Cfg::kTileCols + Cfg::kOCol;
-      auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, a.dev_err));
-      };
-      // S_t(j) = Q_t K_j^T into buffer j & 1, once P V of chunk j - 2 has
-      // read the P that the buffer holds.
+    constexpr uint32_t kIdS = umma_idesc_bf16(ROWS, CHUNK, 0, 0);
+    constexpr uint32_t kIdO = umma_idesc_bf16(ROWS, D, 0, 1);
+    // Descriptors are built once; a start address moves by adding its
+    // offset in 16-byte units (the 14-bit field cannot overflow below 256 KB).
+    const uint64_t q_desc = umma_desc_sw128(smem_addr(qs + t * Cfg::kQBytes), 16, 1024);
+    const uint64_t k_desc = umma_desc_sw128(smem_addr(slots), 16, 1024);
+    const uint64_t v_desc = umma_desc_sw128(smem_addr(slots), CHUNK * 128, 1024);
+    const uint32_t s_tmem = tmem + t * Cfg::kTileCols;
+    const uint32_t o_tmem = tmem + t * Cfg::kTileCols + Cfg::kOCol;
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, a.dev_err));
+    };
+    // Q of tile t of an item: rows past the query tokens of the array read as
+    // 0 (the box's out-of-range fill), rows past the item's tokens are masked.
+    int q_loads = 0, q_seen = 0;
+    auto load_q = [&](const TcItem& y) {
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&q_full[t], KCH * TQ * G * 128);
+        for (int c = 0; c < KCH; ++c)
+          tma_load_3d(qs + t * Cfg::kQBytes + c * (ROWS * 128), &tm_q, &q_full[t], c * 64,
+                      y.it.q_head0, y.it.q_begin + t * TQ);
+      }
+      __syncwarp();
+      ++q_loads;
+    };
+    // When Q was packed by a preceding kernel (launched as its programmatic
+    // dependent), wait for that grid before the first Q copy.
+    grid_dependency_wait();
+    int g = 0, cb = 0, nt = 0, tails = 0;
+    bool ok = true;
+    for (int idx = k_begin; idx < k_end && ok; ++idx) {
+      const TcItem x = tc_item<Cfg>(pf, idx, TQ);
+      if (x.nchunks == 0) continue;
+      const bool tail = x.vt_last < CHUNK;
+      if (t >= x.ntiles) {
+        // An idle tile still releases every slot of the item.
+        for (int i = 0; i < 2 * x.nchunks && ok; ++i) {
+          const int gi = g + i;
+          ok = wait(&kv_full[gi % NSLOT], (gi / NSLOT) & 1);
+          if (ok && elect_one()) mbar_arrive(&kv_empty[gi % NSLOT]);
+          __syncwarp();
+        }
+        g += 2 * x.nchunks;
+        tails += tail ? 1 : 0;
+        continue;
+      }
+      if (q_loads == q_seen) load_q(x);
+      ok = wait(&q_full[t], q_seen & 1);
+      ++q_seen;
+      // S_t(j) = Q_t K_j^T into buffer (cb + j) & 1, once the P V that last
+      // read that buffer (two chunks back) is done.
       auto issue_s = [&](int j) -> bool {
-        const int i = 2 * j, slot = i % NSLOT, b = j & 1;
-        if (!wait(&kv_full[slot], (i / NSLOT) & 1)) return false;
-        if (j >= 2 && !wait(&p_free[2 * t + b], ((j >> 1) - 1) & 1)) return false;
+        const int gi = g + 2 * j, slot = gi % NSLOT, c = cb + j, b = c & 1;
+        if (!wait(&kv_full[slot], (gi / NSLOT) & 1)) return false;
+        if (c >= 2 && !wait(&p_free[2 * t + b], ((c >> 1) - 1) & 1)) return false;
         tmem_fence_after_sync();
         const uint64_t kd = k_desc + static_cast<uint32_t>((slot * Cfg::kSlotBytes) >> 4);
         if (elect_one()) {
@@ -311,15 +387,36 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
         __syncwarp();
         return true;
       };
+      // After the item's last S: once it is done, Q's buffer is free and the
+      // next item this tile takes part in gets its Q copy started.
+      auto after_last_s = [&]() -> bool {
+        if (elect_one()) umma_commit(&q_free[t]);
+        __syncwarp();
+        for (int n = idx + 1; n < k_end; ++n) {
+          const TcItem y = tc_item<Cfg>(pf, n, TQ);
+          if (y.nchunks == 0 || t >= y.ntiles) continue;
+          if (!wait(&q_free[t], nt & 1)) return false;
+          load_q(y);
+          break;
+        }
+        return true;
+      };
+      ok = ok && issue_s(0);
+      if (ok && x.nchunks == 1) ok = after_last_s();
       // Issuing whichever of S and P V became ready first measured the same
       // as this fixed order (S of the next chunk, then P V of this one).
-      bool ok = wait(&q_full[t], 0) && issue_s(0);
-      for (int j = 0; j < nchunks && ok; ++j) {
-        if (j + 1 < nchunks && !issue_s(j + 1)) break;
-        const int i = 2 * j + 1, slot = i % NSLOT, b = j & 1;
-        ok = wait(&kv_full[slot], (i / NSLOT) & 1);
-        if (ok && j == nchunks - 1 && vt_last < CHUNK) ok = wait(v_tail, 0);
-        ok = ok && wait(&p_full[2 * t + b], (j >> 1) & 1);
+      for (int j = 0; j < x.nchunks && ok; ++j) {
+        if (j + 1 < x.nchunks) {
+          ok = issue_s(j + 1);
+          if (ok && j + 2 == x.nchunks) ok = after_last_s();
+          if (!ok) break;
+        }
+        const int gi = g + 2 * j + 1, slot = gi % NSLOT, c = cb + j, b = c & 1;
+        ok = wait(&kv_full[slot], (gi / NSLOT) & 1);
+        if (ok && tail && j == x.nchunks - 1) ok = wait(v_tail, tails & 1);
+        ok = ok && wait(&p_full[2 * t + b], (c >> 1) & 1);
+        // The first P V of an item overwrites O: the previous item's O must be read out.
+        if (ok && j == 0 && nt > 0) ok = wait(&o_empty[t], (nt - 1) & 1);
         if (!ok) break;
         tmem_fence_after_sync();
         const uint64_t vd = v_desc + static_cast<uint32_t>((slot * Cfg::kSlotBytes) >> 4);
@@ -333,152 +430,177 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
         }
         __syncwarp();
       }
-      // o_last completes once every MMA issued above has; TMEM is freed after it.
-      // elect.sync picks the same lane of the fully active warp every time,
-      // so the MMAs above and this commit share one issuing thread.
+      if (!ok) break;
       if (elect_one()) umma_commit(&o_last[t]);
       __syncwarp();
-      wait(&o_last[t], 0);
+      g += 2 * x.nchunks;
+      cb += x.nchunks;
+      tails += tail ? 1 : 0;
+      ++nt;
     }
+    // Before TMEM and shared memory are released: a Q copy still in flight
+    // (after an error), then every MMA this thread issued. elect.sync picks
+    // the same lane of the fully active warp every time, so the MMAs above
+    // and this commit share one issuing thread.
+    if (q_loads > q_seen) wait(&q_full[t], q_seen & 1);
+    if (elect_one()) umma_commit(&mma_done[t]);
+    __syncwarp();
+    wait(&mma_done[t], 0);
   } else {
     // ---- softmax warps: tile t = warp / 4, thread r owns row r (TMEM lane r) --------
     const int t = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
-    const int jq = t * TQ + r / G;                       // query token within the item
-    const bool valid = (r / G) < TQ && jq < it.q_count;
-    const int lim = valid ? it.p0 + jq : -1;             // last token this row attends to
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + t * Cfg::kTileCols;
-    const bool active = t < ntiles;
     const float sl2 = a.scale_log2;
-    float m_used = -INFINITY, l = 0.f;
+    int cb = 0, nt = 0;
     bool ok = true;  // warp-uniform
-    for (int j = 0; j < nchunks && active; ++j) {
-      const int b = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[2 * t + b], (j >> 1) & 1, a.dev_err));
-      if (!ok) break;
-      tmem_fence_after_sync();
-      float sv[CHUNK];
-      tmem_ld64(trow + b * CHUNK, sv);
-      const int c0 = span0 + j * CHUNK;
-      // Scaled logits: x = s * scale * log2(e). Only chunks that reach past
-      // the row's position or the span's end need the mask.
-      const bool whole = c0 + CHUNK <= span_end && c0 + CHUNK - 1 <= lim && sl2 > 0.f;
-      float mx;
-      if (whole) {
-        float m8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float* v = sv + 8 * k;
-          m8[k] = fmax3(fmax3(v[0], v[1], v[2]), fmax3(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
-        }
-        mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
-      } else {
-        mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < CHUNK; ++i) {
-          const int tk = c0 + i;
-          const bool in = tk < span_end && tk <= lim;
-          sv[i] = in ? sv[i] * sl2 : -INFINITY;
-          mx = fmaxf(mx, sv[i]);
-        }
-      }
-      const bool raise = mx > m_used + Cfg::kRescaleThreshold;
-      const bool rescale_o = raise && m_used != -INFINITY;
-      if (__any_sync(0xffffffffu, rescale_o)) {
-        // O must hold every earlier P V product before it is scaled.
-        const int pb = 2 * t + ((j - 1) & 1);
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&p_free[pb], ((j - 1) >> 1) & 1, a.dev_err));
+    for (int idx = k_begin; idx < k_end && ok; ++idx) {
+      const TcItem x = tc_item<Cfg>(pf, idx, TQ);
+      if (t >= x.ntiles) continue;                         // no row of this tile is a query row
+      const PrefillItem& it = x.it;
+      const int nchunks = x.nchunks;
+      const int span_end = x.span_end;
+      const int jq = t * TQ + r / G;                       // query token within the item
+      const bool valid = (r / G) < TQ && jq < it.q_count;
+      const int lim = valid ? it.p0 + jq : -1;             // last token this row attends to
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < nchunks; ++j) {
+        const int c = cb + j;
+        const int b = c & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[2 * t + b], (c >> 1) & 1, a.dev_err));
         if (!ok) break;
         tmem_fence_after_sync();
-        const float alpha = rescale_o ? fast_exp2(m_used - mx) : 1.f;
+        float sv[CHUNK];
+        tmem_ld64(trow + b * CHUNK, sv);
+        const int c0 = x.span0 + j * CHUNK;
+        // Scaled logits: x = s * scale * log2(e). Only chunks that reach past
+        // the row's position or the span's end need the mask.
+        const bool whole = c0 + CHUNK <= span_end && c0 + CHUNK - 1 <= lim && sl2 > 0.f;
+        float mx;
+        if (whole) {
+          float m8[8];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float o32[32];
-          tmem_ld32(trow + Cfg::kOCol + c * 32, o32);
+          for (int k = 0; k < 8; ++k) {
+            const float* v = sv + 8 * k;
+            m8[k] = fmax3(fmax3(v[0], v[1], v[2]), fmax3(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+          }
+          mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
+        } else {
+          mx = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o32[i] *= alpha;
-          tmem_st32(trow + Cfg::kOCol + c * 32, o32);
+          for (int i = 0; i < CHUNK; ++i) {
+            const int tk = c0 + i;
+            const bool in = tk < span_end && tk <= lim;
+            sv[i] = in ? sv[i] * sl2 : -INFINITY;
+            mx = fmaxf(mx, sv[i]);
+          }
         }
+        const bool raise = mx > m_used + Cfg::kRescaleThreshold;
+        const bool rescale_o = raise && m_used != -INFINITY;  // only from the item's second chunk on
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          // O must hold every earlier P V product of the item before it is scaled.
+          const int pb = 2 * t + ((c - 1) & 1);
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&p_free[pb], ((c - 1) >> 1) & 1, a.dev_err));
+          if (!ok) break;
+          tmem_fence_after_sync();
+          const float alpha = rescale_o ? fast_exp2(m_used - mx) : 1.f;
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            float o32[32];
+            tmem_ld32(trow + Cfg::kOCol + q * 32, o32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o32[i] *= alpha;
+            tmem_st32(trow + Cfg::kOCol + q * 32, o32);
+          }
+          tmem_fence_before_sync();
+          l *= alpha;
+        }
+        if (raise) m_used = mx;
+        // P = 2^(x - m_used) <= 2^8, as packed bf16 pairs over the logits.
+        uint32_t pk[CHUNK / 2];
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (whole) {
+          const uint64_t sl2_2 = f2_pack(sl2, sl2);
+          const uint64_t nm2 = f2_pack(-m_used, -m_used);
+          uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+          for (int i = 0; i < CHUNK; i += 2) {
+            const uint64_t x2 = f2_fma(f2_pack(sv[i], sv[i + 1]), sl2_2, nm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
+            acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(p0, p1));
+            pk[i >> 1] = pack_bf16x2(p0, p1);
+          }
+          float a0, a1, b0, b1;
+          f2_unpack(acc2[0], a0, a1);
+          f2_unpack(acc2[1], b0, b1);
+          s4[0] = a0; s4[1] = a1; s4[2] = b0; s4[3] = b1;
+        } else {
+          const float mu = (m_used == -INFINITY) ? 0.f : m_used;  // a row with nothing yet: all p = 0
+#pragma unroll
+          for (int i = 0; i < CHUNK; i += 2) {
+            const float p0 = fast_exp2(sv[i] - mu);
+            const float p1 = fast_exp2(sv[i + 1] - mu);
+            s4[(i >> 1) & 3] += p0 + p1;
+            pk[i >> 1] = pack_bf16x2(p0, p1);
+          }
+        }
+        l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        tmem_st32_bits(trow + b * CHUNK, pk);
         tmem_fence_before_sync();
-        l *= alpha;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[2 * t + b]);
       }
-      if (raise) m_used = mx;
-      // P = 2^(x - m_used) <= 2^8, as packed bf16 pairs over the logits.
-      uint32_t pk[CHUNK / 2];
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (whole) {
-        const uint64_t sl2_2 = f2_pack(sl2, sl2);
-        const uint64_t nm2 = f2_pack(-m_used, -m_used);
-        uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-#pragma unroll
-        for (int i = 0; i < CHUNK; i += 2) {
-          const uint64_t x2 = f2_fma(f2_pack(sv[i], sv[i + 1]), sl2_2, nm2);
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          const float p0 = fast_exp2(x0);
-          const float p1 = fast_exp2(x1);
-          acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(p0, p1));
-          pk[i >> 1] = pack_bf16x2(p0, p1);
-        }
-        float a0, a1, b0, b1;
-        f2_unpack(acc2[0], a0, a1);
-        f2_unpack(acc2[1], b0, b1);
-        s4[0] = a0; s4[1] = a1; s4[2] = b0; s4[3] = b1;
-      } else {
-        const float mu = (m_used == -INFINITY) ? 0.f : m_used;  // a row with nothing yet: all p = 0
-#pragma unroll
-        for (int i = 0; i < CHUNK; i += 2) {
-          const float p0 = fast_exp2(sv[i] - mu);
-          const float p1 = fast_exp2(sv[i + 1] - mu);
-          s4[(i >> 1) & 3] += p0 + p1;
-          pk[i >> 1] = pack_bf16x2(p0, p1);
-        }
-      }
-      l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      tmem_st32_bits(trow + b * CHUNK, pk);
-      tmem_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[2 * t + b]);
-    }
-    // ---- epilogue: O from TMEM, normalised (single partition) or as a partial --------------
-    if (active) {
-      if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_last[t], 0, a.dev_err));
-      if (ok) {
+      if (!ok) break;
+      // ---- the item's epilogue: O from TMEM, normalised (single partition) or
+      // as a partial; then O's columns are handed back for the next item.
+      if (nchunks > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_last[t], nt & 1, a.dev_err));
+        if (!ok) break;
         tmem_fence_after_sync();
-        const int64_t tok = !valid ? it.q_begin
-                            : it.out_begin >= 0 ? pf.out_tokens[it.out_begin + jq] : it.q_begin + jq;
-        const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
-        const int64_t row = tok * a.num_q_heads + h;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+      }
+      const int64_t tok = !valid ? it.q_begin
+                          : it.out_begin >= 0 ? pf.out_tokens[it.out_begin + jq] : it.q_begin + jq;
+      const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
+      const int64_t row = tok * a.num_q_heads + h;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float o32[32];
-          if (nchunks > 0) {
-            tmem_ld32(trow + Cfg::kOCol + c * 32, o32);
-          } else {
+      for (int q = 0; q < D / 32; ++q) {
+        float o32[32];
+        if (nchunks > 0) {
+          tmem_ld32(trow + Cfg::kOCol + q * 32, o32);
+        } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = 0.f;
-          }
-          if (!valid) continue;
-          if (it.final_out) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * D + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pack_bf16x2(o32[8 * i] * inv, o32[8 * i + 1] * inv),
-                                  pack_bf16x2(o32[8 * i + 2] * inv, o32[8 * i + 3] * inv),
-                                  pack_bf16x2(o32[8 * i + 4] * inv, o32[8 * i + 5] * inv),
-                                  pack_bf16x2(o32[8 * i + 6] * inv, o32[8 * i + 7] * inv));
-          } else {
-            float4* dst = reinterpret_cast<float4*>(a.part_acc + (row * a.max_partitions + it.part) * D + c * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(o32[4 * i], o32[4 * i + 1], o32[4 * i + 2], o32[4 * i + 3]);
-          }
+          for (int i = 0; i < 32; ++i) o32[i] = 0.f;
         }
-        if (valid && !it.final_out) {
-          a.part_m[row * a.max_partitions + it.part] = m_used;
-          a.part_l[row * a.max_partitions + it.part] = l;
+        if (!valid) continue;
+        if (it.final_out) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * D + q * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(pack_bf16x2(o32[8 * i] * inv, o32[8 * i + 1] * inv),
+                                pack_bf16x2(o32[8 * i + 2] * inv, o32[8 * i + 3] * inv),
+                                pack_bf16x2(o32[8 * i + 4] * inv, o32[8 * i + 5] * inv),
+                                pack_bf16x2(o32[8 * i + 6] * inv, o32[8 * i + 7] * inv));
+        } else {
+          float4* dst = reinterpret_cast<float4*>(a.part_acc + (row * a.max_partitions + it.part) * D + q * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(o32[4 * i], o32[4 * i + 1], o32[4 * i + 2], o32[4 * i + 3]);
         }
+      }
+      if (valid && !it.final_out) {
+        a.part_m[row * a.max_partitions + it.part] = m_used;
+        a.part_l[row * a.max_partitions + it.part] = l;
+      }
+      if (nchunks > 0) {
+        tmem_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_empty[t]);
+        cb += nchunks;
+        ++nt;
       }
     }
   }

@@ -18,7 +18,10 @@ from gpu_util import check_close, device_tables, setup, to_f64
 pytestmark = pytest.mark.gpu
 
 
-KERNELS = ["tcgen05", "mma_sync"]
+# "tcgen05_3ctas": the tcgen05 kernel's persistent launch capped at 3 CTAs,
+# so that every CTA runs many items back to back (idle second tiles, empty
+# spans, partial last chunks and partition items in one CTA's sequence).
+KERNELS = ["tcgen05", "tcgen05_3ctas", "mma_sync"]
 
 
 @pytest.fixture(params=KERNELS)
@@ -27,6 +30,10 @@ def kernel(request, monkeypatch):
         monkeypatch.setenv("PAGEDKV_PREFILL_KERNEL", "mma_sync")
     else:
         monkeypatch.delenv("PAGEDKV_PREFILL_KERNEL", raising=False)
+    if request.param == "tcgen05_3ctas":
+        monkeypatch.setenv("PAGEDKV_PREFILL_CTAS", "3")
+    else:
+        monkeypatch.delenv("PAGEDKV_PREFILL_CTAS", raising=False)
     return request.param
 
 
