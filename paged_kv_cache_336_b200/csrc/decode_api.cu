@@ -743,7 +743,8 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
     a.scale_log2 = r.scale * 1.4426950408889634f;
     pf.items = reinterpret_cast<const PrefillItem*>(ws + L.items_off);
     pf.out_tokens = reinterpret_cast<const int32_t*>(ws + L.members_off);
-    void* args[] = {&tmk, &tmv, &tmq, &pf};
+    // The output map is unused here (rows are scattered through out_tokens).
+    void* args[] = {&tmk, &tmv, &tmq, &tmq, &pf};
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(tc_items.size()));
     cfg.blockDim = dim3(pinst.threads);
@@ -994,14 +995,18 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
   pf.items = reinterpret_cast<const PrefillItem*>(ws + L.items_off);
   pf.out_tokens = nullptr;
   pf.sched_off = persistent ? reinterpret_cast<const int32_t*>(ws + L.sched_off) : nullptr;
-  CUtensorMap tmq;
+  CUtensorMap tmq, tmo;
   void* args3[] = {&tmk, &tmv, &pf};
-  void* args4[] = {&tmk, &tmv, &tmq, &pf};
+  void* args5[] = {&tmk, &tmv, &tmq, &tmo, &pf};
   if (pinst.q_map) {
-    st = q_tensor_map(r.q, total_q, r.num_q_heads, r.head_dim, G, std::max(1, pinst.rows / G), &tmq);
+    // out has q's layout: the same boxes serve the output tiles' stores.
+    const int tile_tokens = std::max(1, pinst.rows / G);
+    st = q_tensor_map(r.q, total_q, r.num_q_heads, r.head_dim, G, tile_tokens, &tmq);
+    if (st != PA_OK) return st;
+    st = q_tensor_map(r.out, total_q, r.num_q_heads, r.head_dim, G, tile_tokens, &tmo);
     if (st != PA_OK) return st;
   }
-  err = cudaLaunchKernel(pinst.kernel, dim3(grid), dim3(pinst.threads), pinst.q_map ? args4 : args3,
+  err = cudaLaunchKernel(pinst.kernel, dim3(grid), dim3(pinst.threads), pinst.q_map ? args5 : args3,
                          pinst.smem, r.stream);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(err));
   if (any_split) {

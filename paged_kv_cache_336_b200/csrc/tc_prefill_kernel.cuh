@@ -93,7 +93,11 @@ struct TcCfg {
   static constexpr int NSLOT = TILES == 2 ? 8 : 4;
   static constexpr int kMinBlocks = TILES == 2 ? 1 : 2;
   static constexpr int kBarBytes = 512;
-  static constexpr int kSmem = 1024 + TILES * kQBytes + NSLOT * kSlotBytes + kBarBytes;
+  // Two-tile CTAs stage each tile's normalised output, 64 columns at a time,
+  // for one TMA store (one-tile CTAs serve scattered output rows).
+  static constexpr bool kTmaOut = TILES == 2;
+  static constexpr int kStageBytes = kTmaOut ? TILES * ROWS * 128 : 0;
+  static constexpr int kSmem = 1024 + TILES * kQBytes + NSLOT * kSlotBytes + kStageBytes + kBarBytes;
   static constexpr int kSoftmaxWarps = 4 * TILES;
   static constexpr int kThreads = (kSoftmaxWarps + 1 + TILES) * 32;
   static constexpr uint32_t kTileCols = 256;            // S buffers [0,128), O [128, 128 + D)
@@ -135,7 +139,8 @@ template <class Cfg>
 __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     tc_prefill_kernel(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_q, const PrefillArgs pf) {
+                      const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_o, const PrefillArgs pf) {
   constexpr int NSLOT = Cfg::NSLOT;
   constexpr int BS = Cfg::BS;
   constexpr int D = Cfg::D;
@@ -151,7 +156,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* qs = smem;                                    // [TILES][KCH][ROWS][128 B]
   uint8_t* slots = qs + Cfg::TILES * Cfg::kQBytes;       // [NSLOT][KCH][CHUNK][128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(slots + NSLOT * Cfg::kSlotBytes);
+  uint8_t* stage = slots + NSLOT * Cfg::kSlotBytes;      // [TILES][ROWS][128 B] output staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage + Cfg::kStageBytes);
   uint64_t* kv_full = bars;               // [NSLOT] TMA bytes landed
   uint64_t* kv_empty = bars + NSLOT;      // [NSLOT] both tiles done with the slot
   uint64_t* s_full = bars + 2 * NSLOT;    // [tile][buffer] S MMA done (commit)
@@ -566,29 +572,66 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
       const int64_t row = tok * a.num_q_heads + h;
       const float inv = l > 0.f ? 1.f / l : 0.f;
+      // A full tile of final rows goes out by TMA: its rows (token-major,
+      // head-minor, as Q came in) are staged 64 columns at a time in the
+      // 128-byte swizzle and stored as one box; one thread per tile issues
+      // the stores. Partial tiles, scattered rows and partials use plain
+      // stores (each thread its own row).
+      const bool tma_out = Cfg::kTmaOut && nchunks > 0 && it.final_out && it.out_begin < 0 &&
+                           it.q_count >= (t + 1) * TQ;
+      if (tma_out) {
+        uint8_t* sbuf = stage + t * (ROWS * 128);
+        const bool leader = (warp & 3) == 0 && lane == 0;
 #pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        float o32[32];
-        if (nchunks > 0) {
-          tmem_ld32(trow + Cfg::kOCol + q * 32, o32);
-        } else {
+        for (int cc = 0; cc < KCH; ++cc) {
+          if (leader) bulk_wait_group_read0();  // the previous store has read the buffer
+          named_bar_sync(1 + t, 128);
+          uint8_t* rowp = sbuf + r * 128;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o32[i] = 0.f;
+          for (int qq = 0; qq < 4; ++qq) {
+            float o16[16];
+            tmem_ld16(trow + Cfg::kOCol + cc * 64 + qq * 16, o16);
+#pragma unroll
+            for (int p = 0; p < 2; ++p)
+              *reinterpret_cast<uint4*>(rowp + (((qq * 2 + p) ^ (r & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(o16[8 * p] * inv, o16[8 * p + 1] * inv),
+                             pack_bf16x2(o16[8 * p + 2] * inv, o16[8 * p + 3] * inv),
+                             pack_bf16x2(o16[8 * p + 4] * inv, o16[8 * p + 5] * inv),
+                             pack_bf16x2(o16[8 * p + 6] * inv, o16[8 * p + 7] * inv));
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1 + t, 128);
+          if (leader) {
+            tma_store_3d(&tm_o, sbuf, cc * 64, it.q_head0, it.q_begin + t * TQ);
+            bulk_commit_group();
+          }
         }
-        if (!valid) continue;
-        if (it.final_out) {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * D + q * 32);
+      }
+      if (!tma_out) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pack_bf16x2(o32[8 * i] * inv, o32[8 * i + 1] * inv),
-                                pack_bf16x2(o32[8 * i + 2] * inv, o32[8 * i + 3] * inv),
-                                pack_bf16x2(o32[8 * i + 4] * inv, o32[8 * i + 5] * inv),
-                                pack_bf16x2(o32[8 * i + 6] * inv, o32[8 * i + 7] * inv));
-        } else {
-          float4* dst = reinterpret_cast<float4*>(a.part_acc + (row * a.max_partitions + it.part) * D + q * 32);
+        for (int q = 0; q < D / 32; ++q) {
+          float o32[32];
+          if (nchunks > 0) {
+            tmem_ld32(trow + Cfg::kOCol + q * 32, o32);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(o32[4 * i], o32[4 * i + 1], o32[4 * i + 2], o32[4 * i + 3]);
+            for (int i = 0; i < 32; ++i) o32[i] = 0.f;
+          }
+          if (!valid) continue;
+          if (it.final_out) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * D + q * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16x2(o32[8 * i] * inv, o32[8 * i + 1] * inv),
+                                  pack_bf16x2(o32[8 * i + 2] * inv, o32[8 * i + 3] * inv),
+                                  pack_bf16x2(o32[8 * i + 4] * inv, o32[8 * i + 5] * inv),
+                                  pack_bf16x2(o32[8 * i + 6] * inv, o32[8 * i + 7] * inv));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(a.part_acc + (row * a.max_partitions + it.part) * D + q * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(o32[4 * i], o32[4 * i + 1], o32[4 * i + 2], o32[4 * i + 3]);
+          }
         }
       }
       if (valid && !it.final_out) {
@@ -604,6 +647,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       }
     }
   }
+  // Output stores complete before the CTA (and its staging memory) ends.
+  if (Cfg::kTmaOut && warp < SMW && (warp & 3) == 0 && lane == 0) bulk_wait_group0();
   tmem_fence_before_sync();
   __syncthreads();
   if (warp == 0) {
