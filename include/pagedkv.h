@@ -273,6 +273,31 @@ pa_status_t pa_prefill(const void* q, const void* k_pool, const void* v_pool,
                        uint32_t* dev_err, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * pa_prefill_plan - the work plan pa_prefill makes for its tcgen05 kernel,
+ * for inspection and tests; host only (no CUDA call, no device needed).
+ * Items are (sequence, run of query tokens, KV head, KV partition): one per
+ * partition of partition_tokens tokens of each KV head of each run of
+ * 2 x (128 / group) query tokens, in sequence order with each sequence's
+ * runs last-first. With max_ctas > 0 and more items than max_ctas, the
+ * items are scheduled over max_ctas CTAs: each goes, in that order, to the
+ * CTA with the least estimated work so far (ties to the lowest CTA), and
+ * the items are listed CTA by CTA, each CTA's in that order (the order the
+ * kernel runs them). Otherwise item i runs on CTA i.
+ *
+ * context_lens, query_lens: HOST int32 [num_seqs] (as for pa_prefill).
+ * num_items, num_ctas: out, the item count and the grid. items_out: NULL
+ * (counts only) or HOST int32 [max_items][6] rows (seq, first query token,
+ * query tokens, kv head, partition, cta); max_items below the item count is
+ * PA_ERR_INVALID_ARG. block_size 16 or 32, else PA_ERR_UNSUPPORTED.
+ * pa_prefill plans the same way, with max_ctas = the kernel's resident CTAs
+ * (capped by PAGEDKV_PREFILL_CTAS).
+ * ------------------------------------------------------------------------- */
+pa_status_t pa_prefill_plan(const int32_t* context_lens, const int32_t* query_lens, int num_seqs,
+                            int num_q_heads, int num_kv_heads, int block_size, int partition_tokens,
+                            int max_ctas, int32_t* items_out, int max_items, int* num_items,
+                            int* num_ctas);
+
+/* ---------------------------------------------------------------------------
  * pa_swap_out / pa_swap_in - the data movement of swapping: whole blocks
  * (K and V, all heads; block_bytes each) between the device pools and two
  * host buffers of num_host_slots blocks each. pairs (device int64

@@ -99,6 +99,8 @@ _SIGNATURES = {
     "pa_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "pa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P,
                         _SZ, _P, _P, _P]),
+    "pa_prefill_plan": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _I, ctypes.POINTER(_I),
+                             ctypes.POINTER(_I)]),
     "pa_bm_swap_out": (_I, [_P, _I64, _P, _I, ctypes.POINTER(_I)]),
     "pa_bm_swap_in": (_I, [_P, _I64, _P, _I, ctypes.POINTER(_I)]),
     "pa_swap_out": (_I, [_P, _P, _P, _P, _P, _I, _SZ, _I, _I, _P, _P]),
@@ -341,6 +343,26 @@ def prefill(q, k_pool, v_pool, block_tables, context_lens, query_lens, scale: fl
         B, total, Hq, Hkv, D, BS, NB, MBS, float(scale), _dtype_code(q), int(partition_tokens),
         workspace.ptr, workspace.nbytes, _ptr(out), _ptr(dev_err), _stream_ptr(stream)))
     return out
+
+
+def prefill_plan(context_lens, query_lens, num_q_heads: int, num_kv_heads: int, block_size: int,
+                 partition_tokens: int, max_ctas: int = 0):
+    """pa_prefill_plan (host only): the tcgen05 prefill kernel's items as an
+    int32 array [n, 6] of (seq, first query token, query tokens, kv head,
+    partition, cta), in the order the kernel runs them, and the grid size."""
+    import numpy as np
+    ctx = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    qlen = np.ascontiguousarray(np.asarray(query_lens, dtype=np.int32))
+    if ctx.shape != qlen.shape or ctx.ndim != 1:
+        raise InvalidArgumentError(PA_ERR_INVALID_ARG, "bad length arrays")
+    n, grid = ctypes.c_int(0), ctypes.c_int(0)
+    args = (ctx.ctypes.data, qlen.ctypes.data, len(ctx), int(num_q_heads), int(num_kv_heads),
+            int(block_size), int(partition_tokens), int(max_ctas))
+    _check(library().pa_prefill_plan(*args, None, 0, ctypes.byref(n), ctypes.byref(grid)))
+    items = np.zeros((n.value, 6), dtype=np.int32)
+    _check(library().pa_prefill_plan(*args, items.ctypes.data, n.value, ctypes.byref(n),
+                                     ctypes.byref(grid)))
+    return items, grid.value
 
 
 class Workspace:

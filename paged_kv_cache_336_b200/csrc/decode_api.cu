@@ -828,6 +828,124 @@ PrefillLayout prefill_layout(int num_seqs, int total_q, int num_q_heads, int num
   return L;
 }
 
+// The prefill items: one per (sequence, run of tq query tokens, KV head, KV
+// partition of pb blocks), in sequence order with each sequence's query
+// tiles last-first (the longest spans first), so that work handed out last
+// is short. lens (optional) receives each query token's attended length.
+void prefill_items(int B, const int32_t* ctx_host, const int32_t* qlen_host, int num_kv_heads, int G,
+                   int block_size, int tq, int pb, std::vector<PrefillItem>& items,
+                   std::vector<int32_t>* lens, bool* any_split) {
+  items.clear();
+  *any_split = false;
+  int q_base = 0;
+  for (int s = 0; s < B; ++s) {
+    const int qlen = qlen_host[s], ctx = ctx_host[s];
+    for (int t = qlen > 0 ? (qlen - 1) / tq * tq : -1; t >= 0; t -= tq) {
+      const int count = std::min(tq, qlen - t);
+      const int p0 = ctx - qlen + t;
+      const int kv_end = p0 + count;  // last position + 1
+      const int nblk = (kv_end + block_size - 1) / block_size;
+      const int nparts = (nblk + pb - 1) / pb;
+      *any_split = *any_split || nparts > 1;
+      if (lens != nullptr)
+        for (int i = 0; i < count; ++i) (*lens)[q_base + t + i] = kv_end;
+      for (int h = 0; h < num_kv_heads; ++h)
+        for (int p = 0; p < nparts; ++p)
+          items.push_back(PrefillItem{s, q_base + t, count, p0, p * pb, std::min(nblk, (p + 1) * pb),
+                                      kv_end, h, p, nparts == 1 ? 1 : 0, h * G, -1});
+    }
+    q_base += qlen;
+  }
+}
+
+// Persistent schedule over `ctas` CTAs: each item goes, in list order, to
+// the CTA with the least estimated work so far (cost ~ KV chunks x active
+// tiles, plus a constant per item; ties to the lowest CTA), and each CTA's
+// items are stored together, in list order: CTA b runs sched_items
+// [sched_offs[b], sched_offs[b + 1]). owner (optional) receives each item's CTA.
+void prefill_schedule(const std::vector<PrefillItem>& items, unsigned ctas, int block_size,
+                      int tile_tokens, std::vector<PrefillItem>& sched_items,
+                      std::vector<int32_t>& sched_offs, std::vector<int32_t>& owner) {
+  using Load = std::pair<int64_t, int32_t>;
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (unsigned b = 0; b < ctas; ++b) heap.push(Load{0, static_cast<int32_t>(b)});
+  owner.resize(items.size());
+  sched_offs.assign(ctas + 1, 0);
+  for (size_t i = 0; i < items.size(); ++i) {
+    const PrefillItem& it = items[i];
+    const int64_t span = std::max(0, std::min(it.block_end * block_size, it.kv_end) -
+                                         it.block_begin * block_size);
+    const int64_t cost = span * (it.q_count > tile_tokens ? 21 : 15) / 64 + 20;
+    const Load ld = heap.top();
+    heap.pop();
+    owner[i] = ld.second;
+    ++sched_offs[ld.second + 1];
+    heap.push(Load{ld.first + cost, ld.second});
+  }
+  for (unsigned b = 0; b < ctas; ++b) sched_offs[b + 1] += sched_offs[b];
+  sched_items.resize(items.size());
+  thread_local std::vector<int32_t> fill;
+  fill.assign(sched_offs.begin(), sched_offs.end() - 1);
+  for (size_t i = 0; i < items.size(); ++i) sched_items[fill[owner[i]]++] = items[i];
+}
+
+// The plan pa_prefill makes for the tcgen05 kernel, exposed for inspection
+// (pa_prefill_plan). Host-only: no CUDA call.
+pa_status_t prefill_plan(const int32_t* ctx_host, const int32_t* qlen_host, int B, int num_q_heads,
+                         int num_kv_heads, int block_size, int partition_tokens, int max_ctas,
+                         int32_t* items_out, int max_items, int* num_items, int* num_ctas) {
+  if (num_items == nullptr || num_ctas == nullptr)
+    return fail(PA_ERR_INVALID_ARG, "num_items and num_ctas are required");
+  if (B < 0 || (B > 0 && (ctx_host == nullptr || qlen_host == nullptr)))
+    return fail(PA_ERR_INVALID_ARG, "context_lens and query_lens (host) are required");
+  if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                num_q_heads, num_kv_heads);
+  PrefixInstance pinst;
+  if (!find_prefill_bf16(128, block_size, true, &pinst))
+    return fail(PA_ERR_UNSUPPORTED, "no tcgen05 prefill kernel for block_size=%d", block_size);
+  if (partition_tokens <= 0 || partition_tokens % block_size != 0)
+    return fail(PA_ERR_INVALID_ARG, "partition_tokens (%d) must be a positive multiple of block_size",
+                partition_tokens);
+  for (int s = 0; s < B; ++s)
+    if (qlen_host[s] < 0 || ctx_host[s] < qlen_host[s])
+      return fail(PA_ERR_INVALID_ARG, "sequence %d: query_len %d, context_len %d out of range", s,
+                  qlen_host[s], ctx_host[s]);
+  const int G = num_q_heads / num_kv_heads;
+  const int tile_tokens = std::max(1, pinst.rows / G);
+  thread_local std::vector<PrefillItem> items, sched_items;
+  thread_local std::vector<int32_t> sched_offs, owner;
+  bool any_split = false;
+  prefill_items(B, ctx_host, qlen_host, num_kv_heads, G, block_size, pinst.tiles * tile_tokens,
+                partition_tokens / block_size, items, nullptr, &any_split);
+  const size_t n = items.size();
+  const bool persistent = max_ctas > 0 && n > static_cast<size_t>(max_ctas);
+  *num_items = static_cast<int>(n);
+  *num_ctas = persistent ? max_ctas : static_cast<int>(n);
+  if (items_out == nullptr) return ok();
+  if (max_items < 0 || static_cast<size_t>(max_items) < n)
+    return fail(PA_ERR_INVALID_ARG, "max_items %d < %zu items", max_items, n);
+  const PrefillItem* list = items.data();
+  if (persistent) {
+    prefill_schedule(items, static_cast<unsigned>(max_ctas), block_size, tile_tokens, sched_items,
+                     sched_offs, owner);
+    list = sched_items.data();
+  }
+  int b = 0;
+  for (size_t i = 0; i < n; ++i) {
+    while (persistent && static_cast<size_t>(sched_offs[b + 1]) <= i) ++b;
+    const PrefillItem& it = list[i];
+    int32_t* row = items_out + 6 * i;
+    row[0] = it.seq;
+    row[1] = it.q_begin;
+    row[2] = it.q_count;
+    row[3] = it.kvh;
+    row[4] = it.part;
+    row[5] = persistent ? b : static_cast<int32_t>(i);
+  }
+  return ok();
+}
+
 pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const int32_t* qlen_host,
                         int total_q, int partition_tokens, void* workspace, size_t workspace_bytes) {
   // With no new tokens q and out are never touched and may be NULL; every
@@ -880,37 +998,16 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
   thread_local std::vector<int32_t> lens;
   thread_local std::vector<PrefillItem> items;
   lens.assign(total_q, 0);
-  items.clear();
   bool any_split = false;
-  int q_base = 0;
-  // Items in sequence order, each sequence's query tiles last-first (the
-  // longest spans first), so that the work handed out last is short.
-  for (int s = 0; s < B; ++s) {
-    const int qlen = qlen_host[s], ctx = ctx_host[s];
-    for (int t = qlen > 0 ? (qlen - 1) / tq * tq : -1; t >= 0; t -= tq) {
-      const int count = std::min(tq, qlen - t);
-      const int p0 = ctx - qlen + t;
-      const int kv_end = p0 + count;  // last position + 1
-      const int nblk = (kv_end + r.block_size - 1) / r.block_size;
-      const int nparts = (nblk + pb - 1) / pb;
-      any_split = any_split || nparts > 1;
-      for (int i = 0; i < count; ++i) lens[q_base + t + i] = kv_end;
-      for (int h = 0; h < r.num_kv_heads; ++h)
-        for (int p = 0; p < nparts; ++p)
-          items.push_back(PrefillItem{s, q_base + t, count, p0, p * pb, std::min(nblk, (p + 1) * pb),
-                                      kv_end, h, p, nparts == 1 ? 1 : 0, h * G, -1});
-    }
-    q_base += qlen;
-  }
+  prefill_items(B, ctx_host, qlen_host, r.num_kv_heads, G, r.block_size, tq, pb, items, &lens,
+                &any_split);
   if (items.size() > L.max_items) return fail(PA_ERR_INVALID_ARG, "too many prefill items");
   st = prepare_kernel(pinst.kernel, pinst.smem);
   if (st != PA_OK) return st;
 
   // The tcgen05 kernel runs persistently when there are more items than
-  // resident CTAs: each item goes, in list order, to the CTA with the least
-  // estimated work so far (cost ~ KV chunks x active tiles, plus a constant
-  // per item), and each CTA's items are stored together. A CTA starts the
-  // next item's loads while it finishes the current one.
+  // resident CTAs (prefill_schedule); a CTA starts the next item's loads
+  // while it finishes the current one.
   thread_local std::vector<PrefillItem> sched_items;
   thread_local std::vector<int32_t> sched_offs, owner;
   unsigned grid = static_cast<unsigned>(items.size());
@@ -931,28 +1028,8 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
     if (items.size() > ctas) {
       persistent = true;
       grid = static_cast<unsigned>(ctas);
-      const int tile_tokens = std::max(1, pinst.rows / G);
-      using Load = std::pair<int64_t, int32_t>;
-      std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
-      for (unsigned b = 0; b < grid; ++b) heap.push(Load{0, static_cast<int32_t>(b)});
-      owner.resize(items.size());
-      sched_offs.assign(grid + 1, 0);
-      for (size_t i = 0; i < items.size(); ++i) {
-        const PrefillItem& it = items[i];
-        const int64_t span = std::max(0, std::min(it.block_end * r.block_size, it.kv_end) -
-                                             it.block_begin * r.block_size);
-        const int64_t cost = span * (it.q_count > tile_tokens ? 21 : 15) / 64 + 20;
-        Load ld = heap.top();
-        heap.pop();
-        owner[i] = ld.second;
-        ++sched_offs[ld.second + 1];
-        heap.push(Load{ld.first + cost, ld.second});
-      }
-      for (unsigned b = 0; b < grid; ++b) sched_offs[b + 1] += sched_offs[b];
-      sched_items.resize(items.size());
-      thread_local std::vector<int32_t> fill;
-      fill.assign(sched_offs.begin(), sched_offs.end() - 1);
-      for (size_t i = 0; i < items.size(); ++i) sched_items[fill[owner[i]]++] = items[i];
+      prefill_schedule(items, grid, r.block_size, std::max(1, pinst.rows / G), sched_items,
+                       sched_offs, owner);
       upload_items = sched_items.data();
     }
   }
@@ -1215,6 +1292,14 @@ pa_status_t pa_prefill(const void* q, const void* k_pool, const void* v_pool,
               static_cast<cudaStream_t>(stream)};
   return run_prefill(r, context_lens, query_lens, total_q, partition_tokens, workspace,
                      workspace_bytes);
+}
+
+pa_status_t pa_prefill_plan(const int32_t* context_lens, const int32_t* query_lens, int num_seqs,
+                            int num_q_heads, int num_kv_heads, int block_size, int partition_tokens,
+                            int max_ctas, int32_t* items_out, int max_items, int* num_items,
+                            int* num_ctas) {
+  return prefill_plan(context_lens, query_lens, num_seqs, num_q_heads, num_kv_heads, block_size,
+                      partition_tokens, max_ctas, items_out, max_items, num_items, num_ctas);
 }
 
 }  // extern "C"
