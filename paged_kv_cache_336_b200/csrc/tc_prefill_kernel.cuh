@@ -31,11 +31,15 @@
 //     past the row's position, and keeps a reference max m: P = 2^(x - m)
 //     is written back as packed bf16 over the logits it came from (the A
 //     operand of P V); m moves only when the chunk's max exceeds it by more
-//     than 2^8, and then O (in TMEM) and l are scaled by 2^(m_old - m_new).
-//     The unmasked path runs on packed fp32 pairs (f32x2 FMA/add) and a
-//     three-input max. The softmax is bound by issue slots, not by MUFU:
-//     moving a share of the exponentials to an FMA-pipe polynomial measured
-//     slower at every share tried (1/4, 3/8, 1/2).
+//     than 8 (log2 units, so P <= 2^8), and then O (in TMEM) and l are scaled
+//     by 2^(m_old - m_new). The unmasked path runs on packed fp32 pairs
+//     (f32x2 FMA/add) and a three-input max. The softmax is bound by each
+//     warp's own instruction latency (two softmax warps per SM
+//     sub-partition), not by MUFU: moving a share of the exponentials to an
+//     FMA-pipe polynomial measured slower at every share tried (1/4, 3/8,
+//     1/2). After an item's last chunk the same warps write its output: a
+//     full tile of final rows through a 128-byte-swizzled staging buffer and
+//     one TMA store per 64 columns, other rows with plain stores.
 // TMEM per tile: two 64-column S / P buffers (chunk parity) and head_dim O
 // columns; 512 columns for the CTA. The tensor core reads its shared-memory
 // operands at about 128 bytes per clock per SM, so P stays out of shared
