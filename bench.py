@@ -194,19 +194,24 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def kernel_source_hash() -> str:
+DECODE_SOURCES = ("decode_kernel.cuh", "device_common.cuh")
+PREFILL_SOURCES = ("tc_prefill_kernel.cuh", "prefill_kernel.cuh", "device_common.cuh")
+
+
+def kernel_source_hash(names=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_336_b200", "csrc")
-    for name in ("decode_kernel.cuh", "device_common.cuh"):
+    for name in names:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.txt")
+def profiled_traffic(workload: str, kind: str = "decode", sources=DECODE_SOURCES):
+    """DRAM bytes per launch from the committed ncu summary
+    profiles/<kind>_<workload>_traffic.txt, if it was taken on the current
+    kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kind}_{workload}_traffic.txt")
     try:
         kv = {}
         with open(path) as f:
@@ -214,7 +219,7 @@ def profiled_traffic(workload: str):
                 if ":" in line and not line.lstrip().startswith("#"):
                     k, v = line.split(":", 1)
                     kv[k.strip()] = v.strip()
-        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash(sources):
             return None
         return int(kv["dram_bytes_per_launch"])
     except Exception:
@@ -662,6 +667,8 @@ def run_prefill_bench(args, device_index):
                        "kernel": os.environ.get("PAGEDKV_PREFILL_KERNEL", "tcgen05")},
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                          "peak_kind": kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                         "traffic": (profiled_traffic("b16", "prefill", PREFILL_SOURCES)
+                                     if (B, prior, chunk, part) == (16, 1024, 1024, 2048) else None),
                          "kv_bytes_per_call": kv_bytes,
                          "kv_GBs": round(kv_bytes / (ms * 1e-3) / 1e9, 1)}}
 
