@@ -668,7 +668,9 @@ def run_prefill_bench(args, device_index):
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                          "peak_kind": kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
                          "traffic": (profiled_traffic("b16", "prefill", PREFILL_SOURCES)
-                                     if (B, prior, chunk, part) == (16, 1024, 1024, 2048) else None),
+                                     if (B, prior, chunk, part) == (16, 1024, 1024, 2048)
+                                     and os.environ.get("PAGEDKV_PREFILL_KERNEL") != "mma_sync"
+                                     else None),
                          "kv_bytes_per_call": kv_bytes,
                          "kv_GBs": round(kv_bytes / (ms * 1e-3) / 1e9, 1)}}
 
