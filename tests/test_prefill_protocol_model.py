@@ -5,17 +5,21 @@ Each CTA role is a generator that follows the kernel's loops and running
 counts: the producer (K/V ring, partial-chunk V clears), the two MMA
 issuers (Q copies, S and P V MMAs, commits) and the two tiles' softmax
 warps (P, epilogue). Barriers count arrivals and completed phases as
-mbarriers do. TMA copies and tensor-core work finish after random delays;
-the tensor pipe runs MMAs in issue order, and a commit arrives once its
-thread's earlier MMAs are done.
+mbarriers do. TMA copies and tensor-core work finish after random delays.
+MMAs are ordered only where tcgen05 orders them: those accumulating into the
+same TMEM region run in issue order; others may overlap or overtake one
+another. A commit arrives once all of its thread's earlier MMAs are done.
 
 A kernel wait only knows a parity, so it is right only while the barrier
 has completed the phase it means or the one before it. The model checks that
 at every poll (no wait early by a phase, none lapped), that no role
-deadlocks, and that Q and O are never overwritten while in use. Random item
-lists mix idle second tiles, empty spans, one-chunk items and partial last
-chunks. The last tests plant each guard's absence and expect the model to
-catch it."""
+deadlocks, and that no buffer is overwritten while in use: a ring slot is
+refilled only after every MMA reading its last use has finished; an S MMA
+starts only after the softmax is done with the buffer's previous chunk and
+that chunk's P V has read its P; Q, O and a partial chunk's cleared V rows
+likewise. Random item lists mix idle second tiles, empty spans, one-chunk
+items and partial last chunks. The last tests plant each guard's absence and
+expect the model to catch it."""
 
 import heapq
 import random
@@ -35,7 +39,7 @@ class Bar:
             self.pending = self.count
 
 
-def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True):
+def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True, s_waits_p_free=True):
     """items: (chunks, active tiles, partial last chunk) per item, in one
     CTA's order. Returns None, or a description of the first fault."""
     rnd = random.Random(seed)
@@ -53,19 +57,28 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True):
 
     now = [0]
     events, seq = [], [0]
-    pipe_end, last_of = [0], {}
+    last_of = {}
     s_end, o_read = {}, {}
+    slot_read_end = {}                 # ring slot -> end of the last MMA reading it
+    sm_done, pv_end = {}, {}           # (tile, chunk) -> softmax finished / its P V ended
+    tail_cleared = {}                  # ring index of a partial chunk's V -> time cleared
     faults = []
+
+    def reads_slot(slot, end):
+        slot_read_end[slot] = max(slot_read_end.get(slot, 0), end)
 
     def later(t, bar):
         seq[0] += 1
         heapq.heappush(events, (t, seq[0], bar))
 
-    def mma(tid, dur):
-        start = max(pipe_end[0], now[0])
-        pipe_end[0] = start + dur
-        last_of[tid] = pipe_end[0]
-        return start, pipe_end[0]
+    acc_end = {}
+
+    def mma(tid, dur, acc):
+        start = max(acc_end.get(acc, 0), now[0]) + rnd.randint(0, 300)
+        end = start + dur
+        acc_end[acc] = end
+        last_of[tid] = max(last_of.get(tid, 0), end)
+        return start, end
 
     def commit(tid, bar):
         later(max(last_of.get(tid, 0), now[0]) + 1, bar)
@@ -82,6 +95,8 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True):
                 gi = g + i
                 if gi >= nslot:
                     yield wait(kv_empty[gi % nslot], gi // nslot - 1)
+                if now[0] < slot_read_end.get(gi % nslot, 0):
+                    faults.append(f"slot {gi % nslot} refilled while an MMA still reads it")
                 later(now[0] + rnd.randint(50, 3000), kv_full[gi % nslot])
                 yield ("delay", rnd.randint(5, 60))
             if tail:
@@ -90,6 +105,7 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True):
                 if tail_guard and prev_tail >= 0 and gi - prev_tail < nslot:
                     yield wait(kv_empty[prev_tail % nslot], prev_tail // nslot)
                 yield ("delay", 100)
+                tail_cleared[gi] = now[0]
                 v_tail.arrive()
                 prev_tail = gi
             g += 2 * nch
@@ -126,10 +142,13 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True):
             def issue_s(j):
                 gi, c = g + 2 * j, cb + j
                 yield wait(kv_full[gi % nslot], gi // nslot)
-                if c >= 2:
+                if c >= 2 and s_waits_p_free:
                     yield wait(p_free[2 * t + (c & 1)], (c >> 1) - 1)
-                _, end = mma(tid, rnd.randint(200, 500))
-                s_end[t] = end
+                start, end = mma(tid, rnd.randint(200, 500), ("S", t, c & 1))
+                if c >= 2 and start < max(sm_done.get((t, c - 2), 1 << 60), pv_end.get((t, c - 2), 1 << 60)):
+                    faults.append(f"tile {t}: S({c}) overwrote a buffer still in use for chunk {c - 2}")
+                reads_slot(gi % nslot, end)
+                s_end[t] = max(s_end.get(t, 0), end)
                 commit(tid, s_full[2 * t + (c & 1)])
                 commit(tid, kv_empty[gi % nslot])
 
@@ -158,9 +177,13 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True):
                 yield wait(p_full[2 * t + (c & 1)], c >> 1)
                 if j == 0 and nt > 0:
                     yield wait(o_empty[t], nt - 1)
-                start, _ = mma(tid, rnd.randint(150, 400))
+                start, end = mma(tid, rnd.randint(150, 400), ("O", t))
                 if j == 0 and nt > 0 and start < o_read[(t, nt - 1)]:
                     faults.append(f"tile {t}: O overwritten before the epilogue read it")
+                if tail and j == nch - 1 and start < tail_cleared.get(gi, 1 << 60):
+                    faults.append(f"tile {t}: P V read a partial chunk's V before it was cleared")
+                pv_end[(t, c)] = end
+                reads_slot(gi % nslot, end)
                 commit(tid, p_free[2 * t + (c & 1)])
                 commit(tid, kv_empty[gi % nslot])
             commit(tid, o_last[t])
@@ -184,7 +207,10 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True):
                 yield ("delay", rnd.randint(300, 1600))
                 if j >= 1 and rnd.random() < 0.1:  # a rescale of O
                     yield wait(p_free[2 * t + ((c - 1) & 1)], (c - 1) >> 1)
+                    if now[0] < pv_end.get((t, c - 1), 1 << 60):
+                        faults.append(f"tile {t}: O rescaled while P V({c - 1}) still accumulates")
                     yield ("delay", 100)
+                sm_done[(t, c)] = now[0]
                 for _ in range(4):
                     p_full[2 * t + (c & 1)].arrive()
             if nch > 0:
@@ -282,3 +308,8 @@ def test_model_catches_a_missing_tail_guard():
 def test_model_catches_a_missing_q_free_wait():
     fault = _first_fault(q_free_wait=False)
     assert fault is not None and "Q overwritten" in fault
+
+
+def test_model_catches_an_s_mma_that_skips_the_p_free_wait():
+    fault = _first_fault(s_waits_p_free=False)
+    assert fault is not None and "overwrote a buffer" in fault
