@@ -7,22 +7,29 @@ manager's slot/copy-on-write decisions for one appended token per sequence
 the KV-append scatter, and split-context decode attention (partition kernel
 plus log-sum-exp merge) over the paged cache.
 
-Default workload (N=1): MHA decode, 7B-style: batch 64, 32 query heads = 32
-KV heads, head_dim 128, bf16, block size 16, context lengths uniform in
-[1, 2048], pool 16384 blocks placed by a seeded shuffle, values N(0, 1).
-The per-step inputs (queries, new K/V, slots, block tables, lengths) of R
-consecutive decode steps are made ahead of time and cycled; every step does
-the full work of a real decode step at its context lengths. The KV bytes a
-step reads (~1 GB) exceed the 126 MB L2, so no flush is needed.
+Headline workload (N=1 default): long-context split decode: batch 8, context
+131072 tokens each, 64 query heads over 8 KV heads, head_dim 128, bf16,
+block size 16, 512-token partitions, pool 10% larger than needed and placed
+by a seeded shuffle, values N(0, 1); the largest single-GPU configuration
+(~4.3 GB of KV read per step). The per-step inputs (queries, new K/V, slots,
+block tables, lengths) of R consecutive decode steps are made ahead of time
+and cycled; every step does the full work of a real decode step at its
+context lengths. The KV bytes a step reads exceed the 126 MB L2, so no
+flush is needed.
 
 value      = algorithmic bytes of the step (valid K/V tokens + q + out + block
              table entries + lengths + append + copies) / device time, GB/s,
-             summed over ranks, time = max over ranks (CUDA events).
+             summed over ranks, time = max over ranks (CUDA events). Timed in
+             repeats of --steps steps until --min-seconds of device time;
+             value is the median over repeats.
 roofline   = the decode call alone (partition kernel + merge), its algorithmic
              bytes / its event-timed duration, against the measured HBM peak.
+configs    = (one GPU) the same numbers for the other configurations: block
+             size 32, MHA batch 64, GQA batch 256, and both prefix-sharing
+             workloads on the split route and on the shared-prefix route.
 e2e        = the same metric through the public API from pinned host buffers:
              per step the host block manager step, H2D of the step's inputs,
-             the kernels, D2H of the output, stream synchronisation.
+             the kernels, D2H of the output.
 cpu_baseline / --impl reference: the CPU oracle (float64 NumPy) timed on a
              bounded sample of the same workload on the host cores.
 
@@ -142,59 +149,107 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def gpu_uuid(device_index: int) -> str | None:
+    """The GPU's UUID in NVML / nvidia-smi form ("GPU-..."), which names the
+    physical device whatever CUDA_VISIBLE_DEVICES says."""
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(device_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    """SM clock and clock-event-reason samples while a timed region runs
+    (read-only NVML queries from a background thread; nvidia-smi if NVML is
+    not importable). The device is found by UUID, so the samples come from
+    the GPU this process runs on."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, device_index: int):
-        self.device_index = device_index
-        self.proc = None
-        # raw samples go to PAGEDKV_CLOCKS_DIR (default: the system temp dir);
-        # the JSON line carries their summary
-        out_dir = os.environ.get("PAGEDKV_CLOCKS_DIR") or tempfile.gettempdir()
-        self.path = os.path.join(out_dir, f"clocks_rank{device_index}.csv")
+    def __init__(self, device_index: int, period_s: float = 0.05):
+        self.uuid = gpu_uuid(device_index)
+        self.period_s = period_s
+        self.samples = []     # (sm_mhz, sm_max_mhz, reasons bitmask, power W)
+        self._thread = None
+        self._stop = None
+        self._proc = None
+
+    def _nvml_loop(self, handle, nvml):
+        while True:
+            try:
+                sm = nvml.nvmlDeviceGetClockInfo(handle, nvml.NVML_CLOCK_SM)
+                mx = nvml.nvmlDeviceGetMaxClockInfo(handle, nvml.NVML_CLOCK_SM)
+                rs = nvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                pw = nvml.nvmlDeviceGetPowerUsage(handle) / 1000.0
+                self.samples.append((float(sm), float(mx), int(rs), pw))
+            except Exception:
+                pass
+            if self._stop.wait(self.period_s):
+                return
 
     def start(self):
+        import threading
+        self.samples = []
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=self.fh, stderr=subprocess.DEVNULL)
+            import pynvml as nvml
+            nvml.nvmlInit()
+            handle = nvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._nvml_loop, args=(handle, nvml), daemon=True)
+            self._thread.start()
+            return
         except Exception:
-            self.proc = None
+            self._thread = None
+        if self.uuid is None:
+            return
+        try:
+            fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,power.draw")
+            self._fh = tempfile.TemporaryFile(mode="w+")
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={fields}",
+                 "--format=csv,noheader,nounits", "-lms", str(int(self.period_s * 1000))],
+                stdout=self._fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self._proc = None
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+            self._thread = None
+        elif self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except Exception:
+                self._proc.kill()
+            self._fh.seek(0)
+            for line in self._fh:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        if not rows:
+                try:
+                    self.samples.append((float(parts[0]), float(parts[1]), int(parts[2], 16),
+                                         float(parts[3])))
+                except Exception:
+                    pass
+            self._fh.close()
+            self._proc = None
+        if not self.samples:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({name for x in self.samples for bit, name in self.REASONS.items()
+                          if x[2] & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_median": round(statistics.median(x[3] for x in self.samples), 1),
+                "source": "nvml" if self._stop is not None else "nvidia-smi",
+                "gpu": self.uuid}
 
 
 DECODE_SOURCES = ("decode_kernel.cuh", "device_common.cuh")
+PREFIX_SOURCES = ("prefix_kernel.cuh", "decode_kernel.cuh", "device_common.cuh")
 PREFILL_SOURCES = ("tc_prefill_kernel.cuh", "prefill_kernel.cuh", "device_common.cuh")
 
 
@@ -207,10 +262,15 @@ def kernel_source_hash(names=DECODE_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, kind: str = "decode", sources=DECODE_SOURCES):
-    """DRAM bytes per launch from the committed ncu summary
-    profiles/<kind>_<workload>_traffic.txt, if it was taken on the current
-    kernel source; else None."""
+def profiled_traffic(workload: str, kind: str = "decode", sources=None, mode: str = "split"):
+    """DRAM bytes per call from the committed ncu summary
+    profiles/<kind>_<workload>_traffic.txt (decode calls of another route:
+    <route>_<workload>_traffic.txt), if it was taken on the current kernel
+    source; else None."""
+    if kind == "decode" and mode != "split":
+        kind = mode
+    if sources is None:
+        sources = PREFIX_SOURCES if kind == "shared_prefix" else DECODE_SOURCES
     path = os.path.join(ROOT, "profiles", f"{kind}_{workload}_traffic.txt")
     try:
         kv = {}
@@ -333,117 +393,211 @@ class DeviceStep:
         return st
 
 
-def run_ours(args, rank, world, device_index):
+CONFIG_LABELS = {
+    "long16": "long-context split decode (config 5), block 16",
+    "long32": "long-context split decode (config 5), block 32",
+    "mha": "MHA decode, 7B-style (config 2)",
+    "gqa": "GQA decode, 8B-style (config 3)",
+    "prefix": "prefix sharing / parallel sampling (config 4, literal: 4000-token prompts)",
+    "prefix_cow": "prefix sharing copy-on-write step (config 4: 4008-token prompts, 120 copies)",
+    "tiny": "tiny fp32 paged decode (config 1)",
+}
+EXTRA_CONFIGS = ("long32", "mha", "gqa", "prefix", "prefix_cow")
+KERNEL_LABELS = {
+    "split": "pa_decode_split (paged_decode_kernel + lse_merge_kernel)",
+    "whole": "pa_decode (paged_decode_kernel)",
+    "shared_prefix": "pa_decode_shared_prefix (prefix_decode_kernel + paged_decode_kernel "
+                     "+ lse_merge_kernel)",
+    "window": "pa_decode_split_window (paged_decode_kernel + lse_merge_kernel)",
+}
+
+
+def timed_repeats(ds, steps: int, first_index: int, min_ms: float, world: int, device,
+                  max_repeats: int = 10_000):
+    """Times `steps` steps at a time, each repeat bracketed by a barrier and
+    a device synchronisation, until the repeats' max-over-ranks time reaches
+    min_ms. Every rank stops after the same repeat (the stop rule reads the
+    reduced time). Returns the per-repeat records, the decode call durations
+    (us, CUDA events on the launching stream), launches and the next index."""
     import torch
     import torch.distributed as dist
-    from paged_kv_cache_336_b200 import binding
+    reps, calls = [], []
+    launches = 0
+    i = first_index
+    total = 0.0
+    while True:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nbytes = dbytes = ubytes = 0
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record()
+        for k in range(steps):
+            st = ds.run(i, evs[k])
+            i += 1
+            nbytes += st["step_bytes"]
+            dbytes += st["decode_bytes"]
+            ubytes += st["unique_bytes"]
+            launches += ds.launches(st)
+        t1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms = t0.elapsed_time(t1)
+        call_us = [a.elapsed_time(b) * 1e3 for a, b in evs]
+        ms_max, all_bytes, all_tokens = reduce_over_ranks(ms, nbytes, steps * ds.B, device)
+        reps.append({"ms": ms_max, "bytes": all_bytes, "tokens": all_tokens,
+                     "decode_bytes": dbytes, "unique_bytes": ubytes, "decode_us": sum(call_us)})
+        calls.extend(call_us)
+        total += ms_max
+        if total >= min_ms or len(reps) >= max_repeats:
+            return reps, calls, launches, i
 
-    device = torch.device("cuda", device_index)
-    torch.cuda.set_device(device)
-    w = make_workload(args.workload, rank, args.batch)
-    R = max(1, min(args.states, args.steps + args.warmup)) if args.workload != "prefix_cow" else 1
-    ds = DeviceStep(w, R, args.partition_tokens, device, mode=args.decode_mode, window=args.window)
 
+def summarize(ds, reps, calls, steps, world, workload_key, mode, peak, peak_kind, clock_info):
+    """One configuration's numbers: step throughput (median over repeats,
+    with p10/p90), the decode call's roofline and the clocks seen."""
+    w = ds.w
+    gbs = [r["bytes"] / (r["ms"] * 1e-3) / 1e9 for r in reps]
+    ms_step = [r["ms"] / steps for r in reps]
+    tok = [r["tokens"] / (r["ms"] * 1e-3) for r in reps]
+    dbytes = sum(r["decode_bytes"] for r in reps)
+    ubytes = sum(r["unique_bytes"] for r in reps)
+    dus = sum(r["decode_us"] for r in reps)
+    n_calls = len(calls)
+    achieved = dbytes / (dus * 1e-6) / 1e9
+    unique = ubytes / (dus * 1e-6) / 1e9
+    pct = lambda xs, q: round(float(np.percentile(xs, q)), 2)
+    roof = {
+        "bound": "hbm",
+        "kernel": KERNEL_LABELS[mode],
+        "achieved": round(achieved, 2),
+        "peak": peak,
+        "peak_kind": peak_kind,
+        "unit": "GB/s",
+        "frac": round(achieved / peak, 4),
+        "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
+        "traffic": profiled_traffic(workload_key, mode=mode),
+        "algorithmic_bytes_per_launch": int(dbytes / n_calls),
+        "avg_launch_us": round(dus / n_calls, 2),
+        "launch_us_p10_p50_p90": [pct(calls, 10), pct(calls, 50), pct(calls, 90)],
+        # bytes the call must read at least (shared prefixes once); equal to the
+        # algorithmic bytes unless blocks are shared
+        "unique_bytes_per_launch": int(ubytes / n_calls),
+        "unique_achieved": round(unique, 2),
+        "unique_frac": round(unique / peak, 4),
+    }
+    return {
+        "workload": workload_label(w),
+        "config": CONFIG_LABELS.get(workload_key, workload_key),
+        "value": round(statistics.median(gbs), 2),
+        "unit": "GB/s",
+        "value_p10_p90": [pct(gbs, 10), pct(gbs, 90)],
+        "ms_per_step": round(statistics.median(ms_step), 5),
+        "repeats": len(reps),
+        "steps_per_repeat": steps,
+        "timed_ms": round(sum(r["ms"] for r in reps), 2),
+        "decode_tokens_per_s": round(statistics.median(tok), 1),
+        "mean_context": round(float(np.mean([s["ctx_np"].mean() for s in ds.states])), 1),
+        "copies_per_step": round(float(np.mean([s["n_pairs"] for s in ds.states])), 2),
+        "roofline": roof,
+        "clocks": clock_info,
+    }
+
+
+def bench_config(args, workload_key, mode, rank, world, device, device_index, min_ms,
+                 keep=False):
+    """Builds one workload on the device, warms up, times it; returns
+    (summary, DeviceStep if keep else None, launches)."""
+    import torch
+    w = make_workload(workload_key, rank, args.batch)
+    R = max(1, min(args.states, args.steps + args.warmup)) if workload_key != "prefix_cow" else 1
+    ds = DeviceStep(w, R, args.partition_tokens, device, mode=mode, window=args.window)
     for i in range(args.warmup):
         ds.run(i)
     torch.cuda.synchronize()
-
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(device_index)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     clocks.start()
-    t0.record()
-    total_bytes = 0
-    decode_bytes_sum = 0
-    unique_bytes_sum = 0
-    launches = 0
-    for i in range(args.steps):
-        st = ds.run(args.warmup + i, evs[i])
-        total_bytes += st["step_bytes"]
-        decode_bytes_sum += st["decode_bytes"]
-        unique_bytes_sum += st["unique_bytes"]
-        launches += ds.launches(st)
-    t1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    reps, calls, launches, _ = timed_repeats(ds, args.steps, args.warmup, min_ms, world, device)
     clock_info = clocks.stop()
-    ms = t0.elapsed_time(t1)
-    call_us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
-    decode_ms = float(call_us.sum()) / 1e3
-
-    # max time over ranks, bytes summed over ranks
-    ms_max, all_bytes, all_tokens = reduce_over_ranks(ms, total_bytes, args.steps * ds.B, device)
-
-    gbs = all_bytes / (ms_max * 1e-3) / 1e9
-    tok_s = all_tokens / (ms_max * 1e-3)
-    decode_gbs = decode_bytes_sum / (decode_ms * 1e-3) / 1e9
-    unique_gbs = unique_bytes_sum / (decode_ms * 1e-3) / 1e9
     peak, peak_kind = hbm_peak()
+    res = summarize(ds, reps, calls, args.steps, world, workload_key, mode, peak, peak_kind,
+                    clock_info)
+    if not keep:
+        del ds
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        ds = None
+    return res, ds, launches
 
+
+def run_ours(args, rank, world, device_index):
+    import torch
+    device = torch.device("cuda", device_index)
+    torch.cuda.set_device(device)
+    head, ds, launches = bench_config(args, args.workload, args.decode_mode, rank, world, device,
+                                      device_index, args.min_seconds * 1e3, keep=True)
     # ---- end to end through the public API (host buffers, pinned) ----------------
-    e2e = run_e2e(args, ds, rank, world, device)
+    e2e = run_e2e(args, ds, rank, world, device) if args.e2e_steps > 0 else None
+    w = ds.w
+    B = ds.B
+    del ds
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    # ---- the other configurations, each with its own roofline ----------------------
+    extras = {}
+    if args.configs == "all" and world == 1:
+        for key in EXTRA_CONFIGS:
+            if key == args.workload:
+                continue
+            modes = ["split", "shared_prefix"] if key.startswith("prefix") else ["split"]
+            for mode in modes:
+                r, _, n = bench_config(args, key, mode, rank, world, device, device_index,
+                                       args.extra_min_seconds * 1e3)
+                extras[key if mode == "split" else f"{key}/shared_prefix"] = r
+                launches += n
 
     result = None
     if rank == 0:
-        kernel_label = {
-            "split": "pa_decode_split (paged_decode_kernel + lse_merge_kernel)",
-            "whole": "pa_decode (paged_decode_kernel)",
-            "shared_prefix": "pa_decode_shared_prefix (prefix_decode_kernel + paged_decode_kernel "
-                             "+ lse_merge_kernel)",
-            "window": f"pa_decode_split_window (window {args.window}; paged_decode_kernel + "
-                      "lse_merge_kernel)"}[args.decode_mode]
         result = {
             "metric": METRIC,
-            "value": round(gbs, 2),
+            "value": head["value"],
             "unit": "GB/s",
             "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup,
-            "ms_per_step": round(ms_max / args.steps, 5),
+            "ms_per_step": head["ms_per_step"],
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": w.dtype,
             "data": "synthetic (seeded N(0,1) values, seeded shuffled block placement)",
             "config": {
-                "workload": workload_label(w),
-                "global_batch": ds.B * world,
-                "context_lens": ("uniform [1, 2048]" if w.name == "mha" else "see workload"),
-                "mean_context": round(float(np.mean([s["ctx_np"].mean() for s in ds.states])), 1),
+                "workload": head["workload"],
+                "name": head["config"],
+                "global_batch": B * world,
+                "mean_context": head["mean_context"],
                 "partition_tokens": args.partition_tokens,
-                "step": "bm slots/CoW (host, precomputed) + copy_blocks + kv_append + " + kernel_label,
-                "decode_states_cycled": len(ds.states),
+                "step": "bm slots/CoW (host, precomputed) + copy_blocks + kv_append + "
+                        + KERNEL_LABELS[args.decode_mode],
+                "decode_states_cycled": min(args.states, args.steps + args.warmup),
+                "timing": (f"{head['repeats']} repeats of {args.steps} steps (each bracketed by "
+                           f"barrier + synchronize, max over ranks) until >= {args.min_seconds} s "
+                           "of device time; value and ms_per_step are medians over repeats"),
                 "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                 "parallelism": f"independent batch per GPU x{world}",
             },
-            "decode_tokens_per_s": round(tok_s, 1),
-            "roofline": {
-                "bound": "hbm",
-                "kernel": kernel_label,
-                "achieved": round(decode_gbs, 2),
-                "peak": peak,
-                "peak_kind": peak_kind,
-                "unit": "GB/s",
-                "frac": round(decode_gbs / peak, 4),
-                "frac_of_8TBs_spec": round(decode_gbs / 8000.0, 4),
-                "traffic": profiled_traffic(args.workload),
-                "algorithmic_bytes_per_launch": int(decode_bytes_sum / args.steps),
-                "avg_launch_us": round(decode_ms / args.steps * 1e3, 2),
-                "launch_us_p10_p50_p90": [round(float(np.percentile(call_us, q)), 2) for q in (10, 50, 90)],
-                # bytes the call must read at least (shared prefixes once); equal to the
-                # algorithmic bytes unless blocks are shared
-                "unique_bytes_per_launch": int(unique_bytes_sum / args.steps),
-                "unique_achieved": round(unique_gbs, 2),
-                "unique_frac": round(unique_gbs / peak, 4),
-            },
+            "value_p10_p90": head["value_p10_p90"],
+            "repeats": head["repeats"],
+            "decode_tokens_per_s": head["decode_tokens_per_s"],
+            "roofline": head["roofline"],
             "e2e": e2e,
             "gpu_launches": launches,
-            "clocks": clock_info,
+            "clocks": head["clocks"],
+            "configs": extras,
         }
     return result
 
@@ -459,11 +613,21 @@ def run_e2e(args, ds, rank, world, device):
     import torch.distributed as dist
     b = ds.binding
     w = ds.w
-    # the configured step count is split between the two measurements, so the
-    # sequences grow by the same number of tokens as the workload tables allow
-    steps = max(3, min(args.e2e_steps, args.steps) // 2)
+    # Every e2e step appends one token to each sequence: both measurements
+    # together must fit the tables' room and the free blocks, so the step
+    # counts are scaled down (and reported) where the workload is too tight.
     seqs = np.ascontiguousarray(np.asarray(w.step_seqs or w.decode_seqs, dtype=np.int64))
     n = int(seqs.shape[0])
+    piped_steps = max(3, int(args.e2e_steps))
+    sync_steps = max(3, min(64, piped_steps // 4))
+    bs = w.block_size
+    room = min(ds.bm.max_blocks_per_seq * bs - ds.bm.context_len(int(x)) for x in seqs) - 1
+    free = ds.bm.num_free()
+    fits = lambda t: t <= room and n * (t // bs + 2) <= free
+    while not fits(piped_steps + sync_steps) and piped_steps > 3:
+        piped_steps = max(3, piped_steps * 3 // 4)
+        sync_steps = max(3, min(sync_steps, piped_steps // 4))
+    steps = piped_steps
     ring = min(steps, 8)
     hq = [ds.states[i % len(ds.states)]["q"][:n].cpu().pin_memory() for i in range(ring)]
     hk, hv = [], []
@@ -485,6 +649,7 @@ def run_e2e(args, ds, rank, world, device):
     def timed(pipelined: bool):
         # bookkeeping stays out of the timed loop: every step appends one token
         # to each sequence, so step i decodes lengths ctx0 + i + 1
+        steps = piped_steps if pipelined else sync_steps
         ctx0 = np.array([ds.bm.context_len(int(x)) for x in seqs], dtype=np.int64)
         ncows = []
         if world > 1:
@@ -510,13 +675,15 @@ def run_e2e(args, ds, rank, world, device):
     g, ms, h2d, d2h = timed(True)
     return {"value": round(g, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "steps": steps, "ms_per_step": round(ms, 4),
+            "steps": piped_steps, "ms_per_step": round(ms, 4),
+            "timing": "host wall clock (perf_counter) from a synchronised device to the "
+                      "synchronisation after the last step",
             "path": "pa_decode_step (C ABI) per step: host block manager step + pinned H2D "
                     "of the step's inputs + copies/append/split decode + D2H out; two staging "
                     "sets alternated, uploads and downloads on their own streams overlapping the "
                     "neighbouring steps' kernels, one synchronisation at the end",
             "one_step_at_a_time": {"value": round(g_sync, 2), "unit": "GB/s",
-                                   "ms_per_step": round(ms_sync, 4),
+                                   "ms_per_step": round(ms_sync, 4), "steps": sync_steps,
                                    "path": "the same call with a stream synchronisation after "
                                            "every step"}}
 
@@ -557,8 +724,7 @@ def time_oracle(w, budget_s: float, seed: int = 0, threads: int = 1):
             q = workloads.draw_normal((1, w.num_q_heads, D), w.dtype, w.seed * 7 + 3 + int(idx)).double().numpy()
             table = np.arange(nb)[None, :]
             t0 = time.perf_counter()
-            for h in range(w.num_q_heads):
-                oracle.paged_decode_one(q, kp, vp, table, [ctx], w.scale, 0, h)
+            oracle.paged_decode(q, kp, vp, table, [ctx], w.scale)
             elapsed += time.perf_counter() - t0
             done_bytes += decode_bytes(w, np.array([ctx]))
             done_seqs += 1
@@ -740,11 +906,21 @@ def run_swap_bench(args, device_index):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100,
+                    help="steps per timed repeat (repeats continue until --min-seconds)")
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mha",
-                    choices=["mha", "gqa", "prefix", "prefix_cow", "long16", "long32", "tiny"])
+    ap.add_argument("--workload", default="long16",
+                    choices=["mha", "gqa", "prefix", "prefix_cow", "long16", "long32", "tiny"],
+                    help="the headline configuration (default: long-context split decode, "
+                         "block 16, the largest single-GPU configuration)")
+    ap.add_argument("--configs", choices=["all", "headline"], default="all",
+                    help="all: also time the other configurations (one GPU only), each with "
+                         "its own roofline, under \"configs\" in the JSON line")
+    ap.add_argument("--min-seconds", type=float, default=1.0,
+                    help="device time the headline's timed repeats must reach")
+    ap.add_argument("--extra-min-seconds", type=float, default=0.3,
+                    help="device time each other configuration's repeats must reach")
     ap.add_argument("--partition-tokens", type=int, default=512)
     ap.add_argument("--window", type=int, default=4096, help="window tokens for --decode-mode window")
     ap.add_argument("--swap", action="store_true",
@@ -761,7 +937,8 @@ def main(argv=None):
                          "whole: pa_decode (one CTA per sequence and KV head); "
                          "shared_prefix: pa_decode_shared_prefix (shared prompt blocks read once)")
     ap.add_argument("--states", type=int, default=64, help="distinct decode steps cycled")
-    ap.add_argument("--e2e-steps", type=int, default=64)
+    ap.add_argument("--e2e-steps", type=int, default=256,
+                    help="pipelined end-to-end steps (0: no e2e measurement)")
     ap.add_argument("--batch", type=int, default=None,
                     help="mha only: smaller batch and pool (profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")

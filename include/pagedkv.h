@@ -159,15 +159,20 @@ pa_status_t pa_decode_split(const void* q, const void* k_pool, const void* v_poo
  *
  * - Sizes whose scratch would exceed PA_STATIC_SCRATCH_BYTES (see
  *   pa_decode_split_workspace_size) are rejected with PA_ERR_INVALID_ARG and
- *   a message naming both sizes, before anything is enqueued.
- * - The first call on each device, with that device current, looks up the
- *   array's device address (cudaGetSymbolAddress) and caches it; make that
- *   first call before any stream capture.
+ *   a message naming both sizes, before anything is enqueued. Every other
+ *   refusal (bad arguments, more than 4096 sequences, PAGEDKV_VALIDATE
+ *   findings) also happens before the array is touched.
+ * - The first call in each CUDA context (with that context, and so its
+ *   device, current) looks up the array's device address
+ *   (cudaGetSymbolAddress) and caches it, keyed by the context: an address
+ *   is only valid in the context it was taken in. Make that first call
+ *   before any stream capture.
  * - All calls on a device share the one array, and it keeps the previous
- *   call's contents. Each call clears the part that must start at zero (on
- *   `stream`, before its kernels). Calls that may overlap on the GPU (other
- *   streams, other host threads) race on the array and must be serialised
- *   by the caller; calls issued in order on one stream are safe.
+ *   call's contents. Each accepted call clears the part that must start at
+ *   zero (on `stream`, right before its kernels). Calls that may overlap on
+ *   the GPU (other streams, other host threads) race on the array and must
+ *   be serialised by the caller; calls issued in order on one stream are
+ *   safe.
  * ------------------------------------------------------------------------- */
 #define PA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
@@ -335,7 +340,10 @@ pa_status_t pa_kv_append(const void* k_new, const void* v_new,
  * whole physical block (block_bytes = num_kv_heads*block_size*head_dim*elt
  * bytes, a multiple of 16) from src to dst in both pools ([G] section 4 step
  * 3; [Q], Share Without Mutating State). Pairs must not chain (no dst is
- * another pair's src) and dst ids must be unique.
+ * another pair's src) and dst ids must be unique: all pairs are copied at
+ * once, in no order, so a list that breaks either rule has an undefined
+ * result. Lists from the block manager always keep both (each copy goes to
+ * a block it has just taken from the free queue).
  * ------------------------------------------------------------------------- */
 pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pairs,
                            int num_pairs, size_t block_bytes, int num_blocks,

@@ -40,22 +40,23 @@ def gather_sequence(pool, block_table_row, context_len: int, kv_head: int) -> np
 
     Logical token ``t`` lives in logical block ``t // block_size`` at offset
     ``t % block_size``; the block table turns the logical block into the
-    physical one (qubittool glossary, How It Works).
+    physical one (qubittool glossary, How It Works). All ``context_len``
+    tokens are looked up at once with that rule (array indexing, no loop).
+    A negative table entry (a block released before a sliding window, never
+    attended to) yields NaN rows.
 
     Returns float64 ``[context_len, head_dim]``.
     """
     pool = np.asarray(pool)
     block_size = pool.shape[2]
-    head_dim = pool.shape[3]
-    rows = np.empty((context_len, head_dim), dtype=np.float64)
-    for t in range(context_len):
-        logical_block = t // block_size
-        offset = t % block_size
-        physical_block = int(block_table_row[logical_block])
-        if physical_block < 0:   # released before a sliding window; never attended to
-            rows[t, :] = np.nan
-            continue
-        rows[t, :] = pool[physical_block, kv_head, offset, :]
+    t = np.arange(int(context_len))
+    logical_block = t // block_size
+    offset = t % block_size
+    table = np.asarray(block_table_row, dtype=np.int64)
+    physical_block = table[logical_block]
+    released = physical_block < 0
+    rows = pool[np.where(released, 0, physical_block), kv_head, offset, :].astype(np.float64)
+    rows[released, :] = np.nan
     return rows
 
 
@@ -100,15 +101,24 @@ def paged_decode_one(q, k_pool, v_pool, block_tables, context_lens, scale: float
 def paged_decode(q, k_pool, v_pool, block_tables, context_lens, scale: float) -> np.ndarray:
     """Single-query decode attention for every sequence and query head.
 
+    Each sequence's keys and values are gathered once per KV head and serve
+    every query head of that head's group (the same values
+    ``paged_decode_one`` gathers per query head).
+
     Returns float64 ``[num_seqs, num_q_heads, head_dim]``.
     """
     q = np.asarray(q)
     num_seqs, num_q_heads, head_dim = q.shape
+    num_kv_heads = np.asarray(k_pool).shape[1]
+    group = _group(num_q_heads, num_kv_heads)
     out = np.zeros((num_seqs, num_q_heads, head_dim), dtype=np.float64)
     for s in range(num_seqs):
-        for h in range(num_q_heads):
-            out[s, h] = paged_decode_one(q, k_pool, v_pool, block_tables, context_lens,
-                                         scale, s, h)
+        ctx = int(context_lens[s])
+        for kv_head in range(num_kv_heads):
+            K = gather_sequence(k_pool, block_tables[s], ctx, kv_head)
+            V = gather_sequence(v_pool, block_tables[s], ctx, kv_head)
+            for h in range(kv_head * group, (kv_head + 1) * group):
+                out[s, h] = attention_definition(q[s, h], K, V, scale)
     return out
 
 
@@ -151,6 +161,12 @@ def paged_prefill(q, k_pool, v_pool, block_tables, context_lens, query_lens,
     that writes a request's first KV blocks before decoding ("What is
     PagedAttention?", How It Works: prefill allocates enough blocks for the
     input); the attention itself is the plain causal definition.
+
+    Written for all of a sequence's new tokens of one query head at once:
+    the logits z[i, j] = scale * q_i . k_j are kept where j <= p_i and set to
+    -inf elsewhere (the causal mask), each row is normalised two-pass (its
+    maximum, then exponentials and their sum), and the rows of weights
+    multiply V.
     """
     q = np.asarray(q)
     total, num_q_heads, head_dim = q.shape
@@ -163,14 +179,21 @@ def paged_prefill(q, k_pool, v_pool, block_tables, context_lens, query_lens,
         qlen = int(query_lens[s])
         if qlen > ctx:
             raise ValueError("query_lens[s] must not exceed context_lens[s]")
-        Ks = [gather_sequence(k_pool, block_tables[s], ctx, kvh) for kvh in range(num_kv_heads)]
-        Vs = [gather_sequence(v_pool, block_tables[s], ctx, kvh) for kvh in range(num_kv_heads)]
-        for i in range(qlen):
-            pos = ctx - qlen + i
-            for h in range(num_q_heads):
-                out[row, h] = attention_definition(q[row, h], Ks[h // group][:pos + 1],
-                                                   Vs[h // group][:pos + 1], scale)
-            row += 1
+        if qlen == 0:
+            continue
+        position = np.arange(ctx - qlen, ctx)                     # of each new token
+        visible = np.arange(ctx)[None, :] <= position[:, None]    # [qlen, ctx]
+        for kv_head in range(num_kv_heads):
+            K = gather_sequence(k_pool, block_tables[s], ctx, kv_head)
+            V = gather_sequence(v_pool, block_tables[s], ctx, kv_head)
+            for h in range(kv_head * group, (kv_head + 1) * group):
+                Q = _f64(q[row:row + qlen, h])                    # [qlen, D]
+                z = np.where(visible, scale * (Q @ K.T), -np.inf)
+                zmax = np.max(z, axis=1, keepdims=True)           # pass 1: row maxima
+                e = np.exp(z - zmax)                              # masked entries give 0
+                p = e / np.sum(e, axis=1, keepdims=True)
+                out[row:row + qlen, h] = p @ V
+        row += qlen
     if row != total:
         raise ValueError("sum of query_lens must equal q.shape[0]")
     return out

@@ -357,8 +357,12 @@ struct SplitExtras {
   int window = 0;                    // sliding window (0 = none)
 };
 
+// clear_header: zero the workspace's control header on r.stream right before
+// the launch, after every host-side check has passed (a refused call leaves
+// the workspace untouched).
 pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, void* workspace,
-                       size_t workspace_bytes, const SplitExtras* extras = nullptr) {
+                       size_t workspace_bytes, const SplitExtras* extras = nullptr,
+                       bool clear_header = false) {
   DecodeInstance inst;
   pa_status_t st = validate_and_pick(r, &inst);
   if (st != PA_OK) return st;
@@ -444,6 +448,10 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
 
   void* args[] = {&tmk, &tmv, &a};
   cudaError_t err;
+  if (split && clear_header) {
+    err = cudaMemsetAsync(workspace, 0, kWorkspaceHeader, r.stream);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "clearing the workspace header: %s", cudaGetErrorString(err));
+  }
   if (extras != nullptr && extras->after_prefix_kernel) {
     // Runs alongside the shared-prefix kernel (disjoint partial slots) and
     // waits for it at exit, so the merge that depends on this grid sees both.
@@ -1114,25 +1122,56 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_static_split_scratch[kStaticScratchBytes];
 
-// Device address of the array on the current device. In host code the array's
-// name is only a host-side stand-in, so the address is fetched with
-// cudaGetSymbolAddress once per device (with that device current) and cached.
+// Device address of the array in the current context. In host code the
+// array's name is only a host-side stand-in, so the address is fetched with
+// cudaGetSymbolAddress once per context (with that context's device current)
+// and cached, keyed by the current driver context: an address belongs to the
+// context it was taken in.
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<Fn>(p);
+    return static_cast<Fn>(nullptr);
+  }();
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
 pa_status_t static_scratch_address(void** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
   if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_UNSUPPORTED, "device %d >= %d", dev, kMaxDevices);
+  struct Entry {
+    CUcontext ctx;
+    void* addr;
+  };
   static std::mutex mu;
-  static void* addr[kMaxDevices] = {};
+  static std::vector<Entry> cache;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    err = cudaGetSymbolAddress(&p, g_static_split_scratch);
-    if (err != cudaSuccess || p == nullptr)
-      return fail(PA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(err));
-    addr[dev] = p;
+  CUcontext ctx = current_context();
+  for (const Entry& e : cache) {
+    if (ctx != nullptr && e.ctx == ctx) {
+      *out = e.addr;
+      return PA_OK;
+    }
   }
-  *out = addr[dev];
+  // First use in this context (or no context current yet: the runtime call
+  // below then sets up and makes current the device's primary context).
+  void* p = nullptr;
+  err = cudaGetSymbolAddress(&p, g_static_split_scratch);
+  if (err != cudaSuccess || p == nullptr)
+    return fail(PA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(err));
+  ctx = current_context();
+  if (ctx == nullptr) return fail(PA_ERR_CUDA, "no current CUDA context");
+  cache.push_back(Entry{ctx, p});
+  *out = p;
   return PA_OK;
 }
 
@@ -1216,10 +1255,10 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
   st = static_scratch_address(&scratch);
   if (st != PA_OK) return st;
   // The array keeps whatever the last call left; the control header must
-  // start at zero.
-  cudaError_t err = cudaMemsetAsync(scratch, 0, layout.zero_bytes, r.stream);
-  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "clearing static scratch: %s", cudaGetErrorString(err));
-  return run_decode(r, true, partition_tokens, scratch, kStaticScratchBytes);
+  // start at zero. run_decode clears it on the stream after its own checks
+  // (sequence count, PAGEDKV_VALIDATE), so a refused call writes nothing.
+  return run_decode(r, true, partition_tokens, scratch, kStaticScratchBytes, nullptr,
+                    /*clear_header=*/true);
 }
 
 size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,

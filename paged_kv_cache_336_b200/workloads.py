@@ -13,7 +13,8 @@ on; all values are N(0, 1) draws, all block placements seeded shuffles):
             order is a seeded permutation; then fork(3 -> 4), one appended token
             per sequence 0..3 (sequence 3 copies its shared tail), decode 0..4.
 ``mha``     batch 64, 32 query heads = 32 KV heads, head_dim 128, bf16, block
-            size 16, context lengths uniform in [1, 2048], pool 16384 blocks.
+            size 16, context lengths uniform in [1, 2048], pool 16384 blocks;
+            tables have room for 512 more tokens (bench decode steps).
 ``gqa``     batch 256, 32 query heads over 8 KV heads, head_dim 128, bf16, block
             size 16, context lengths log-uniform in [16, 8192], pool 110% of the
             blocks needed.
@@ -23,7 +24,8 @@ on; all values are N(0, 1) draws, all block placements seeded shuffles):
             partial block) and no private tokens, so the next appended token of
             every branch but the last lands in a shared partial tail.
 ``long``    batch 8, context 131072, 64 query heads over 8 KV heads, head_dim
-            128, bf16, block size 16 or 32, 512-token partitions.
+            128, bf16, block size 16 or 32, 512-token partitions; tables have
+            room for 1024 more tokens (bench decode steps).
 """
 
 from __future__ import annotations
@@ -103,7 +105,7 @@ def mha(repeat: int = 0, batch: int = 64) -> Workload:
     nb = 16384
     return Workload(
         name="mha", num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=16,
-        dtype=BF16, num_blocks=nb, max_blocks_per_seq=2048 // 16 + 8,
+        dtype=BF16, num_blocks=nb, max_blocks_per_seq=2048 // 16 + 32,
         context_lens=ctx, free_order=_perm(rng, nb), seed=seed,
         prefill_seqs=list(range(batch)), step_seqs=list(range(batch)),
         decode_seqs=list(range(batch)))
@@ -170,7 +172,8 @@ def long(repeat: int = 0, block_size: int = 16, slack: float = 0.0, batch: int =
     return Workload(
         name=f"long_bs{block_size}", num_q_heads=64, num_kv_heads=8, head_dim=128,
         block_size=block_size, dtype=BF16, num_blocks=nb,
-        max_blocks_per_seq=per_seq + 8, context_lens=ctx, free_order=_perm(rng, nb),
+        max_blocks_per_seq=per_seq + 1024 // block_size, context_lens=ctx,
+        free_order=_perm(rng, nb),
         seed=seed, prefill_seqs=list(range(batch)),
         step_seqs=list(range(batch)) if slack > 0 else [],
         decode_seqs=list(range(batch)), partition_tokens=512)

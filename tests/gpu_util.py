@@ -1,5 +1,6 @@
 """Helpers shared by the GPU parity tests: workload setup on the device and
-oracle evaluation of sampled outputs (the oracle runs on the CPU in float64)."""
+oracle evaluation of whole outputs (the oracle runs on the CPU in float64 and
+walks the real block tables itself)."""
 
 from __future__ import annotations
 
@@ -41,20 +42,42 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def oracle_one(q, k_pool, v_pool, table_row, ctx, scale, s, h):
-    """Oracle output of (s, h), copying to the host only the (block, KV head)
-    tiles that query head reads; the oracle sees a one-KV-head pool holding
-    those tiles in logical order and the query rows of that head's group."""
-    _, Hkv, bs, D = k_pool.shape
-    G = q.shape[1] // Hkv
-    kvh = h // G
-    nb = -(-int(ctx) // bs)
-    blocks = torch.as_tensor(np.asarray(table_row[:nb], dtype=np.int64), device=k_pool.device)
-    kp = to_f64(k_pool[:, kvh:kvh + 1].index_select(0, blocks)) if nb else np.zeros((0, 1, bs, D))
-    vp = to_f64(v_pool[:, kvh:kvh + 1].index_select(0, blocks)) if nb else np.zeros((0, 1, bs, D))
-    qs = to_f64(q[s:s + 1, kvh * G:(kvh + 1) * G])
-    return oracle.paged_decode_one(qs, kp, vp, np.arange(max(nb, 1))[None, :], [int(ctx)], scale,
-                                   0, h - kvh * G)
+def host_slice(pool: torch.Tensor, kv_head: int, bits: bool = False) -> np.ndarray:
+    """One KV head's slice of a device pool, ``[num_blocks, 1, block_size,
+    head_dim]``, copied to the host: float32 values (bf16 widens exactly), or
+    with ``bits`` the raw element bit patterns (int16 for bf16, int32 for
+    fp32) for bit-exact comparisons. Physical block ids are unchanged, so the
+    oracle walks the real block tables over it."""
+    sl = pool[:, kv_head:kv_head + 1].contiguous()
+    if bits:
+        return sl.view(torch.int16 if pool.element_size() == 2 else torch.int32).cpu().numpy()
+    return sl.float().cpu().numpy()
+
+
+def as_bits(t: torch.Tensor) -> np.ndarray:
+    """Raw element bit patterns of a device tensor, on the host."""
+    t = t.contiguous()
+    return t.view(torch.int16 if t.element_size() == 2 else torch.int32).cpu().numpy()
+
+
+def oracle_decode_by_kv_head(q, k_pool, v_pool, tables, ctx, scale) -> np.ndarray:
+    """oracle.paged_decode over every (sequence, query head) of a batch whose
+    pools are too large to copy to the host whole: one KV head at a time, the
+    oracle gets that head's slice of both pools (``host_slice``), the query
+    rows of its group and the real block tables and context lengths, and does
+    its own gather through the tables. Returns float64 [B, Hq, D]."""
+    B, Hq, D = q.shape
+    Hkv = k_pool.shape[1]
+    G = Hq // Hkv
+    q64 = to_f64(q)
+    out = np.empty((B, Hq, D), dtype=np.float64)
+    for kvh in range(Hkv):
+        kp = host_slice(k_pool, kvh)
+        vp = host_slice(v_pool, kvh)
+        out[:, kvh * G:(kvh + 1) * G] = oracle.paged_decode(q64[:, kvh * G:(kvh + 1) * G], kp, vp,
+                                                            tables, ctx, scale)
+        del kp, vp
+    return out
 
 
 def check_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str = ""):
@@ -68,8 +91,3 @@ def check_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str = ""):
     return float(err.max()), float(err.mean())
 
 
-def sample_pairs(rng, num_seqs, num_q_heads, n, must=()):
-    pairs = set(must)
-    while len(pairs) < min(n, num_seqs * num_q_heads):
-        pairs.add((int(rng.integers(num_seqs)), int(rng.integers(num_q_heads))))
-    return sorted(pairs)

@@ -4,7 +4,8 @@ Forked sequences share their prompt's blocks; the shared-prefix route reads
 them once per KV head for the whole group and must still return plain decode
 attention. Small cases are compared with the full float64 oracle (several
 groups, a group wider than one CTA's rows, sequences in no group, block
-sizes 16 and 32); the full-size prefix-sharing workloads with sampled rows.
+sizes 16 and 32); the full-size prefix-sharing workloads on every output
+row as well.
 Both prefix-pass kernels are covered: the mma.sync one (default, 64 query
 rows per CTA) and the tcgen05 one (PAGEDKV_PREFIX_KERNEL=tcgen05, 128).
 """
@@ -16,8 +17,7 @@ import torch
 import oracle
 from paged_kv_cache_336_b200 import binding, workloads
 
-from gpu_util import (build_tables, check_close, device_tables, oracle_one, sample_pairs, setup,
-                      to_f64)
+from gpu_util import (check_close, device_tables, oracle_decode_by_kv_head, setup, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -85,7 +85,10 @@ def test_shared_prefix_small_matches_oracle(kernel, G, bs, branches):
 
 
 @pytest.mark.parametrize("name", ["prefix", "prefix_cow"])
-def test_shared_prefix_full_size(kernel, name):
+def test_shared_prefix_full_size(monkeypatch, name):
+    """Both prefix-pass kernels on the full-size workload after its append
+    step; every output row against one oracle evaluation (the oracle walks
+    the real tables over one KV head's pool slice at a time)."""
     w = workloads.WORKLOADS[name]()
     bm, k_pool, v_pool = setup(w)
     slots, pairs = bm.append_slots_arrays(w.step_seqs)
@@ -99,14 +102,16 @@ def test_shared_prefix_full_size(kernel, name):
     assert len(groups[2]) == 8
     q = workloads.draw_queries(w, len(seqs), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = binding.decode_shared_prefix(q, k_pool, v_pool, bt, ctx, w.scale, groups, dev_err=err)
-    ref = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale)
+    outs = {}
+    for kern in ("mma_sync", "tcgen05"):
+        if kern == "tcgen05":
+            monkeypatch.setenv("PAGEDKV_PREFIX_KERNEL", "tcgen05")
+        else:
+            monkeypatch.delenv("PAGEDKV_PREFIX_KERNEL", raising=False)
+        outs[kern] = binding.decode_shared_prefix(q, k_pool, v_pool, bt, ctx, w.scale, groups,
+                                                  dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
-    check_close(to_f64(out), to_f64(ref), w.dtype, "shared prefix vs split")
-    rng = np.random.default_rng(w.seed)
-    got, want = [], []
-    for s, h in sample_pairs(rng, len(seqs), w.num_q_heads, 8, [(0, 0), (len(seqs) - 1, 31)]):
-        want.append(oracle_one(q, k_pool, v_pool, tables[s], ctx_np[s], w.scale, s, h))
-        got.append(to_f64(out[s, h]))
-    check_close(np.stack(got), np.stack(want), w.dtype, name)
+    want = oracle_decode_by_kv_head(q, k_pool, v_pool, tables, ctx_np, w.scale)
+    for kern, out in outs.items():
+        check_close(to_f64(out), want, w.dtype, f"{name}[{kern}]")

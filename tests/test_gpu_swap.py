@@ -1,15 +1,18 @@
 """Swap round trip on the GPU: a sequence is preempted (its blocks copied to
 pinned host memory and reclaimed), the pool reuses the blocks, the sequence
-comes back into new blocks; the host copies are bit-exact and its decode
-output is bit-identical to before (placement does not matter)."""
+comes back into new blocks. The host copies and the swapped-in blocks are
+checked bit for bit against the oracle's gather through the old and new
+tables; the decode before and after is checked against the oracle, and is
+bit-identical across the swap (placement does not matter)."""
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from paged_kv_cache_336_b200 import binding, workloads
 
-from gpu_util import device_tables, setup
+from gpu_util import check_close, device_tables, setup, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -19,9 +22,13 @@ def test_swap_out_reuse_swap_in(dtype, G):
     w = workloads.random_small(90 + G, num_seqs=4, num_q_heads=2 * G, num_kv_heads=2, head_dim=128,
                                block_size=16, dtype=dtype, max_ctx=150, min_ctx=40, spare_blocks=2)
     bm, k_pool, v_pool = setup(w)
+    bs, Hkv = w.block_size, w.num_kv_heads
     q = workloads.draw_queries(w, 4, device="cuda")
-    bt, ctx, tables, _ = device_tables(bm, [0, 1, 2, 3])
+    bt, ctx, tables, ctx_np = device_tables(bm, [0, 1, 2, 3])
+    k0, v0 = to_f64(k_pool), to_f64(v_pool)
     before = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=32)
+    check_close(to_f64(before), oracle.paged_decode(to_f64(q), k0, v0, tables, ctx_np, w.scale),
+                dtype, "before swap")
 
     # preempt sequence 1: copy its blocks to host slots 0..n-1
     old = bm.swap_out(1)
@@ -32,8 +39,14 @@ def test_swap_out_reuse_swap_in(dtype, G):
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     binding.swap_out(k_pool, v_pool, host_k, host_v, out_pairs, dev_err=err)
     torch.cuda.synchronize()
-    idx = torch.tensor(old, device="cuda")
-    assert torch.equal(host_k, k_pool[idx].cpu()) and torch.equal(host_v, v_pool[idx].cpu())
+    # the host copies hold every slot of the sequence's blocks: the oracle's
+    # gather through its old table over the pool equals its gather through
+    # host slots 0..n-1 over the host buffers, bit for bit
+    hk, hv = to_f64(host_k), to_f64(host_v)
+    for kvh in range(Hkv):
+        for pool, host in ((k0, hk), (v0, hv)):
+            assert np.array_equal(oracle.gather_sequence(host, list(range(n)), n * bs, kvh),
+                                  oracle.gather_sequence(pool, old, n * bs, kvh))
 
     # the pool reuses the reclaimed blocks: another sequence overwrites them
     bm.allocate(10, n * 16)
@@ -46,10 +59,19 @@ def test_swap_out_reuse_swap_in(dtype, G):
     in_pairs = torch.tensor([[i, b] for i, b in enumerate(new)], dtype=torch.int64, device="cuda")
     binding.swap_in(host_k, host_v, k_pool, v_pool, in_pairs, dev_err=err)
 
-    bt2, ctx2, _, _ = device_tables(bm, [1, 2, 3])
+    bt2, ctx2, tables2, ctx2_np = device_tables(bm, [1, 2, 3])
     after = binding.decode_split(q[1:], k_pool, v_pool, bt2, ctx2, w.scale, partition_tokens=32)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
+    k1, v1 = to_f64(k_pool), to_f64(v_pool)
+    # the swapped-in blocks hold the host copies, bit for bit
+    for kvh in range(Hkv):
+        for pool, host in ((k1, hk), (v1, hv)):
+            assert np.array_equal(oracle.gather_sequence(pool, new, n * bs, kvh),
+                                  oracle.gather_sequence(host, list(range(n)), n * bs, kvh))
+    check_close(to_f64(after), oracle.paged_decode(to_f64(q[1:]), k1, v1, tables2, ctx2_np, w.scale),
+                dtype, "after swap-in")
+    # placement does not matter: the same result as before the swap, bit for bit
     assert torch.equal(after, before[1:])
 
 

@@ -4,10 +4,11 @@ It exists for callers that cannot call cudaMalloc (their device memory is
 owned by another allocator, or an allocation in the middle of a decode loop
 is not acceptable); its scratch is a fixed array inside the library. These
 tests call it through the C ABI and compare it with pa_decode_split, which
-takes a caller workspace, within the tolerances used by every decode test
-(fp32 max-abs 1e-5; bf16 max-abs 2e-2 and mean-abs 2e-3), on two calls in a
-row, since the array keeps the previous call's contents. Oversized requests
-must be refused before anything is enqueued.
+takes a caller workspace, and with the float64 oracle, within the tolerances
+used by every decode test (fp32 max-abs 1e-5; bf16 max-abs 2e-2 and
+mean-abs 2e-3), on two calls in a row, since the array keeps the previous
+call's contents. Oversized requests, and requests refused for any other
+reason, must be turned away before anything is enqueued.
 
 This file sorts last so that a run stopping at the first failure has run
 every other test first; it also passes when run alone in a fresh process.
@@ -17,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from paged_kv_cache_336_b200 import binding, workloads
 
 from gpu_util import check_close, device_tables, setup, to_f64
@@ -45,12 +47,14 @@ def test_static_scratch_matches_workspace_entry_point(dtype, G):
                                fixed_lens=[0, 1, 400])
     bm, k_pool, v_pool = setup(w)
     q = workloads.draw_queries(w, 9, device="cuda")
-    bt, ctx, _, _ = device_tables(bm, list(range(9)))
+    bt, ctx, tables, ctx_np = device_tables(bm, list(range(9)))
     partition = 48  # several partitions per sequence, ragged last one
     need = binding.decode_split_workspace_size(9, 2 * G, 128, 16, bt.shape[1], partition)
     assert need <= STATIC_SCRATCH_BYTES
     ref = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=partition)
     ref_np = to_f64(ref)
+    want = oracle.paged_decode(to_f64(q), to_f64(k_pool), to_f64(v_pool), tables, ctx_np, w.scale)
+    check_close(ref_np, want, dtype, "workspace entry point vs oracle")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     for call in range(2):
         out = torch.full_like(q, float("nan"))
@@ -58,7 +62,8 @@ def test_static_scratch_matches_workspace_entry_point(dtype, G):
         assert status == binding.PA_OK, binding.library().pa_last_error_string()
         torch.cuda.synchronize()
         assert int(err.item()) == 0, f"call {call}: device error word {int(err.item()):#x}"
-        check_close(to_f64(out), ref_np, dtype, f"static scratch, call {call}")
+        check_close(to_f64(out), ref_np, dtype, f"static scratch vs workspace, call {call}")
+        check_close(to_f64(out), want, dtype, f"static scratch vs oracle, call {call}")
     assert torch.all(out[0] == 0)   # empty context
 
 
@@ -83,3 +88,24 @@ def test_static_scratch_refuses_oversized_requests():
     assert b"static" in lib.pa_last_error_string() and b"scratch" in lib.pa_last_error_string()
     torch.cuda.synchronize()
     assert int(err.item()) == 0 and torch.all(out == 0)
+
+    # more sequences than the split decode takes (4096), with scratch to
+    # spare: refused by the sequence-count check, which comes before the
+    # call touches the shared array
+    n = 4097
+    q1 = torch.zeros(n, 1, 128, dtype=torch.bfloat16, device="cuda")
+    bt1 = torch.zeros(n, 1, dtype=torch.int32, device="cuda")
+    ctx1 = torch.zeros(n, dtype=torch.int32, device="cuda")
+    out1 = torch.zeros_like(q1)
+    assert binding.decode_split_workspace_size(n, 1, 128, 16, 1, 16) <= STATIC_SCRATCH_BYTES
+    status = lib.pa_decode_split_static(
+        q1.data_ptr(), pool.data_ptr(), pool.data_ptr(), bt1.data_ptr(), ctx1.data_ptr(), n, 1, 1,
+        128, 16, 8, 1, 0.1, binding.PA_BF16, 16, out1.data_ptr(), err.data_ptr(),
+        torch.cuda.current_stream().cuda_stream)
+    assert status == binding.PA_ERR_UNSUPPORTED
+    assert b"4096" in lib.pa_last_error_string()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and torch.all(out1 == 0)
+
+    # a call after the refusals still matches the oracle
+    test_static_scratch_matches_workspace_entry_point(workloads.BF16, 8)
