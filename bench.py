@@ -80,9 +80,9 @@ def make_workload(name: str, rank: int, batch: int | None = None):
     if name == "prefix_cow":
         return workloads.prefix_cow(repeat=rank)
     if name == "long16":
-        return workloads.long(repeat=rank, block_size=16, slack=0.1)
+        return workloads.long(repeat=rank, block_size=16, slack=0.1, batch=batch or 8)
     if name == "long32":
-        return workloads.long(repeat=rank, block_size=32, slack=0.1)
+        return workloads.long(repeat=rank, block_size=32, slack=0.1, batch=batch or 8)
     if name == "tiny":
         return workloads.tiny(repeat=rank)
     raise SystemExit(f"unknown workload {name}")
@@ -940,7 +940,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=256,
                     help="pipelined end-to-end steps (0: no e2e measurement)")
     ap.add_argument("--batch", type=int, default=None,
-                    help="mha only: smaller batch and pool (profiling captures)")
+                    help="mha, long16, long32: smaller batch and pool (profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -1,10 +1,15 @@
 """Build libpagedkv.so in-tree with nvcc for sm_100a.
 
-Usage: python -m paged_kv_cache_336_b200.build [--force] [--verbose-ptxas]
+Usage: python -m paged_kv_cache_336_b200.build [--force] [--verbose-ptxas] [--nvtx]
 
-Objects go to <repo>/_build/, the shared library next to this file. A source
-is recompiled when it or any header in csrc/ or include/ is newer than its
-object. nvcc cross-compiles; no GPU is needed.
+Objects go to <repo>/_build/ (<repo>/_build/nvtx/ for the NVTX variant), the
+shared library next to this file. A source is recompiled when it or any
+header in csrc/ or include/ is newer than its object. nvcc cross-compiles; no
+GPU is needed.
+
+--nvtx (or PAGEDKV_NVTX=1 in the environment) compiles NVTX ranges around
+every C-ABI call that enqueues GPU work (PAGEDKV_NVTX defined); the default
+build has none.
 """
 
 from __future__ import annotations
@@ -49,8 +54,8 @@ def headers_mtime() -> float:
     return t
 
 
-def _compile(src: str, obj: str, ptxas_verbose: bool) -> tuple[str, str]:
-    cmd = [nvcc(), *ARCH, *COMMON, "-c", src, "-o", obj]
+def _compile(src: str, obj: str, ptxas_verbose: bool, defines=()) -> tuple[str, str]:
+    cmd = [nvcc(), *ARCH, *COMMON, *(f"-D{d}" for d in defines), "-c", src, "-o", obj]
     if ptxas_verbose and src.endswith(".cu"):
         cmd += ["-Xptxas", "-v"]
     p = subprocess.run(cmd, capture_output=True, text=True)
@@ -59,22 +64,35 @@ def _compile(src: str, obj: str, ptxas_verbose: bool) -> tuple[str, str]:
     return src, p.stdout + p.stderr
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = None,
+          nvtx: bool | None = None) -> str:
+    if nvtx is None:
+        nvtx = os.environ.get("PAGEDKV_NVTX") == "1"
+    build_dir = os.path.join(BUILD, "nvtx") if nvtx else BUILD
+    defines = ("PAGEDKV_NVTX=1",) if nvtx else ()
+    os.makedirs(build_dir, exist_ok=True)
     hdr = headers_mtime()
     todo, objs = [], []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         objs.append(obj)
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr):
             todo.append((src, obj))
     logs = []
     if todo:
         with cf.ThreadPoolExecutor(max_workers=jobs or min(len(todo), os.cpu_count() or 4)) as ex:
-            for src, log in ex.map(lambda so: _compile(so[0], so[1], ptxas_verbose), todo):
+            for src, log in ex.map(lambda so: _compile(so[0], so[1], ptxas_verbose, defines), todo):
                 if log.strip():
                     logs.append(f"== {os.path.basename(src)}\n{log}")
-    relink = bool(todo) or not os.path.exists(LIB) or any(
+    # which variant the library was last linked from
+    stamp = os.path.join(BUILD, "variant")
+    variant = "nvtx" if nvtx else "plain"
+    try:
+        with open(stamp) as f:
+            linked = f.read().strip()
+    except OSError:
+        linked = ""
+    relink = bool(todo) or not os.path.exists(LIB) or linked != variant or any(
         os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs)
     if relink:
         tmp = LIB + ".tmp"
@@ -83,8 +101,10 @@ def build(force: bool = False, ptxas_verbose: bool = False, jobs: int | None = N
         if p.returncode != 0:
             raise RuntimeError(f"link failed:\n{' '.join(cmd)}\n{p.stdout}\n{p.stderr}")
         os.replace(tmp, LIB)
+        with open(stamp, "w") as f:
+            f.write(variant)
     if ptxas_verbose and logs:
-        with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+        with open(os.path.join(build_dir, "ptxas.log"), "w") as f:
             f.write("\n".join(logs))
     return LIB
 
@@ -93,8 +113,9 @@ def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--nvtx", action="store_true", help="compile NVTX ranges around the C-ABI calls")
     args = ap.parse_args(argv)
-    lib = build(force=args.force, ptxas_verbose=args.verbose_ptxas)
+    lib = build(force=args.force, ptxas_verbose=args.verbose_ptxas, nvtx=args.nvtx or None)
     print(lib)
     return 0
 

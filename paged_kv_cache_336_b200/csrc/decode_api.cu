@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <functional>
+#include <memory>
 #include <mutex>
 #include <queue>
 #include <utility>
@@ -322,12 +323,14 @@ pa_status_t launch_error(const char* what) {
 }
 
 // Workspace of the split decode:
-//   [0, 256)   control header: ticket counter, finished-CTA counter
+//   [0, 256)   control header (zero; kept for the workspace contract)
+//   pieces     int32 [num_seqs][num_q_heads] (>= one per (sequence, KV head))
 //   m, l       float [num_seqs][num_q_heads][pmax]
 //   acc        float [num_seqs][num_q_heads][pmax][head_dim]
-// The header must be zero before a call; calls leave it zero.
+// pmax bounds the pieces of one (sequence, KV head): a warp takes at least
+// partition_tokens of it, so at most ceil(max_blocks_per_seq / pb) + 1.
 struct SplitLayout {
-  size_t m_off, l_off, acc_off, total;
+  size_t seg_off, m_off, l_off, acc_off, total;
   size_t zero_bytes;  // bytes that must start at zero (the header)
   int pmax;
 };
@@ -336,10 +339,11 @@ SplitLayout split_layout(int num_seqs, int num_q_heads, int head_dim, int block_
                          int max_blocks_per_seq, int partition_tokens) {
   SplitLayout L{};
   const int pb = partition_tokens / block_size;
-  L.pmax = (max_blocks_per_seq + pb - 1) / pb;
+  L.pmax = (max_blocks_per_seq + pb - 1) / pb + 1;
   const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * L.pmax;
-  L.m_off = kWorkspaceHeader;
+  L.seg_off = kWorkspaceHeader;
   L.zero_bytes = kWorkspaceHeader;
+  L.m_off = L.seg_off + align256(static_cast<size_t>(num_seqs) * num_q_heads * 4);
   L.l_off = L.m_off + align256(rows * 4);
   L.acc_off = L.l_off + align256(rows * 4);
   L.total = L.acc_off + align256(rows * head_dim * 4);
@@ -351,11 +355,28 @@ SplitLayout split_layout(int num_seqs, int num_q_heads, int head_dim, int block_
 struct SplitExtras {
   const int32_t* seq_skip_blocks = nullptr;
   const int32_t* seq_part_base = nullptr;
-  size_t m_off = 0, l_off = 0, acc_off = 0, total = 0;
+  size_t seg_off = 0, m_off = 0, l_off = 0, acc_off = 0, total = 0;
   int pmax = 0;
   bool after_prefix_kernel = false;  // launched right after the prefix kernel
   int window = 0;                    // sliding window (0 = none)
 };
+
+// Which split-decode kernel runs. Measured on B200 (bf16, head_dim 128):
+//  * the balanced kernel (every warp an equal run of units, one pass over
+//    each warp's range) streams 131072-token contexts at 0.96-0.99 of the
+//    measured HBM copy peak against 0.93-0.94 for partition tickets, and a
+//    4096-token window over them at 0.51 against 0.41;
+//  * partition tickets (each CTA pulls 512-token items; the warps of a CTA
+//    split an item) stream MHA batch 64 / GQA batch 256 at 0.94 / 0.93
+//    against 0.91 / 0.90, and the shared-prefix suffix pass 10% faster.
+// So tables that can hold 32k tokens or more take the balanced kernel.
+// PAGEDKV_SPLIT_KERNEL=stream|ticket overrides the choice (tests run both).
+bool use_stream_kernel(const DecodeReq& r) {
+  const char* e = std::getenv("PAGEDKV_SPLIT_KERNEL");
+  if (e != nullptr && std::strcmp(e, "stream") == 0) return true;
+  if (e != nullptr && std::strcmp(e, "ticket") == 0) return false;
+  return static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size >= kDeepContextTokens;
+}
 
 // clear_header: zero the workspace's control header on r.stream right before
 // the launch, after every host-side check has passed (a refused call leaves
@@ -386,6 +407,8 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
   a.l2_hint = l2_hint_default();
 
   int smem = inst.fixed_smem;
+  const void* kernel = inst.kernel;
+  int threads = inst.threads;
   dim3 grid;
   if (split) {
     if (partition_tokens <= 0 || partition_tokens % r.block_size != 0)
@@ -400,6 +423,7 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
     if (extras != nullptr && extras->window > 0) {
       a.window = extras->window;
     } else if (extras != nullptr) {
+      L.seg_off = extras->seg_off;
       L.m_off = extras->m_off;
       L.l_off = extras->l_off;
       L.acc_off = extras->acc_off;
@@ -418,18 +442,46 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
     a.partition_blocks = partition_tokens / r.block_size;
     a.max_partitions = L.pmax;
     a.persistent = 1;
-    smem += (r.num_seqs + 1) * 4;
-    st = prepare_kernel(inst.kernel, smem);
-    if (st != PA_OK) return st;
     DeviceInfo dinfo;
     st = device_info(&dinfo);
     if (st != PA_OK) return st;
     int occ = 0;
-    st = occupancy(inst.kernel, inst.threads, smem, &occ);
-    if (st != PA_OK) return st;
-    const int64_t max_items = static_cast<int64_t>(r.num_seqs) * r.num_kv_heads * L.pmax;
-    const int64_t ctas = std::min<int64_t>(max_items, static_cast<int64_t>(dinfo.sms) * occ);
-    grid = dim3(static_cast<unsigned>(ctas > 0 ? ctas : 1));
+    if (use_stream_kernel(r)) {
+      // Balanced pieces per warp (paged_decode_stream_kernel). At most this
+      // many pieces per (sequence, KV head): the slots after the prefix
+      // pass's (none outside shared-prefix decode).
+      a.seg_pieces = reinterpret_cast<int32_t*>(ws + L.seg_off);
+      const int pb = partition_tokens / r.block_size;
+      a.max_pieces = (r.max_blocks_per_seq + pb - 1) / pb + 1;
+      // Units of one KV head's list, at most: bounds the grid for small batches.
+      const int64_t units_max = static_cast<int64_t>(r.num_seqs) *
+                                ((static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size + 15) / 16);
+      if (units_max >= (int64_t(1) << 31))
+        return fail(PA_ERR_UNSUPPORTED, "num_seqs * max context / 16 must be < 2^31");
+      kernel = inst.stream_kernel;
+      threads = inst.stream_threads;
+      smem = inst.stream_fixed_smem + (2 * r.num_seqs + 1) * 4;
+      st = prepare_kernel(kernel, smem);
+      if (st != PA_OK) return st;
+      st = occupancy(kernel, threads, smem, &occ);
+      if (st != PA_OK) return st;
+      // One warp per KV head and group of units; no more groups than units.
+      const int64_t W = inst.stream_warps;
+      const int64_t need = (units_max * r.num_kv_heads + W - 1) / W;
+      const int64_t at_least = (r.num_kv_heads + W - 1) / W;
+      const int64_t ctas = std::max(at_least, std::min<int64_t>(need, static_cast<int64_t>(dinfo.sms) * occ));
+      grid = dim3(static_cast<unsigned>(ctas));
+    } else {
+      // Partition tickets (paged_decode_kernel, persistent mode).
+      smem += (r.num_seqs + 1) * 4;
+      st = prepare_kernel(inst.kernel, smem);
+      if (st != PA_OK) return st;
+      st = occupancy(inst.kernel, inst.threads, smem, &occ);
+      if (st != PA_OK) return st;
+      const int64_t max_items = static_cast<int64_t>(r.num_seqs) * r.num_kv_heads * L.pmax;
+      const int64_t ctas = std::min<int64_t>(max_items, static_cast<int64_t>(dinfo.sms) * occ);
+      grid = dim3(static_cast<unsigned>(ctas > 0 ? ctas : 1));
+    }
   } else {
     a.partition_blocks = r.max_blocks_per_seq;
     a.max_partitions = 1;
@@ -458,7 +510,7 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
     a.wait_prior_at_exit = 1;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(inst.threads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = r.stream;
     cudaLaunchAttribute attr[1];
@@ -466,12 +518,12 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelExC(&cfg, inst.kernel, args);
+    err = cudaLaunchKernelExC(&cfg, kernel, args);
   } else {
-    err = cudaLaunchKernel(inst.kernel, grid, dim3(inst.threads), args, smem, r.stream);
+    err = cudaLaunchKernel(kernel, grid, dim3(threads), args, smem, r.stream);
   }
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
-  if (split && (a.max_partitions > 1 || a.seq_part_base != nullptr)) {
+  if (split) {
     // The merge grid is a programmatic dependent of the decode grid: it may be
     // scheduled before the decode grid ends and waits on the device
     // (griddepcontrol.wait) until the partials are complete and visible.
@@ -493,10 +545,134 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
   return launch_error("decode");
 }
 
+// ---- uploads of host-built plans --------------------------------------------------------
+// pa_prefill and pa_decode_shared_prefix build small plans on the host (work
+// items, schedules, group arrays). An upload from pageable memory may make
+// the host wait for the stream, so each call copies its plan into a slot of
+// a pool of page-locked buffers (one pool per device) and uploads it from
+// there with cudaMemcpyAsync, which returns at once. An event recorded after
+// the uploads marks the slot busy until the copies have read it. A call takes
+// the next slot whose uploads are done; when every slot is still busy (the
+// host has run ahead of the stream) the pool grows by one slot, up to
+// kMaxSlots, and only past that does a call wait, for the oldest slot. A slot
+// grows (a page-locked allocation) when a plan outgrows it.
+struct UploadPiece {
+  void* dst;         // device destination
+  const void* src;   // host source (the plan)
+  size_t bytes;
+};
+
+class PlanStaging {
+ public:
+  static constexpr int kMaxSlots = 64;
+
+  pa_status_t upload(const UploadPiece* pieces, int n, cudaStream_t stream) {
+    size_t total = 0;
+    for (int i = 0; i < n; ++i) total += (pieces[i].bytes + 15) & ~static_cast<size_t>(15);
+    if (total == 0) return PA_OK;
+    std::lock_guard<std::mutex> lock(mu_);
+    Slot* sl = nullptr;
+    pa_status_t st = acquire(&sl);
+    if (st != PA_OK) return st;
+    cudaError_t err;
+    if (sl->cap < total) {
+      if (sl->host != nullptr) cudaFreeHost(sl->host);
+      sl->host = nullptr;
+      sl->cap = 0;
+      const size_t cap = std::max<size_t>(total, 64 * 1024);
+      if ((err = cudaHostAlloc(reinterpret_cast<void**>(&sl->host), cap, cudaHostAllocPortable)) != cudaSuccess)
+        return fail(PA_ERR_CUDA, "plan staging buffer: %s", cudaGetErrorString(err));
+      sl->cap = cap;
+    }
+    size_t off = 0;
+    for (int i = 0; i < n; ++i) {
+      if (pieces[i].bytes == 0) continue;
+      std::memcpy(sl->host + off, pieces[i].src, pieces[i].bytes);
+      if ((err = cudaMemcpyAsync(pieces[i].dst, sl->host + off, pieces[i].bytes, cudaMemcpyHostToDevice,
+                                 stream)) != cudaSuccess)
+        return fail(PA_ERR_CUDA, "plan upload: %s", cudaGetErrorString(err));
+      off += (pieces[i].bytes + 15) & ~static_cast<size_t>(15);
+    }
+    if ((err = cudaEventRecord(sl->done, stream)) != cudaSuccess)
+      return fail(PA_ERR_CUDA, "plan staging record: %s", cudaGetErrorString(err));
+    return PA_OK;
+  }
+
+ private:
+  struct Slot {
+    uint8_t* host = nullptr;
+    size_t cap = 0;
+    cudaEvent_t done = nullptr;
+  };
+
+  // True when the slot's previous uploads are complete (or it has none). A
+  // "not ready" answer is not an error: it is cleared from the runtime's
+  // last-error state unless an error was already pending there.
+  static bool idle(const Slot& sl) {
+    if (sl.done == nullptr) return true;
+    const cudaError_t pending = cudaPeekAtLastError();
+    const cudaError_t q = cudaEventQuery(sl.done);
+    if (q == cudaErrorNotReady && pending == cudaSuccess) (void)cudaGetLastError();
+    return q == cudaSuccess;
+  }
+
+  pa_status_t acquire(Slot** out) {
+    const int n = static_cast<int>(slots_.size());
+    for (int t = 0; t < n; ++t) {
+      Slot* sl = slots_[(next_ + t) % n].get();
+      if (idle(*sl)) {
+        next_ = (next_ + t + 1) % n;
+        *out = sl;
+        return ensure_event(sl);
+      }
+    }
+    if (n < kMaxSlots) {
+      slots_.push_back(std::make_unique<Slot>());
+      *out = slots_.back().get();
+      return ensure_event(*out);
+    }
+    Slot* sl = slots_[next_].get();  // every slot busy: wait for the oldest
+    next_ = (next_ + 1) % n;
+    const cudaError_t err = cudaEventSynchronize(sl->done);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "plan staging wait: %s", cudaGetErrorString(err));
+    *out = sl;
+    return PA_OK;
+  }
+
+  static pa_status_t ensure_event(Slot* sl) {
+    if (sl->done != nullptr) return PA_OK;
+    const cudaError_t err = cudaEventCreateWithFlags(&sl->done, cudaEventDisableTiming);
+    if (err != cudaSuccess) return fail(PA_ERR_CUDA, "plan staging event: %s", cudaGetErrorString(err));
+    return PA_OK;
+  }
+
+  std::mutex mu_;
+  std::vector<std::unique_ptr<Slot>> slots_;
+  int next_ = 0;
+};
+
+// The current device's ring (rings live until the process exits).
+pa_status_t upload_plan(const UploadPiece* pieces, int n, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+  static std::mutex mu;
+  static std::vector<PlanStaging*> rings;
+  PlanStaging* ring;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (static_cast<int>(rings.size()) <= dev) rings.resize(dev + 1, nullptr);
+    if (rings[dev] == nullptr) rings[dev] = new PlanStaging();
+    ring = rings[dev];
+  }
+  return ring->upload(pieces, n, stream);
+}
+
 // ---- shared-prefix decode ------------------------------------------------------------
 // Workspace: [0,256) header | skip int32 [B] | part_base int32 [B] |
-// members int32 [B] | items PrefixItem [B*Hkv*kMaxPrefixParts] |
-// m, l float [B][Hq][pmax] | acc float [B][Hq][pmax][D], where
+// members int32 [B] | items PrefixItem [B*Hkv*kMaxPrefixParts] | q tiles |
+// packed q | pieces int32 [B][Hq] | m, l float [B][Hq][pmax] |
+// acc float [B][Hq][pmax][D], where
 // pmax = kMaxPrefixParts + ceil(max_blocks_per_seq / partition blocks) + 1.
 constexpr int kMaxPrefixParts = 16;
 constexpr int kPrefixRows = 64;  // query rows per prefix CTA (4 warps x 16)
@@ -533,7 +709,8 @@ PrefixLayout prefix_layout(int num_seqs, int num_q_heads, int num_kv_heads, int 
   L.qpack_off = L.qtiles_off + align256(L.max_qtiles * sizeof(QPackTile));
   const size_t qpack_bytes = L.max_qtiles * kTcPrefixRows * static_cast<size_t>(head_dim) * 2;
   const size_t rows = B * num_q_heads * L.ex.pmax;
-  L.ex.m_off = L.qpack_off + align256(qpack_bytes);
+  L.ex.seg_off = L.qpack_off + align256(qpack_bytes);
+  L.ex.m_off = L.ex.seg_off + align256(B * num_q_heads * 4);
   L.ex.l_off = L.ex.m_off + align256(rows * 4);
   L.ex.acc_off = L.ex.l_off + align256(rows * 4);
   L.ex.total = L.ex.acc_off + align256(rows * static_cast<size_t>(head_dim) * 4);
@@ -694,22 +871,15 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaError_t err;
-  if ((err = cudaMemcpyAsync(ws + L.skip_off, skip.data(), B * 4, cudaMemcpyHostToDevice, r.stream)) != cudaSuccess ||
-      (err = cudaMemcpyAsync(ws + L.base_off, base.data(), B * 4, cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
-    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
-  if (!mem.empty() &&
-      (err = cudaMemcpyAsync(ws + L.members_off, mem.data(), mem.size() * 4, cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
-    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
-  if (!items.empty() &&
-      (err = cudaMemcpyAsync(ws + L.items_off, items.data(), items.size() * sizeof(PrefixItem),
-                             cudaMemcpyHostToDevice, r.stream)) != cudaSuccess)
-    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
-  if (!tc_items.empty() &&
-      ((err = cudaMemcpyAsync(ws + L.items_off, tc_items.data(), tc_items.size() * sizeof(PrefillItem),
-                              cudaMemcpyHostToDevice, r.stream)) != cudaSuccess ||
-       (err = cudaMemcpyAsync(ws + L.qtiles_off, qtiles.data(), qtiles.size() * sizeof(QPackTile),
-                              cudaMemcpyHostToDevice, r.stream)) != cudaSuccess))
-    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
+  const UploadPiece plan[] = {
+      {ws + L.skip_off, skip.data(), static_cast<size_t>(B) * 4},
+      {ws + L.base_off, base.data(), static_cast<size_t>(B) * 4},
+      {ws + L.members_off, mem.data(), mem.size() * 4},
+      {ws + L.items_off, items.data(), items.size() * sizeof(PrefixItem)},
+      {ws + L.items_off, tc_items.data(), tc_items.size() * sizeof(PrefillItem)},
+      {ws + L.qtiles_off, qtiles.data(), qtiles.size() * sizeof(QPackTile)}};
+  st = upload_plan(plan, 6, r.stream);
+  if (st != PA_OK) return st;
 
   SplitExtras ex = L.ex;
   ex.seq_skip_blocks = reinterpret_cast<const int32_t*>(ws + L.skip_off);
@@ -1044,14 +1214,12 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaError_t err;
-  if ((err = cudaMemcpyAsync(ws + L.lens_off, lens.data(), lens.size() * 4, cudaMemcpyHostToDevice,
-                             r.stream)) != cudaSuccess ||
-      (err = cudaMemcpyAsync(ws + L.items_off, upload_items, items.size() * sizeof(PrefillItem),
-                             cudaMemcpyHostToDevice, r.stream)) != cudaSuccess ||
-      (persistent &&
-       (err = cudaMemcpyAsync(ws + L.sched_off, sched_offs.data(), sched_offs.size() * 4,
-                              cudaMemcpyHostToDevice, r.stream)) != cudaSuccess))
-    return fail(PA_ERR_CUDA, "upload: %s", cudaGetErrorString(err));
+  const UploadPiece plan[] = {
+      {ws + L.lens_off, lens.data(), lens.size() * 4},
+      {ws + L.items_off, upload_items, items.size() * sizeof(PrefillItem)},
+      {ws + L.sched_off, sched_offs.data(), persistent ? sched_offs.size() * 4 : 0}};
+  st = upload_plan(plan, 3, r.stream);
+  if (st != PA_OK) return st;
   const int rows = r.num_blocks * r.num_kv_heads * r.block_size;
   CUtensorMap tmk, tmv;
   st = pool_tensor_map(r.k_pool, rows, r.head_dim, r.block_size, r.dtype, &tmk);
@@ -1187,6 +1355,7 @@ pa_status_t pa_decode(const void* q, const void* k_pool, const void* v_pool,
                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                       int num_blocks, int max_blocks_per_seq, float scale, pa_dtype_t dtype,
                       void* out, uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_decode");
   DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
               head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
               static_cast<cudaStream_t>(stream)};
@@ -1204,6 +1373,7 @@ size_t pa_decode_split_workspace_size(int num_seqs, int num_q_heads, int head_di
 }
 
 pa_status_t pa_decode_split_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  PA_NVTX_RANGE("pa_decode_split_workspace_init");
   if (workspace == nullptr || workspace_bytes < kWorkspaceHeader)
     return fail(PA_ERR_INVALID_ARG, "workspace must hold at least %zu bytes", kWorkspaceHeader);
   cudaError_t err =
@@ -1218,6 +1388,7 @@ pa_status_t pa_decode_split(const void* q, const void* k_pool, const void* v_poo
                             int num_blocks, int max_blocks_per_seq, float scale, pa_dtype_t dtype,
                             int partition_tokens, void* workspace, size_t workspace_bytes,
                             void* out, uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_decode_split");
   DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
               head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
               static_cast<cudaStream_t>(stream)};
@@ -1230,6 +1401,7 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
                                    int block_size, int num_blocks, int max_blocks_per_seq,
                                    float scale, pa_dtype_t dtype, int partition_tokens, void* out,
                                    uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_decode_split_static");
   DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
               head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
               static_cast<cudaStream_t>(stream)};
@@ -1282,6 +1454,7 @@ pa_status_t pa_decode_shared_prefix(const void* q, const void* k_pool, const voi
                                     const int32_t* group_blocks, void* workspace,
                                     size_t workspace_bytes, void* out, uint32_t* dev_err,
                                     void* stream) {
+  PA_NVTX_RANGE("pa_decode_shared_prefix");
   DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
               head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
               static_cast<cudaStream_t>(stream)};
@@ -1296,6 +1469,7 @@ pa_status_t pa_decode_split_window(const void* q, const void* k_pool, const void
                                    float scale, pa_dtype_t dtype, int partition_tokens, int window,
                                    void* workspace, size_t workspace_bytes, void* out,
                                    uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_decode_split_window");
   if (window < 1) return fail(PA_ERR_INVALID_ARG, "window must be >= 1");
   DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
               head_dim, block_size, num_blocks, max_blocks_per_seq, scale, dtype, out, dev_err,
@@ -1324,6 +1498,7 @@ pa_status_t pa_prefill(const void* q, const void* k_pool, const void* v_pool,
                        int max_blocks_per_seq, float scale, pa_dtype_t dtype,
                        int partition_tokens, void* workspace, size_t workspace_bytes, void* out,
                        uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_prefill");
   // validate_and_pick checks the device-side shapes; context_lens here is a
   // host array, so a placeholder non-null device pointer is not needed.
   DecodeReq r{q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,

@@ -8,12 +8,17 @@
 namespace pagedkv {
 
 struct DecodeInstance {
-  const void* kernel = nullptr;  // paged_decode_kernel<Cfg>
+  const void* kernel = nullptr;  // paged_decode_kernel<Cfg> (whole-context decode)
   const void* merge = nullptr;   // lse_merge_kernel<T, D>
   int threads = 0;
   int fixed_smem = 0;            // dynamic smem bytes before the prefix array
   int stages = 0;
   const char* name = "";
+  // Split decode: paged_decode_stream_kernel<Cfg> (balanced pieces per warp).
+  const void* stream_kernel = nullptr;
+  int stream_threads = 0;
+  int stream_fixed_smem = 0;     // dynamic smem bytes before the per-sequence arrays
+  int stream_warps = 0;
 };
 
 // Each returns false when (head_dim, block_size, group) has no instance.

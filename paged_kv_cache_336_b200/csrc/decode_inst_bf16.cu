@@ -8,8 +8,12 @@
 //  * deep: 2 warps x 3 stages (48 KB; four CTAs per SM). Best measured for
 //    131072-token contexts in 512-token partitions (96.9% against 91.7% for
 //    wide): each warp walks more units of an item per fill and drain.
+#include <cstdlib>
+#include <cstring>
+
 #include "decode_dispatch.h"
 #include "decode_kernel.cuh"
+#include "decode_stream_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefix_kernel.cuh"
 #include "tc_prefill_kernel.cuh"
@@ -29,6 +33,35 @@ static DecodeInstance make_bf16(const char* name) {
   return r;
 }
 
+template <int BS, int D, int W, int NS>
+static void add_stream(DecodeInstance* r) {
+  using Cfg = DecodeCfg<__nv_bfloat16, BS, D, 0, W, NS>;
+  r->stream_kernel = reinterpret_cast<const void*>(&paged_decode_stream_kernel<Cfg>);
+  r->stream_threads = Cfg::kThreads;
+  r->stream_fixed_smem = StreamCfg<Cfg>::kFixedSmem;
+  r->stream_warps = Cfg::W;
+}
+
+// Balanced split-decode CTA shape (warps x ring stages of 16-token K+V
+// units); every shape keeps 192 KB of ring per SM at head_dim 128. Default
+// 8 x 3, one CTA per SM: its 8 warps are the 8 KV heads of one group in the
+// long-context batches, reading the same blocks together; measured on the
+// 131072-token batch at 0.988 of the HBM copy peak against 0.962-0.970 for
+// 4 x 2, 4 x 3 and 2 x 3 at the same SM clock. PAGEDKV_STREAM_SHAPE selects
+// another for measurements: "4x3", "4x2", "2x3".
+template <int BS, int D>
+static void pick_stream(DecodeInstance* r) {
+  const char* e = std::getenv("PAGEDKV_STREAM_SHAPE");
+  if constexpr (D == 256) {
+    add_stream<BS, D, 4, 2>(r);
+  } else {
+    if (e != nullptr && std::strcmp(e, "4x2") == 0) add_stream<BS, D, 4, 2>(r);
+    else if (e != nullptr && std::strcmp(e, "2x3") == 0) add_stream<BS, D, 2, 3>(r);
+    else if (e != nullptr && std::strcmp(e, "4x3") == 0) add_stream<BS, D, 4, 3>(r);
+    else add_stream<BS, D, 8, 3>(r);
+  }
+}
+
 template <int BS, int D>
 static void pick(bool deep, DecodeInstance* out) {
   if constexpr (D == 256) {
@@ -38,6 +71,7 @@ static void pick(bool deep, DecodeInstance* out) {
     if (deep) *out = make_bf16<BS, D, 2, 3>("mma_bf16_deep");
     else *out = make_bf16<BS, D, 4, 2>("mma_bf16_wide");
   }
+  pick_stream<BS, D>(out);
 }
 
 bool find_decode_bf16_mma(int head_dim, int block_size, bool deep, DecodeInstance* out) {

@@ -1,6 +1,7 @@
 // fp32 instances of the paged decode kernel (CUDA-core path).
 #include "decode_dispatch.h"
 #include "decode_kernel.cuh"
+#include "decode_stream_kernel.cuh"
 
 namespace pagedkv {
 
@@ -14,6 +15,10 @@ static DecodeInstance make_f32() {
   r.fixed_smem = Cfg::kFixedSmem;
   r.stages = Cfg::NS;
   r.name = "simt_f32";
+  r.stream_kernel = reinterpret_cast<const void*>(&paged_decode_stream_kernel<Cfg>);
+  r.stream_threads = Cfg::kThreads;
+  r.stream_fixed_smem = StreamCfg<Cfg>::kFixedSmem;
+  r.stream_warps = Cfg::W;
   return r;
 }
 

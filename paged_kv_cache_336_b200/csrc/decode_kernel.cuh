@@ -79,6 +79,12 @@ struct DecodeArgs {
   float scale_log2;      // scale * log2(e)
   int persistent;        // 1: ticket loop + partials; 0: item = blockIdx.x, whole context
   int l2_hint;           // L2 policy of the KV stream: 0 normal, 1 evict-first, 2 evict-last
+  // Balanced split decode (paged_decode_stream_kernel): the number of pieces
+  // each (sequence, KV head) was cut into, written by the kernel and read by
+  // the merge ([B][Hkv]; NULL for the other kernels), and the most pieces one
+  // (sequence, KV head) may be cut into (its partial slots after the base).
+  int32_t* seg_pieces;
+  int max_pieces;
 };
 
 template <typename T, int BS, int D>
@@ -232,6 +238,35 @@ struct SimtWarp {
           for (int j = 0; j < VEC; ++j) acc[h][j] = fmaf(pt, vf[j], acc[h][j]);
         }
       }
+    }
+  }
+
+  // Writes rows 0..G-1 as final outputs (acc / l) to out_rows (G rows of D
+  // contiguous elements); a row with l == 0 gets zeros.
+  __device__ __forceinline__ void store_final(T* out_rows, int lane) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float lt = warp_sum(l[h]);
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) out_rows[h * D + lane * VEC + j] = Elt<T>::from_f32(acc[h][j] * inv);
+    }
+  }
+
+  // Writes rows 0..G-1 as partials (m, l, unnormalised acc) to slots
+  // pr0 + h * row_stride.
+  __device__ __forceinline__ void store_partials(const DecodeArgs& a, int64_t pr0, int64_t row_stride,
+                                                 int lane) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float lt = warp_sum(l[h]);
+      const int64_t pr = pr0 + h * row_stride;
+      if (lane == 0) {
+        a.part_m[pr] = m[h];
+        a.part_l[pr] = lt;
+      }
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) a.part_acc[pr * D + lane * VEC + j] = acc[h][j];
     }
   }
 
@@ -862,7 +897,11 @@ __global__ void __launch_bounds__(128)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int s = row / a.num_q_heads;
   const int base_parts = a.seq_part_base ? a.seq_part_base[s] : 0;
-  const int np = base_parts + seq_partitions(a, s, a.max_blocks_per_seq * block_size, block_size);
+  const int own = a.seg_pieces != nullptr
+                      ? a.seg_pieces[static_cast<int64_t>(s) * a.num_kv_heads +
+                                     (row - s * a.num_q_heads) / a.group]
+                      : seq_partitions(a, s, a.max_blocks_per_seq * block_size, block_size);
+  const int np = min(base_parts + own, a.max_partitions);
   if (np <= 1 && base_parts == 0) return;
   const int64_t base = static_cast<int64_t>(row) * a.max_partitions;
   float M = -INFINITY;

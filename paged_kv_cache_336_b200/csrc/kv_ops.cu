@@ -157,6 +157,7 @@ pa_status_t pa_kv_append(const void* k_new, const void* v_new, const int64_t* sl
                          int num_tokens, int num_kv_heads, int head_dim, int block_size,
                          int num_blocks, pa_dtype_t dtype, void* k_pool, void* v_pool,
                          uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_kv_append");
   if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens < 0");
   if (num_tokens == 0) return ok();
   if (k_new == nullptr || v_new == nullptr || slot_mapping == nullptr || k_pool == nullptr ||
@@ -184,6 +185,7 @@ pa_status_t pa_kv_append(const void* k_new, const void* v_new, const int64_t* sl
 
 pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pairs, int num_pairs,
                            size_t block_bytes, int num_blocks, uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_copy_blocks");
   if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs < 0");
   if (num_pairs == 0) return ok();
   if (k_pool == nullptr || v_pool == nullptr || src_dst_pairs == nullptr)
@@ -206,6 +208,7 @@ pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pa
 pa_status_t pa_swap_out(const void* k_pool, const void* v_pool, void* host_k, void* host_v,
                         const int64_t* pairs, int num_pairs, size_t block_bytes, int num_blocks,
                         int num_host_slots, uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_swap_out");
   if (num_pairs == 0) return ok();
   if (host_k == nullptr || host_v == nullptr) return fail(PA_ERR_INVALID_ARG, "NULL host buffer");
   void *dk = nullptr, *dv = nullptr;
@@ -219,6 +222,7 @@ pa_status_t pa_swap_out(const void* k_pool, const void* v_pool, void* host_k, vo
 pa_status_t pa_swap_in(const void* host_k, const void* host_v, void* k_pool, void* v_pool,
                        const int64_t* pairs, int num_pairs, size_t block_bytes, int num_blocks,
                        int num_host_slots, uint32_t* dev_err, void* stream) {
+  PA_NVTX_RANGE("pa_swap_in");
   if (num_pairs == 0) return ok();
   if (host_k == nullptr || host_v == nullptr) return fail(PA_ERR_INVALID_ARG, "NULL host buffer");
   void *dk = nullptr, *dv = nullptr;

@@ -67,6 +67,7 @@ pa_status_t pa_decode_step(pa_bm_t bm, const pa_step_buffers_t* b, const int64_t
                            const void* q_host, const void* k_new_host, const void* v_new_host,
                            void* out_host, int* num_copies, int synchronize, uint32_t* dev_err,
                            void* stream_ptr) {
+  PA_NVTX_RANGE("pa_decode_step");
   if (bm == nullptr || b == nullptr) return fail(PA_ERR_INVALID_ARG, "bm or buffers is NULL");
   if (n < 0 || n > b->max_seqs) return fail(PA_ERR_INVALID_ARG, "n=%d outside [0, max_seqs=%d]", n, b->max_seqs);
   if (num_copies) *num_copies = 0;

@@ -362,3 +362,30 @@ def test_shared_prefix_rejects_bad_groups_on_host():
     assert call([0, 2], [0, 1], [99], 1) == binding.PA_ERR_INVALID_ARG     # more blocks than the table
     base[13] = binding.PA_F32
     assert call([0, 2], [0, 1], [1], 1) == binding.PA_ERR_UNSUPPORTED      # bf16 only
+
+
+def test_nvtx_ranges_compile_in_only_with_the_build_flag(tmp_path):
+    """With PAGEDKV_NVTX defined (build.py --nvtx) the C-ABI sources carry
+    NVTX ranges around the calls that enqueue GPU work; the default build
+    references no NVTX symbol."""
+    import subprocess
+    from paged_kv_cache_336_b200 import build as B
+    src = os.path.join(B.CSRC, "step_api.cu")
+    syms = {}
+    for variant, defines in (("plain", ()), ("nvtx", ("PAGEDKV_NVTX=1",))):
+        obj = str(tmp_path / f"step_{variant}.o")
+        B._compile(src, obj, False, defines)
+        syms[variant] = subprocess.run(["nm", obj], capture_output=True, text=True,
+                                       check=True).stdout
+    assert "nvtxRangePushA" in syms["nvtx"] or "nvtxGlobals" in syms["nvtx"]
+    assert "nvtx" not in syms["plain"].lower()
+    # every C entry point that launches work opens a range
+    for name, path in (("pa_decode", "decode_api.cu"), ("pa_decode_split", "decode_api.cu"),
+                       ("pa_decode_split_static", "decode_api.cu"),
+                       ("pa_decode_shared_prefix", "decode_api.cu"),
+                       ("pa_decode_split_window", "decode_api.cu"), ("pa_prefill", "decode_api.cu"),
+                       ("pa_kv_append", "kv_ops.cu"), ("pa_copy_blocks", "kv_ops.cu"),
+                       ("pa_swap_out", "kv_ops.cu"), ("pa_swap_in", "kv_ops.cu"),
+                       ("pa_decode_step", "step_api.cu")):
+        text = open(os.path.join(B.CSRC, path)).read()
+        assert f'PA_NVTX_RANGE("{name}");' in text, name

@@ -27,10 +27,22 @@ def _err_word():
 
 
 def _run_decode(kind, q, k_pool, v_pool, bt, ctx, scale, partition=512, err=None):
+    """kind: "decode" (pa_decode), "split" (pa_decode_split, the kernel the
+    library picks), "split_ticket" / "split_stream" (pa_decode_split on the
+    partition-ticket or the balanced kernel)."""
     if kind == "decode":
         return binding.decode(q, k_pool, v_pool, bt, ctx, scale, dev_err=err)
-    return binding.decode_split(q, k_pool, v_pool, bt, ctx, scale, partition_tokens=partition,
-                                dev_err=err)
+    prev = os.environ.get("PAGEDKV_SPLIT_KERNEL")
+    if kind != "split":
+        os.environ["PAGEDKV_SPLIT_KERNEL"] = kind.split("_")[1]
+    try:
+        return binding.decode_split(q, k_pool, v_pool, bt, ctx, scale, partition_tokens=partition,
+                                    dev_err=err)
+    finally:
+        if prev is None:
+            os.environ.pop("PAGEDKV_SPLIT_KERNEL", None)
+        else:
+            os.environ["PAGEDKV_SPLIT_KERNEL"] = prev
 
 
 def _full_oracle(q, k_pool, v_pool, tables, ctx, scale):
@@ -54,7 +66,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("kind", ["decode", "split"])
+@pytest.mark.parametrize("kind", ["decode", "split_ticket", "split_stream"])
 @pytest.mark.parametrize("dtype,Hq,Hkv,D,bs", CASES)
 def test_decode_matches_oracle_small(kind, dtype, Hq, Hkv, D, bs):
     w = workloads.random_small(1000 + Hq * 7 + D + bs, num_seqs=7, num_q_heads=Hq,
@@ -86,14 +98,15 @@ def test_long_table_shape_matches_oracle(bs, G):
     q = workloads.draw_queries(w, 6, device="cuda")
     bt, ctx, tables, ctx_np = device_tables(bm, list(range(6)))
     want = _full_oracle(q, k_pool, v_pool, tables, ctx_np, w.scale)
-    for kind in ("decode", "split"):
+    for kind in ("decode", "split_ticket", "split_stream"):
         out = _run_decode(kind, q, k_pool, v_pool, bt, ctx, w.scale, partition=3 * bs)
         check_close(to_f64(out), want, w.dtype, f"deep {kind}")
 
 
 @pytest.mark.parametrize("dtype,G", [(workloads.F32, 1), (workloads.BF16, 1), (workloads.BF16, 8)])
 @pytest.mark.parametrize("partition_blocks", [1, 2, 3, 5, 64])
-def test_split_any_partition_equals_oracle(dtype, G, partition_blocks):
+@pytest.mark.parametrize("kind", ["split_ticket", "split_stream"])
+def test_split_any_partition_equals_oracle(kind, dtype, G, partition_blocks):
     bs = 16
     w = workloads.random_small(77 + partition_blocks, num_seqs=5, num_q_heads=2 * G,
                                num_kv_heads=2, head_dim=128, block_size=bs, dtype=dtype,
@@ -102,11 +115,10 @@ def test_split_any_partition_equals_oracle(dtype, G, partition_blocks):
     bm, k_pool, v_pool = setup(w)
     q = workloads.draw_queries(w, 5, device="cuda")
     bt, ctx, tables, ctx_np = device_tables(bm, list(range(5)))
-    out = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale,
-                               partition_tokens=partition_blocks * bs)
+    out = _run_decode(kind, q, k_pool, v_pool, bt, ctx, w.scale, partition=partition_blocks * bs)
     ref = binding.decode(q, k_pool, v_pool, bt, ctx, w.scale)
     want = _full_oracle(q, k_pool, v_pool, tables, ctx_np, w.scale)
-    check_close(to_f64(out), want, dtype, "split")
+    check_close(to_f64(out), want, dtype, kind)
     check_close(to_f64(ref), want, dtype, "unsplit")
 
 
@@ -135,7 +147,7 @@ def test_tiny_workload_full_step():
     assert ctx_np.tolist() == [2, 16, 17, 34, 33]
     q = workloads.draw_queries(w, len(w.decode_seqs), device="cuda")
     want = _full_oracle(q, k_pool, v_pool, tables, ctx_np, w.scale)
-    for kind in ("decode", "split"):
+    for kind in ("decode", "split_ticket", "split_stream"):
         out = _run_decode(kind, q, k_pool, v_pool, bt, ctx, w.scale, partition=16, err=err)
         check_close(to_f64(out), want, w.dtype, kind)
     torch.cuda.synchronize()
@@ -193,7 +205,7 @@ def test_device_error_word_and_skipped_accesses():
     # a block id past the pool in sequence 1
     bt_bad = bt.clone()
     bt_bad[1, 1] = w.num_blocks + 5
-    for kind in ("decode", "split"):
+    for kind in ("decode", "split_ticket", "split_stream"):
         err = _err_word()
         out = _run_decode(kind, q, k_pool, v_pool, bt_bad, ctx, w.scale, partition=32, err=err)
         torch.cuda.synchronize()
@@ -236,7 +248,7 @@ def test_gpu_output_independent_of_physical_placement(dtype, G):
     k2[perm] = k_pool
     v2[perm] = v_pool
     bt2 = torch.where(bt >= 0, perm[bt.clamp(min=0).long()].int(), bt)
-    for kind in ("decode", "split"):
+    for kind in ("decode", "split_ticket", "split_stream"):
         a = _run_decode(kind, q, k_pool, v_pool, bt, ctx, w.scale, partition=48)
         b = _run_decode(kind, q, k2, v2, bt2, ctx, w.scale, partition=48)
         assert torch.equal(a, b), kind
@@ -249,7 +261,7 @@ def test_single_token_returns_v_exactly(dtype, G):
     bm, k_pool, v_pool = setup(w)
     q = workloads.draw_queries(w, 3, device="cuda") * 30
     bt, ctx, tables, _ = device_tables(bm, [0, 1, 2])
-    for kind in ("decode", "split"):
+    for kind in ("decode", "split_ticket", "split_stream"):
         out = _run_decode(kind, q, k_pool, v_pool, bt, ctx, w.scale, partition=16)
         for s in range(3):
             b = int(tables[s, 0])
@@ -286,7 +298,12 @@ def test_large_logits_stay_finite():
 
 
 def test_cow_isolation_on_gpu():
-    """A branch's copy-on-write and append leave its siblings' outputs bit-identical."""
+    """A branch's copy-on-write and append leave its siblings' outputs
+    unchanged: bit for bit on pa_decode (one CTA per sequence and KV head, so
+    a sequence's arithmetic does not depend on the rest of the batch), and
+    within the tolerance on pa_decode_split, whose even cut of the batch's
+    work moves piece boundaries when another sequence grows (both against
+    the oracle too)."""
     w = workloads.random_small(14, num_seqs=1, num_q_heads=16, num_kv_heads=4, head_dim=128,
                                block_size=16, dtype=workloads.BF16, max_ctx=0, spare_blocks=12)
     bm = BlockManager(w.num_blocks, 16, 8, w.free_order)
@@ -295,22 +312,32 @@ def test_cow_isolation_on_gpu():
     for c in (1, 2, 3):
         bm.fork(0, c)
     q = workloads.draw_queries(w, 4, device="cuda")
-    bt, ctx, _, _ = device_tables(bm, [0, 1, 2, 3])
-    before = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=32)
+    bt, ctx, tables, ctx_np = device_tables(bm, [0, 1, 2, 3])
+    before = {kind: _run_decode(kind, q, k_pool, v_pool, bt, ctx, w.scale, partition=32)
+              for kind in ("decode", "split_ticket", "split_stream")}
+    want_before = _full_oracle(q, k_pool, v_pool, tables, ctx_np, w.scale)
     slots, pairs = bm.append_slots_arrays([2])
     assert len(pairs) == 1
     binding.copy_blocks(k_pool, v_pool, torch.from_numpy(pairs).cuda())
     kn, vn = workloads.draw_new_kv(w, 1, device="cuda")
     binding.kv_append(kn, vn, torch.from_numpy(slots).cuda(), k_pool, v_pool)
-    bt2, ctx2, _, _ = device_tables(bm, [0, 1, 2, 3])
-    after = binding.decode_split(q, k_pool, v_pool, bt2, ctx2, w.scale, partition_tokens=32)
-    for s in (0, 1, 3):
-        assert torch.equal(before[s], after[s]), s
-    assert not torch.equal(before[2], after[2])
+    bt2, ctx2, tables2, ctx2_np = device_tables(bm, [0, 1, 2, 3])
+    want_after = _full_oracle(q, k_pool, v_pool, tables2, ctx2_np, w.scale)
+    for s in (0, 1, 3):   # the oracle's siblings are unchanged, bit for bit
+        assert np.array_equal(want_before[s], want_after[s]), s
+    for kind in ("decode", "split_ticket", "split_stream"):
+        after = _run_decode(kind, q, k_pool, v_pool, bt2, ctx2, w.scale, partition=32)
+        check_close(to_f64(after), want_after, w.dtype, f"after the copy [{kind}]")
+        for s in (0, 1, 3):
+            if kind == "decode":
+                assert torch.equal(before[kind][s], after[s]), (kind, s)
+            check_close(to_f64(after[s]), to_f64(before[kind][s]), w.dtype, f"sibling {s} [{kind}]")
+        assert not torch.equal(before[kind][2], after[2])
 
 
 def test_repeated_split_calls_reuse_workspace():
-    """The ticket counters in the workspace header return to zero after every call."""
+    """The workspace header (the ticket kernel's counters) is zero again after
+    every call, and repeated calls give the same result."""
     w = workloads.random_small(15, num_seqs=9, num_q_heads=8, num_kv_heads=2, head_dim=128,
                                block_size=16, dtype=workloads.BF16, max_ctx=700)
     bm, k_pool, v_pool = setup(w)

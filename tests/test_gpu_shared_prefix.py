@@ -33,7 +33,9 @@ def kernel(request, monkeypatch):
 
 @pytest.mark.parametrize("G,bs,branches", [(1, 16, 5), (4, 16, 16), (8, 32, 12), (4, 32, 3),
                                            (16, 16, 20), (6, 32, 7)])
-def test_shared_prefix_small_matches_oracle(kernel, G, bs, branches):
+@pytest.mark.parametrize("split_kernel", ["ticket", "stream"])
+def test_shared_prefix_small_matches_oracle(monkeypatch, kernel, split_kernel, G, bs, branches):
+    monkeypatch.setenv("PAGEDKV_SPLIT_KERNEL", split_kernel)
     Hkv, D = 2, 128
     rng = np.random.default_rng(40 + G + bs)
     NB = 400

@@ -29,6 +29,9 @@ def test_swap_out_reuse_swap_in(dtype, G):
     before = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=32)
     check_close(to_f64(before), oracle.paged_decode(to_f64(q), k0, v0, tables, ctx_np, w.scale),
                 dtype, "before swap")
+    # the batch decoded after the swap-in (sequences 1..3), on the old placement
+    before_123 = binding.decode_split(q[1:], k_pool, v_pool, bt[1:].contiguous(), ctx[1:].contiguous(),
+                                      w.scale, partition_tokens=32)
 
     # preempt sequence 1: copy its blocks to host slots 0..n-1
     old = bm.swap_out(1)
@@ -71,8 +74,9 @@ def test_swap_out_reuse_swap_in(dtype, G):
                                   oracle.gather_sequence(host, list(range(n)), n * bs, kvh))
     check_close(to_f64(after), oracle.paged_decode(to_f64(q[1:]), k1, v1, tables2, ctx2_np, w.scale),
                 dtype, "after swap-in")
-    # placement does not matter: the same result as before the swap, bit for bit
-    assert torch.equal(after, before[1:])
+    # placement does not matter: the same batch gives the same result as
+    # before the swap, bit for bit
+    assert torch.equal(after, before_123)
 
 
 def test_swap_rejects_pageable_host_memory():

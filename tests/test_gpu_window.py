@@ -18,7 +18,9 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("dtype,G,bs", [(workloads.F32, 1, 16), (workloads.BF16, 1, 32),
                                         (workloads.BF16, 8, 16), (workloads.F32, 2, 32)])
 @pytest.mark.parametrize("window", [1, 7, 16, 40, 97, 10_000])
-def test_window_matches_oracle(dtype, G, bs, window):
+@pytest.mark.parametrize("split_kernel", ["ticket", "stream"])
+def test_window_matches_oracle(monkeypatch, split_kernel, dtype, G, bs, window):
+    monkeypatch.setenv("PAGEDKV_SPLIT_KERNEL", split_kernel)
     w = workloads.random_small(60 + G + bs, num_seqs=7, num_q_heads=2 * G, num_kv_heads=2,
                                head_dim=128, block_size=bs, dtype=dtype, max_ctx=12 * bs,
                                fixed_lens=[0, 1, 12 * bs, bs + 1])

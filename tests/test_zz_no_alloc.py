@@ -14,6 +14,8 @@ This file sorts last so that a run stopping at the first failure has run
 every other test first; it also passes when run alone in a fresh process.
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -41,6 +43,15 @@ def _call_static(q, k_pool, v_pool, bt, ctx, scale, partition_tokens, out, err):
 
 @pytest.mark.parametrize("dtype,G", [(workloads.F32, 1), (workloads.BF16, 1), (workloads.BF16, 8)])
 def test_static_scratch_matches_workspace_entry_point(dtype, G):
+    for split_kernel in ("ticket", "stream"):
+        os.environ["PAGEDKV_SPLIT_KERNEL"] = split_kernel
+        try:
+            _static_matches(dtype, G)
+        finally:
+            os.environ.pop("PAGEDKV_SPLIT_KERNEL", None)
+
+
+def _static_matches(dtype, G):
     torch.cuda.set_device(0)
     w = workloads.random_small(31 + G, num_seqs=9, num_q_heads=2 * G, num_kv_heads=2,
                                head_dim=128, block_size=16, dtype=dtype, max_ctx=400,
@@ -108,4 +119,4 @@ def test_static_scratch_refuses_oversized_requests():
     assert int(err.item()) == 0 and torch.all(out1 == 0)
 
     # a call after the refusals still matches the oracle
-    test_static_scratch_matches_workspace_entry_point(workloads.BF16, 8)
+    _static_matches(workloads.BF16, 8)
