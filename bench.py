@@ -248,8 +248,9 @@ class ClockSampler:
                 "gpu": self.uuid}
 
 
-DECODE_SOURCES = ("decode_kernel.cuh", "device_common.cuh")
-PREFIX_SOURCES = ("prefix_kernel.cuh", "decode_kernel.cuh", "device_common.cuh")
+DECODE_SOURCES = ("decode_kernel.cuh", "decode_stream_kernel.cuh", "device_common.cuh")
+PREFIX_SOURCES = ("prefix_kernel.cuh", "decode_kernel.cuh", "decode_stream_kernel.cuh",
+                  "device_common.cuh")
 PREFILL_SOURCES = ("tc_prefill_kernel.cuh", "prefill_kernel.cuh", "device_common.cuh")
 
 
@@ -362,15 +363,66 @@ class DeviceStep:
         return ((1 if st["n_pairs"] else 0) + (1 if self.T else 0) + 1 + prefix +
                 (1 if self.merge_launched else 0))
 
-    def run(self, i, ev=None):
-        st = self.states[i % len(self.states)]
+    def _writes(self, st):
         b = self.binding
         if st["n_pairs"]:
             b.copy_blocks(self.k_pool, self.v_pool, st["pairs"])
         if self.T:
             b.kv_append(st["k_new"], st["v_new"], st["slots"], self.k_pool, self.v_pool)
+
+    def capture(self) -> str | None:
+        """Captures each state's step as two CUDA graphs (the copies and
+        append; the decode call), so that a timed step costs two graph
+        launches of host time instead of several library calls. Returns None
+        on success, else why the step stays eager. The shared-prefix route
+        stays eager: its call uploads a host-built plan, which a graph would
+        re-read from a reused staging slot at replay."""
+        if self.mode == "shared_prefix":
+            return "shared-prefix calls upload a host plan per call"
+        torch = self.torch
+        graphs = []
+        try:
+            torch.cuda.synchronize()
+            for st in self.states:
+                g_w = None
+                if st["n_pairs"] or self.T:
+                    g_w = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g_w):
+                        self._writes(st)
+                g_d = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g_d):
+                    self._decode(st)
+                graphs.append((g_w, g_d))
+            torch.cuda.synchronize()
+        except Exception as e:  # capture refused: stay eager, say why
+            torch.cuda.synchronize()
+            return f"{type(e).__name__}: {e}"[:200]
+        self.graphs = graphs
+        return None
+
+    def run(self, i, ev=None):
+        st = self.states[i % len(self.states)]
+        graphs = getattr(self, "graphs", None)
+        if graphs is not None:
+            g_w, g_d = graphs[i % len(self.states)]
+            if g_w is not None:
+                g_w.replay()
+            if ev is not None:
+                ev[0].record()
+            g_d.replay()
+            if ev is not None:
+                ev[1].record()
+            return st
+        self._writes(st)
         if ev is not None:
             ev[0].record()
+        self._decode(st)
+        if ev is not None:
+            ev[1].record()
+        return st
+
+    def _decode(self, st):
+        b = self.binding
         if self.whole:
             b.decode(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"], self.w.scale,
                      out=self.out)
@@ -388,9 +440,6 @@ class DeviceStep:
             b.decode_split(st["q"], self.k_pool, self.v_pool, st["tables"], st["ctx"],
                            self.w.scale, partition_tokens=self.partition_tokens, out=self.out,
                            workspace=self.ws)
-        if ev is not None:
-            ev[1].record()
-        return st
 
 
 CONFIG_LABELS = {
@@ -518,6 +567,10 @@ def bench_config(args, workload_key, mode, rank, world, device, device_index, mi
     for i in range(args.warmup):
         ds.run(i)
     torch.cuda.synchronize()
+    eager_why = ds.capture() if args.graphs else "--graphs off"
+    for i in range(args.warmup):
+        ds.run(i)
+    torch.cuda.synchronize()
     clocks = ClockSampler(device_index)
     clocks.start()
     reps, calls, launches, _ = timed_repeats(ds, args.steps, args.warmup, min_ms, world, device)
@@ -525,6 +578,9 @@ def bench_config(args, workload_key, mode, rank, world, device, device_index, mi
     peak, peak_kind = hbm_peak()
     res = summarize(ds, reps, calls, args.steps, world, workload_key, mode, peak, peak_kind,
                     clock_info)
+    res["launch"] = ("CUDA graphs, one per state for the copies and append and one for the "
+                     "decode call (captured library calls)" if eager_why is None
+                     else f"eager library calls ({eager_why})")
     if not keep:
         del ds
         torch.cuda.synchronize()
@@ -590,6 +646,7 @@ def run_ours(args, rank, world, device_index):
                 "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                 "parallelism": f"independent batch per GPU x{world}",
             },
+            "launch": head["launch"],
             "value_p10_p90": head["value_p10_p90"],
             "repeats": head["repeats"],
             "decode_tokens_per_s": head["decode_tokens_per_s"],
@@ -696,6 +753,18 @@ def b_new_kv(w, n, i, device):
 # ---------------------------------------------------------------------------
 # the CPU oracle (cpu_baseline leg and --impl reference)
 
+_ORACLE_INPUT = [None, None]   # (key, inputs) of the last sequence drawn for the oracle
+
+
+def seq_context(w, s: int) -> int:
+    """Context length of sequence s before the step (a forked sequence has
+    its parent's)."""
+    parents = {child: parent for parent, child in w.forks}
+    while s >= len(w.context_lens) and s in parents:
+        s = parents[s]
+    return int(w.context_lens[s])
+
+
 def time_oracle(w, budget_s: float, seed: int = 0, threads: int = 1):
     """Times the float64 oracle on whole sequences of the workload (all query
     heads of each), with `threads` BLAS/torch threads, until ~budget_s seconds
@@ -716,12 +785,18 @@ def time_oracle(w, budget_s: float, seed: int = 0, threads: int = 1):
     torch.set_num_threads(threads)
     with threadpool_limits(limits=threads):
         for idx in order:
-            ctx = int(w.context_lens[idx]) + (1 if w.step_seqs else 0)
+            ctx = seq_context(w, int(idx)) + (1 if w.step_seqs else 0)
             nb = -(-ctx // bs)
             # a contiguous one-sequence pool drawn from the same distribution
-            kp = workloads.draw_normal((nb, Hkv, bs, D), w.dtype, w.seed * 7 + int(idx)).double().numpy()
-            vp = workloads.draw_normal((nb, Hkv, bs, D), w.dtype, w.seed * 7 + 99991 + int(idx)).double().numpy()
-            q = workloads.draw_normal((1, w.num_q_heads, D), w.dtype, w.seed * 7 + 3 + int(idx)).double().numpy()
+            # (drawn outside the timed region; the last one is kept for reuse)
+            key = (w.name, w.seed, int(idx))
+            if _ORACLE_INPUT[0] != key:
+                _ORACLE_INPUT[:] = [None, None]
+                kp = workloads.draw_normal((nb, Hkv, bs, D), w.dtype, w.seed * 7 + int(idx)).double().numpy()
+                vp = workloads.draw_normal((nb, Hkv, bs, D), w.dtype, w.seed * 7 + 99991 + int(idx)).double().numpy()
+                q = workloads.draw_normal((1, w.num_q_heads, D), w.dtype, w.seed * 7 + 3 + int(idx)).double().numpy()
+                _ORACLE_INPUT[:] = [key, (kp, vp, q)]
+            kp, vp, q = _ORACLE_INPUT[1]
             table = np.arange(nb)[None, :]
             t0 = time.perf_counter()
             oracle.paged_decode(q, kp, vp, table, [ctx], w.scale)
@@ -742,13 +817,15 @@ def run_reference(args, rank, world):
         return None
     w = make_workload(args.workload, 0, args.batch)
     # each step: a bounded sample of the workload (at least one whole sequence),
-    # sized so that the whole run ends within a few minutes
-    per_step = min(10.0, 120.0 / max(1, args.steps + args.warmup))
+    # sized so that the whole run ends within a few minutes; with long
+    # sequences (seconds of oracle work each) every step times the same one
+    per_step = min(10.0, 60.0 / max(1, args.steps + args.warmup))
+    long_seqs = float(np.max(w.context_lens)) >= 32768
     for _ in range(args.warmup):
         time_oracle(w, per_step / 4)
     vals, tok, descs, secs = [], [], [], 0.0
     for i in range(args.steps):
-        g, t, d, el = time_oracle(w, per_step, seed=i)
+        g, t, d, el = time_oracle(w, per_step, seed=0 if long_seqs else i)
         vals.append(g)
         tok.append(t)
         descs.append(d)
@@ -937,12 +1014,16 @@ def main(argv=None):
                          "whole: pa_decode (one CTA per sequence and KV head); "
                          "shared_prefix: pa_decode_shared_prefix (shared prompt blocks read once)")
     ap.add_argument("--states", type=int, default=64, help="distinct decode steps cycled")
+    ap.add_argument("--graphs", choices=["on", "off"], default="on",
+                    help="time the device-resident step as replays of captured CUDA graphs "
+                         "(the shared-prefix route always runs eagerly)")
     ap.add_argument("--e2e-steps", type=int, default=256,
                     help="pipelined end-to-end steps (0: no e2e measurement)")
     ap.add_argument("--batch", type=int, default=None,
                     help="mha, long16, long32: smaller batch and pool (profiling captures)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     args = ap.parse_args(argv)
+    args.graphs = args.graphs == "on"
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 

@@ -203,6 +203,13 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
  * pa_decode_shared_prefix_workspace_size(...) bytes, 256-byte aligned,
  * initialised once with pa_decode_split_workspace_init (the same contract as
  * pa_decode_split).
+ *
+ * Host plans (this call and pa_prefill): the plan built from the host
+ * arrays is copied into a page-locked staging slot owned by the library and
+ * uploaded from there on `stream`; the call returns without waiting for the
+ * stream. Slots are reused once their upload has completed, so these two
+ * calls must not be captured into a CUDA graph (a replay would read a slot
+ * that has since been reused).
  * ------------------------------------------------------------------------- */
 size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                               int head_dim, int block_size,
@@ -343,7 +350,9 @@ pa_status_t pa_kv_append(const void* k_new, const void* v_new,
  * another pair's src) and dst ids must be unique: all pairs are copied at
  * once, in no order, so a list that breaks either rule has an undefined
  * result. Lists from the block manager always keep both (each copy goes to
- * a block it has just taken from the free queue).
+ * a block it has just taken from the free queue). With PAGEDKV_VALIDATE=1
+ * the pairs are read back (synchronously) and such a list, or a pair outside
+ * [0, num_blocks), is refused with PA_ERR_INVALID_ARG before any copy.
  * ------------------------------------------------------------------------- */
 pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pairs,
                            int num_pairs, size_t block_bytes, int num_blocks,

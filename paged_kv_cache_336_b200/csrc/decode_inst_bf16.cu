@@ -116,9 +116,9 @@ static PrefixInstance make_prefill() {
 // faster than one tile per CTA at two CTAs per SM).
 constexpr int kTcPrefillTiles = 2;
 
-template <int BS, int D, int TILES = kTcPrefillTiles>
+template <int BS, int D, int TILES = kTcPrefillTiles, int HALVES = 1>
 static PrefixInstance make_tc_prefill() {
-  using Cfg = TcCfg<BS, D, TILES>;
+  using Cfg = TcCfg<BS, D, TILES, HALVES>;
   PrefixInstance r;
   r.kernel = reinterpret_cast<const void*>(&tc_prefill_kernel<Cfg>);
   r.threads = Cfg::kThreads;
@@ -129,9 +129,14 @@ static PrefixInstance make_tc_prefill() {
   return r;
 }
 
+// Threads per query row in the tcgen05 softmax: PAGEDKV_PREFILL_HALVES=2
+// splits each row's logits between two threads (16 softmax warps).
 template <int BS, int D>
 static PrefixInstance pick_prefill(bool tcgen05) {
-  return tcgen05 ? make_tc_prefill<BS, D>() : make_prefill<BS, D>();
+  if (!tcgen05) return make_prefill<BS, D>();
+  const char* e = std::getenv("PAGEDKV_PREFILL_HALVES");
+  if (e != nullptr && std::strcmp(e, "2") == 0) return make_tc_prefill<BS, D, kTcPrefillTiles, 2>();
+  return make_tc_prefill<BS, D>();
 }
 
 bool find_prefill_bf16(int head_dim, int block_size, bool tcgen05, PrefixInstance* out) {

@@ -17,6 +17,9 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
+#include <unordered_set>
+#include <vector>
 #include <cstdint>
 
 #include "device_common.cuh"
@@ -147,6 +150,14 @@ int sm_count() {
 }
 
 }  // namespace
+bool validate_copy_pairs() {
+  static const bool enabled = [] {
+    const char* e = std::getenv("PAGEDKV_VALIDATE");
+    return e != nullptr && e[0] == '1';
+  }();
+  return enabled;
+}
+
 }  // namespace pagedkv
 
 using namespace pagedkv;
@@ -194,6 +205,28 @@ pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pa
     return fail(PA_ERR_INVALID_ARG, "block_bytes must be a positive multiple of 16");
   if (num_blocks <= 0) return fail(PA_ERR_INVALID_ARG, "num_blocks must be positive");
   if (!aligned16(k_pool) || !aligned16(v_pool)) return fail(PA_ERR_INVALID_ARG, "pools must be 16-byte aligned");
+  if (validate_copy_pairs()) {
+    // PAGEDKV_VALIDATE=1: the pairs come to the host (synchronously) and a list
+    // whose result would depend on the order of the copies is refused.
+    std::vector<int64_t> h(2 * static_cast<size_t>(num_pairs));
+    cudaError_t e = cudaMemcpyAsync(h.data(), src_dst_pairs, h.size() * 8, cudaMemcpyDeviceToHost,
+                                    static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "PAGEDKV_VALIDATE copy failed: %s", cudaGetErrorString(e));
+    std::unordered_set<int64_t> dst;
+    for (int i = 0; i < num_pairs; ++i) {
+      const int64_t a = h[2 * i], b = h[2 * i + 1];
+      if (a < 0 || a >= num_blocks || b < 0 || b >= num_blocks)
+        return fail(PA_ERR_INVALID_ARG, "copy pair %d (%lld, %lld) outside [0, %d)", i, (long long)a,
+                    (long long)b, num_blocks);
+      if (!dst.insert(b).second)
+        return fail(PA_ERR_INVALID_ARG, "copy pairs: destination %lld appears twice", (long long)b);
+    }
+    for (int i = 0; i < num_pairs; ++i)
+      if (dst.count(h[2 * i]))
+        return fail(PA_ERR_INVALID_ARG, "copy pairs: block %lld is both a source and a destination",
+                    (long long)h[2 * i]);
+  }
   const int64_t upb = static_cast<int64_t>(block_bytes / 16);
   const int gx = static_cast<int>(std::min<int64_t>((upb + 1023) / 1024, 64));
   const int gy = std::min(num_pairs, 65535);

@@ -79,7 +79,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-template <int BS_, int D_, int TILES_>
+template <int BS_, int D_, int TILES_, int HALVES_ = 1>
 struct TcCfg {
   static constexpr int BS = BS_;
   static constexpr int D = D_;
@@ -91,18 +91,27 @@ struct TcCfg {
   static constexpr int KCH = D * 2 / 128;               // 128-byte column chunks of a row
   static constexpr int kQBytes = ROWS * D * 2;          // one tile's Q
   static constexpr int kSlotBytes = CHUNK * D * 2;      // K or V of one chunk
+  // Threads per query row in the softmax (1 or 2): with two, each takes half
+  // of a chunk's 64 logits and half of O's columns.
+  static constexpr int HALVES = HALVES_;
   // ring: K_0 V_0 K_1 V_1 ...; one-tile CTAs run two per SM (TMEM and
   // shared memory for two), so one CTA's prologue and epilogue overlap the
-  // other's main loop.
-  static constexpr int NSLOT = TILES == 2 ? 8 : 4;
+  // other's main loop. Two-tile CTAs with two threads per row keep 7 slots:
+  // the eighth's 16 KB went to the halves' exchange buffers.
+  static constexpr int NSLOT = TILES == 2 ? (HALVES == 2 ? 7 : 8) : 4;
   static constexpr int kMinBlocks = TILES == 2 ? 1 : 2;
   static constexpr int kBarBytes = 512;
   // Two-tile CTAs stage each tile's normalised output, 64 columns at a time,
   // for one TMA store (one-tile CTAs serve scattered output rows).
   static constexpr bool kTmaOut = TILES == 2;
   static constexpr int kStageBytes = kTmaOut ? TILES * ROWS * 128 : 0;
-  static constexpr int kSmem = 1024 + TILES * kQBytes + NSLOT * kSlotBytes + kStageBytes + kBarBytes;
-  static constexpr int kSoftmaxWarps = 4 * TILES;
+  // The halves of a row swap row maxima (each chunk) and row sums (each item)
+  // through [tile][buffer][half][row] floats, double-buffered.
+  static constexpr int kXchgBytes = HALVES == 2 ? TILES * 2 * HALVES * ROWS * 4 : 0;
+  static constexpr int kSmem =
+      1024 + TILES * kQBytes + NSLOT * kSlotBytes + kStageBytes + kXchgBytes + kBarBytes;
+  static constexpr int kTileWarps = 4 * HALVES;         // softmax warps per tile
+  static constexpr int kSoftmaxWarps = kTileWarps * TILES;
   static constexpr int kThreads = (kSoftmaxWarps + 1 + TILES) * 32;
   static constexpr uint32_t kTileCols = 256;            // S buffers [0,128), O [128, 128 + D)
   static constexpr uint32_t kTmemCols = TILES * kTileCols;
@@ -115,6 +124,7 @@ struct TcCfg {
   static_assert(kTmemCols * kMinBlocks <= 512, "tensor memory");
   static_assert(kSmem * kMinBlocks <= 228 * 1024, "shared memory per SM");
   static_assert(TILES == 1 || TILES == 2, "tiles");
+  static_assert(HALVES == 1 || HALVES == 2, "threads per row");
 };
 
 // One work item as every role of the CTA sees it.
@@ -161,19 +171,21 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
   uint8_t* qs = smem;                                    // [TILES][KCH][ROWS][128 B]
   uint8_t* slots = qs + Cfg::TILES * Cfg::kQBytes;       // [NSLOT][KCH][CHUNK][128 B]
   uint8_t* stage = slots + NSLOT * Cfg::kSlotBytes;      // [TILES][ROWS][128 B] output staging
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stage + Cfg::kStageBytes);
+  float* xval = reinterpret_cast<float*>(stage + Cfg::kStageBytes);  // [TILES][2][HALVES][ROWS]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage + Cfg::kStageBytes + Cfg::kXchgBytes);
   uint64_t* kv_full = bars;               // [NSLOT] TMA bytes landed
   uint64_t* kv_empty = bars + NSLOT;      // [NSLOT] both tiles done with the slot
   uint64_t* s_full = bars + 2 * NSLOT;    // [tile][buffer] S MMA done (commit)
-  uint64_t* p_full = s_full + 4;          // [tile][buffer] P written (4 warp arrivals)
+  uint64_t* p_full = s_full + 4;          // [tile][buffer] P written (a tile's softmax warps)
   uint64_t* p_free = p_full + 4;          // [tile][buffer] P V MMA done (commit)
   uint64_t* q_full = p_free + 4;          // [tile] Q in shared memory (TMA bytes)
   uint64_t* q_free = q_full + 2;          // [tile] the item's last S MMA done (commit)
   uint64_t* o_last = q_free + 2;          // [tile] every MMA of the item done (commit)
-  uint64_t* o_empty = o_last + 2;         // [tile] O read out of TMEM (4 warp arrivals)
+  uint64_t* o_empty = o_last + 2;         // [tile] O read out of TMEM (a tile's softmax warps)
   uint64_t* mma_done = o_empty + 2;       // [tile] every MMA of the CTA done (commit), once
   uint64_t* v_tail = mma_done + 2;        // a last chunk's V tail rows cleared (producer)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_tail + 1);
+  uint64_t* xchg = v_tail + 1;            // [tile][buffer] both halves' values written (threads)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xchg + 4);
 
   grid_dependents_launch();
   const int tid = threadIdx.x;
@@ -193,14 +205,15 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], Cfg::kTileWarps);
       mbar_init(&p_free[i], 1);
+      mbar_init(&xchg[i], Cfg::kTileWarps * 32);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&q_full[t], 1);
       mbar_init(&q_free[t], 1);
       mbar_init(&o_last[t], 1);
-      mbar_init(&o_empty[t], 4);
+      mbar_init(&o_empty[t], Cfg::kTileWarps);
       mbar_init(&mma_done[t], 1);
     }
     mbar_init(v_tail, 1);
@@ -457,13 +470,43 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     __syncwarp();
     wait(&mma_done[t], 0);
   } else {
-    // ---- softmax warps: tile t = warp / 4, thread r owns row r (TMEM lane r) --------
-    const int t = warp >> 2;
-    const int r = (warp & 3) * 32 + lane;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + t * Cfg::kTileCols;
+    // ---- softmax warps: tile t = warp / (4 HALVES). Warp w of the tile reads
+    // TMEM lane quarter w % 4 (rows 32 (w % 4) ..); with two threads per row,
+    // half hf = w / 4 of the columns: logits 32 hf .. 32 hf + 31 of each chunk,
+    // O columns hf D/2 .. of the row. Thread (quarter, lane) owns row r = 32
+    // quarter + lane, with its partner thread of the other half; the two swap
+    // their row maximum every chunk (and their row sum at the item's end)
+    // through xval, completed by xchg (every thread of the tile arrives, so
+    // each thread's own store is released by its arrival).
+    constexpr int HALF_CHUNK = CHUNK / Cfg::HALVES;
+    constexpr int HALF_D = D / Cfg::HALVES;
+    const int t = warp / Cfg::kTileWarps;
+    const int wt = warp % Cfg::kTileWarps;
+    const int hf = wt >> 2;
+    const int r = (wt & 3) * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (wt & 3)) << 16) + t * Cfg::kTileCols;
+    float* xt = xval + t * (2 * Cfg::HALVES * ROWS);
     const float sl2 = a.scale_log2;
-    int cb = 0, nt = 0;
+    int cb = 0, nt = 0, ex = 0;
     bool ok = true;  // warp-uniform
+    // Publishes v, waits (bounded) until both halves of the tile published,
+    // returns the partner's value. Buffers alternate, so a half can run at
+    // most one exchange ahead of its partner's read.
+    // The tcgen05 fences order this thread's TMEM loads before the partner's
+    // later TMEM stores (P over the buffer's first columns).
+    auto exchange = [&](float v, bool& good, float none) -> float {
+      good = true;
+      if constexpr (Cfg::HALVES == 1) return none;
+      const int buf = ex & 1;
+      xt[(buf * Cfg::HALVES + hf) * ROWS + r] = v;
+      tmem_fence_before_sync();
+      mbar_arrive(&xchg[2 * t + buf]);
+      good = __all_sync(0xffffffffu, mbar_wait_bounded(&xchg[2 * t + buf], (ex >> 1) & 1, a.dev_err));
+      tmem_fence_after_sync();
+      const float other = xt[(buf * Cfg::HALVES + (1 - hf)) * ROWS + r];
+      ++ex;
+      return other;
+    };
     for (int idx = k_begin; idx < k_end && ok; ++idx) {
       const TcItem x = tc_item<Cfg>(pf, idx, TQ);
       if (t >= x.ntiles) continue;                         // no row of this tile is a query row
@@ -473,38 +516,53 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       const int jq = t * TQ + r / G;                       // query token within the item
       const bool valid = (r / G) < TQ && jq < it.q_count;
       const int lim = valid ? it.p0 + jq : -1;             // last token this row attends to
-      float m_used = -INFINITY, l = 0.f;
+      float m_used = -INFINITY, l = 0.f;                   // m_used: the same in both halves
       for (int j = 0; j < nchunks; ++j) {
         const int c = cb + j;
         const int b = c & 1;
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[2 * t + b], (c >> 1) & 1, a.dev_err));
         if (!ok) break;
         tmem_fence_after_sync();
-        float sv[CHUNK];
-        tmem_ld64(trow + b * CHUNK, sv);
-        const int c0 = x.span0 + j * CHUNK;
-        // Scaled logits: x = s * scale * log2(e). Only chunks that reach past
-        // the row's position or the span's end need the mask.
-        const bool whole = c0 + CHUNK <= span_end && c0 + CHUNK - 1 <= lim && sl2 > 0.f;
+        float sv[HALF_CHUNK];
+        if constexpr (Cfg::HALVES == 2) {
+          tmem_ld32(trow + b * CHUNK + hf * HALF_CHUNK, sv);
+        } else {
+          tmem_ld64(trow + b * CHUNK, sv);
+        }
+        const int c0 = x.span0 + j * CHUNK + hf * HALF_CHUNK;  // this half's first token
+        // Scaled logits: x = s * scale * log2(e). Only a chunk that reaches
+        // past the row's position or the span's end needs the mask.
+        const int chunk_last = x.span0 + j * CHUNK + CHUNK - 1;
+        const bool whole = chunk_last < span_end && chunk_last <= lim && sl2 > 0.f;
         float mx;
         if (whole) {
-          float m8[8];
+          constexpr int NG = HALF_CHUNK / 8;
+          float mg[NG];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
+          for (int k = 0; k < NG; ++k) {
             const float* v = sv + 8 * k;
-            m8[k] = fmax3(fmax3(v[0], v[1], v[2]), fmax3(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+            mg[k] = fmax3(fmax3(v[0], v[1], v[2]), fmax3(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
           }
-          mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
+          mx = mg[0];
+#pragma unroll
+          for (int k = 1; k < NG; ++k) mx = fmaxf(mx, mg[k]);
+          mx *= sl2;
         } else {
           mx = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < CHUNK; ++i) {
+          for (int i = 0; i < HALF_CHUNK; ++i) {
             const int tk = c0 + i;
             const bool in = tk < span_end && tk <= lim;
             sv[i] = in ? sv[i] * sl2 : -INFINITY;
             mx = fmaxf(mx, sv[i]);
           }
         }
+        // Both halves have read this chunk's logits once the exchange completes,
+        // so P may then be written over the buffer's first 32 columns.
+        bool good;
+        mx = fmaxf(mx, exchange(mx, good, -INFINITY));
+        ok = good;
+        if (!ok) break;
         const bool raise = mx > m_used + Cfg::kRescaleThreshold;
         const bool rescale_o = raise && m_used != -INFINITY;  // only from the item's second chunk on
         if (__any_sync(0xffffffffu, rescale_o)) {
@@ -515,26 +573,27 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
           tmem_fence_after_sync();
           const float alpha = rescale_o ? fast_exp2(m_used - mx) : 1.f;
 #pragma unroll
-          for (int q = 0; q < D / 32; ++q) {
-            float o32[32];
-            tmem_ld32(trow + Cfg::kOCol + q * 32, o32);
+          for (int q = 0; q < HALF_D / 16; ++q) {
+            float o16[16];
+            tmem_ld16(trow + Cfg::kOCol + hf * HALF_D + q * 16, o16);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] *= alpha;
-            tmem_st32(trow + Cfg::kOCol + q * 32, o32);
+            for (int i = 0; i < 16; ++i) o16[i] *= alpha;
+            tmem_st16(trow + Cfg::kOCol + hf * HALF_D + q * 16, o16);
           }
           tmem_fence_before_sync();
           l *= alpha;
         }
         if (raise) m_used = mx;
-        // P = 2^(x - m_used) <= 2^8, as packed bf16 pairs over the logits.
-        uint32_t pk[CHUNK / 2];
+        // P = 2^(x - m_used) <= 2^8, as packed bf16 pairs: this half's 32
+        // tokens go to columns 16 hf .. 16 hf + 15 of the buffer.
+        uint32_t pk[HALF_CHUNK / 2];
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
         if (whole) {
           const uint64_t sl2_2 = f2_pack(sl2, sl2);
           const uint64_t nm2 = f2_pack(-m_used, -m_used);
           uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-          for (int i = 0; i < CHUNK; i += 2) {
+          for (int i = 0; i < HALF_CHUNK; i += 2) {
             const uint64_t x2 = f2_fma(f2_pack(sv[i], sv[i + 1]), sl2_2, nm2);
             float x0, x1;
             f2_unpack(x2, x0, x1);
@@ -550,7 +609,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
         } else {
           const float mu = (m_used == -INFINITY) ? 0.f : m_used;  // a row with nothing yet: all p = 0
 #pragma unroll
-          for (int i = 0; i < CHUNK; i += 2) {
+          for (int i = 0; i < HALF_CHUNK; i += 2) {
             const float p0 = fast_exp2(sv[i] - mu);
             const float p1 = fast_exp2(sv[i + 1] - mu);
             s4[(i >> 1) & 3] += p0 + p1;
@@ -558,7 +617,11 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
           }
         }
         l += (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        tmem_st32_bits(trow + b * CHUNK, pk);
+        if constexpr (Cfg::HALVES == 2) {
+          tmem_st16_bits(trow + b * CHUNK + hf * (HALF_CHUNK / 2), pk);
+        } else {
+          tmem_st32_bits(trow + b * CHUNK, pk);
+        }
         tmem_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[2 * t + b]);
@@ -571,6 +634,12 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
         if (!ok) break;
         tmem_fence_after_sync();
       }
+      {
+        bool good;
+        l += exchange(l, good, 0.f);                       // the row sum over both halves
+        ok = good;
+        if (!ok) break;
+      }
       const int64_t tok = !valid ? it.q_begin
                           : it.out_begin >= 0 ? pf.out_tokens[it.out_begin + jq] : it.q_begin + jq;
       const int64_t h = static_cast<int64_t>(it.kvh) * G + (r % G);
@@ -579,32 +648,35 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       // A full tile of final rows goes out by TMA: its rows (token-major,
       // head-minor, as Q came in) are staged 64 columns at a time in the
       // 128-byte swizzle and stored as one box; one thread per tile issues
-      // the stores. Partial tiles, scattered rows and partials use plain
-      // stores (each thread its own row).
+      // the stores. Each half stages the 16-byte units of its own columns.
+      // Partial tiles, scattered rows and partials use plain stores (each
+      // thread its row's half).
       const bool tma_out = Cfg::kTmaOut && nchunks > 0 && it.final_out && it.out_begin < 0 &&
                            it.q_count >= (t + 1) * TQ;
       if (tma_out) {
         uint8_t* sbuf = stage + t * (ROWS * 128);
-        const bool leader = (warp & 3) == 0 && lane == 0;
+        const bool leader = wt == 0 && lane == 0;
 #pragma unroll
         for (int cc = 0; cc < KCH; ++cc) {
           if (leader) bulk_wait_group_read0();  // the previous store has read the buffer
-          named_bar_sync(1 + t, 128);
+          named_bar_sync(1 + t, Cfg::kTileWarps * 32);
           uint8_t* rowp = sbuf + r * 128;
+          const int lo = max(cc * 64, hf * HALF_D), hi = min(cc * 64 + 64, (hf + 1) * HALF_D);
 #pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
+          for (int col = 0; col < 64; col += 16) {
+            if (cc * 64 + col < lo || cc * 64 + col >= hi) continue;
             float o16[16];
-            tmem_ld16(trow + Cfg::kOCol + cc * 64 + qq * 16, o16);
+            tmem_ld16(trow + Cfg::kOCol + cc * 64 + col, o16);
 #pragma unroll
             for (int p = 0; p < 2; ++p)
-              *reinterpret_cast<uint4*>(rowp + (((qq * 2 + p) ^ (r & 7)) << 4)) =
+              *reinterpret_cast<uint4*>(rowp + ((((col >> 3) + p) ^ (r & 7)) << 4)) =
                   make_uint4(pack_bf16x2(o16[8 * p] * inv, o16[8 * p + 1] * inv),
                              pack_bf16x2(o16[8 * p + 2] * inv, o16[8 * p + 3] * inv),
                              pack_bf16x2(o16[8 * p + 4] * inv, o16[8 * p + 5] * inv),
                              pack_bf16x2(o16[8 * p + 6] * inv, o16[8 * p + 7] * inv));
           }
           fence_proxy_async_smem();
-          named_bar_sync(1 + t, 128);
+          named_bar_sync(1 + t, Cfg::kTileWarps * 32);
           if (leader) {
             tma_store_3d(&tm_o, sbuf, cc * 64, it.q_head0, it.q_begin + t * TQ);
             bulk_commit_group();
@@ -613,32 +685,33 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       }
       if (!tma_out) {
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          float o32[32];
+        for (int q = 0; q < HALF_D / 16; ++q) {
+          const int col = hf * HALF_D + q * 16;
+          float o16[16];
           if (nchunks > 0) {
-            tmem_ld32(trow + Cfg::kOCol + q * 32, o32);
+            tmem_ld16(trow + Cfg::kOCol + col, o16);
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = 0.f;
+            for (int i = 0; i < 16; ++i) o16[i] = 0.f;
           }
           if (!valid) continue;
           if (it.final_out) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * D + q * 32);
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * D + col);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              dst[i] = make_uint4(pack_bf16x2(o16[8 * i] * inv, o16[8 * i + 1] * inv),
+                                  pack_bf16x2(o16[8 * i + 2] * inv, o16[8 * i + 3] * inv),
+                                  pack_bf16x2(o16[8 * i + 4] * inv, o16[8 * i + 5] * inv),
+                                  pack_bf16x2(o16[8 * i + 6] * inv, o16[8 * i + 7] * inv));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(a.part_acc + (row * a.max_partitions + it.part) * D + col);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pack_bf16x2(o32[8 * i] * inv, o32[8 * i + 1] * inv),
-                                  pack_bf16x2(o32[8 * i + 2] * inv, o32[8 * i + 3] * inv),
-                                  pack_bf16x2(o32[8 * i + 4] * inv, o32[8 * i + 5] * inv),
-                                  pack_bf16x2(o32[8 * i + 6] * inv, o32[8 * i + 7] * inv));
-          } else {
-            float4* dst = reinterpret_cast<float4*>(a.part_acc + (row * a.max_partitions + it.part) * D + q * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(o32[4 * i], o32[4 * i + 1], o32[4 * i + 2], o32[4 * i + 3]);
+              dst[i] = make_float4(o16[4 * i], o16[4 * i + 1], o16[4 * i + 2], o16[4 * i + 3]);
           }
         }
       }
-      if (valid && !it.final_out) {
+      if (valid && !it.final_out && hf == 0) {
         a.part_m[row * a.max_partitions + it.part] = m_used;
         a.part_l[row * a.max_partitions + it.part] = l;
       }
@@ -652,7 +725,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     }
   }
   // Output stores complete before the CTA (and its staging memory) ends.
-  if (Cfg::kTmaOut && warp < SMW && (warp & 3) == 0 && lane == 0) bulk_wait_group0();
+  if (Cfg::kTmaOut && warp < SMW && warp % Cfg::kTileWarps == 0 && lane == 0) bulk_wait_group0();
   tmem_fence_before_sync();
   __syncthreads();
   if (warp == 0) {

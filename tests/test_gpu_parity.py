@@ -357,8 +357,9 @@ def test_repeated_split_calls_reuse_workspace():
 
 def test_host_validation_flag_rejects_bad_tables():
     """PAGEDKV_VALIDATE=1 copies the tables and lengths to the host and rejects
-    an out-of-range entry before launching (the flag is read once per
-    process, so the check runs in a child)."""
+    an out-of-range entry before launching, and refuses copy lists with a
+    repeated destination or a block that is both source and destination (the
+    flag is read once per process, so the check runs in a child)."""
     import subprocess
     import sys
     import textwrap
@@ -380,6 +381,15 @@ def test_host_validation_flag_rejects_bad_tables():
         except binding.InvalidArgumentError as e:
             assert "block_tables[1][0]" in str(e), e
             print("rejected")
+        # copy lists whose result would depend on the order of the copies
+        assert w.num_blocks > 6
+        binding.copy_blocks(k, v, torch.tensor([[0, 5], [1, 6]], device="cuda"))   # fine
+        for pairs, why in (([[0, 5], [1, 5]], "twice"), ([[0, 5], [5, 6]], "both a source")):
+            try:
+                binding.copy_blocks(k, v, torch.tensor(pairs, device="cuda"))
+            except binding.InvalidArgumentError as e:
+                assert why in str(e), e
+                print("pairs rejected")
     """) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
             os.path.dirname(os.path.abspath(__file__)))
     env = dict(os.environ, PAGEDKV_VALIDATE="1")
@@ -387,3 +397,4 @@ def test_host_validation_flag_rejects_bad_tables():
                        timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     assert "rejected" in r.stdout
+    assert r.stdout.count("pairs rejected") == 2

@@ -21,7 +21,10 @@ pytestmark = pytest.mark.gpu
 # "tcgen05_3ctas": the tcgen05 kernel's persistent launch capped at 3 CTAs,
 # so that every CTA runs many items back to back (idle second tiles, empty
 # spans, partial last chunks and partition items in one CTA's sequence).
-KERNELS = ["tcgen05", "tcgen05_3ctas", "mma_sync"]
+# "tcgen05_halves" / "tcgen05_halves_3ctas": the tcgen05 kernel with two
+# softmax threads per query row (PAGEDKV_PREFILL_HALVES=2), full grid and
+# capped at 3 CTAs.
+KERNELS = ["tcgen05", "tcgen05_3ctas", "tcgen05_halves", "tcgen05_halves_3ctas", "mma_sync"]
 
 
 @pytest.fixture(params=KERNELS)
@@ -30,10 +33,14 @@ def kernel(request, monkeypatch):
         monkeypatch.setenv("PAGEDKV_PREFILL_KERNEL", "mma_sync")
     else:
         monkeypatch.delenv("PAGEDKV_PREFILL_KERNEL", raising=False)
-    if request.param == "tcgen05_3ctas":
+    if request.param.endswith("_3ctas"):
         monkeypatch.setenv("PAGEDKV_PREFILL_CTAS", "3")
     else:
         monkeypatch.delenv("PAGEDKV_PREFILL_CTAS", raising=False)
+    if request.param.startswith("tcgen05_halves"):
+        monkeypatch.setenv("PAGEDKV_PREFILL_HALVES", "2")
+    else:
+        monkeypatch.delenv("PAGEDKV_PREFILL_HALVES", raising=False)
     return request.param
 
 

@@ -4,7 +4,10 @@ hand-over protocol (csrc/tc_prefill_kernel.cuh), run on the CPU.
 Each CTA role is a generator that follows the kernel's loops and running
 counts: the producer (K/V ring, partial-chunk V clears), the two MMA
 issuers (Q copies, S and P V MMAs, commits) and the two tiles' softmax
-warps (P, epilogue). Barriers count arrivals and completed phases as
+warps (P, epilogue), two per tile since each row's 64 logits are split
+between two threads of different warps: the halves swap their row maxima
+every chunk (and their row sums at an item's end) through a double-buffered
+exchange completed by an mbarrier. Barriers count arrivals and completed phases as
 mbarriers do. TMA copies and tensor-core work finish after random delays.
 MMAs are ordered only where tcgen05 orders them: those accumulating into the
 same TMEM region run in issue order; others may overlap or overtake one
@@ -39,28 +42,35 @@ class Bar:
             self.pending = self.count
 
 
-def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True, s_waits_p_free=True):
+def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True, s_waits_p_free=True,
+             exchange_wait=True):
     """items: (chunks, active tiles, partial last chunk) per item, in one
     CTA's order. Returns None, or a description of the first fault."""
     rnd = random.Random(seed)
     kv_full = [Bar(f"kv_full{i}", 1) for i in range(nslot)]
     kv_empty = [Bar(f"kv_empty{i}", tiles) for i in range(nslot)]
     s_full = [Bar(f"s_full{i}", 1) for i in range(4)]
-    p_full = [Bar(f"p_full{i}", 4) for i in range(4)]
+    p_full = [Bar(f"p_full{i}", 8) for i in range(4)]
     p_free = [Bar(f"p_free{i}", 1) for i in range(4)]
     q_full = [Bar(f"q_full{i}", 1) for i in range(2)]
     q_free = [Bar(f"q_free{i}", 1) for i in range(2)]
     o_last = [Bar(f"o_last{i}", 1) for i in range(2)]
-    o_empty = [Bar(f"o_empty{i}", 4) for i in range(2)]
+    o_empty = [Bar(f"o_empty{i}", 8) for i in range(2)]
     mma_done = [Bar(f"mma_done{i}", 1) for i in range(2)]
     v_tail = Bar("v_tail", 1)
+    # the two halves of a tile's softmax swap their row maxima (and, at an
+    # item's end, their row sums) through a double-buffered exchange; one
+    # arrival here stands for the 128 threads of a half
+    xchg = [Bar(f"xchg{i}", 2) for i in range(4)]
+    xval = {}                          # (tile, buffer, half) -> (exchange written, read yet)
 
     now = [0]
     events, seq = [], [0]
     last_of = {}
     s_end, o_read = {}, {}
     slot_read_end = {}                 # ring slot -> end of the last MMA reading it
-    sm_done, pv_end = {}, {}           # (tile, chunk) -> softmax finished / its P V ended
+    sm_done, pv_end = {}, {}           # (tile, chunk[, half]) -> softmax finished / its P V ended
+    s_read = {}                        # (tile, chunk, half) -> that half read its logits
     tail_cleared = {}                  # ring index of a partial chunk's V -> time cleared
     faults = []
 
@@ -145,7 +155,8 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True, s_wai
                 if c >= 2 and s_waits_p_free:
                     yield wait(p_free[2 * t + (c & 1)], (c >> 1) - 1)
                 start, end = mma(tid, rnd.randint(200, 500), ("S", t, c & 1))
-                if c >= 2 and start < max(sm_done.get((t, c - 2), 1 << 60), pv_end.get((t, c - 2), 1 << 60)):
+                done = max(sm_done.get((t, c - 2, h), 1 << 60) for h in (0, 1))
+                if c >= 2 and start < max(done, pv_end.get((t, c - 2), 1 << 60)):
                     faults.append(f"tile {t}: S({c}) overwrote a buffer still in use for chunk {c - 2}")
                 reads_slot(gi % nslot, end)
                 s_end[t] = max(s_end.get(t, 0), end)
@@ -178,7 +189,7 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True, s_wai
                 if j == 0 and nt > 0:
                     yield wait(o_empty[t], nt - 1)
                 start, end = mma(tid, rnd.randint(150, 400), ("O", t))
-                if j == 0 and nt > 0 and start < o_read[(t, nt - 1)]:
+                if j == 0 and nt > 0 and start < max(o_read[(t, nt - 1, h)] for h in (0, 1)):
                     faults.append(f"tile {t}: O overwritten before the epilogue read it")
                 if tail and j == nch - 1 and start < tail_cleared.get(gi, 1 << 60):
                     faults.append(f"tile {t}: P V read a partial chunk's V before it was cleared")
@@ -196,36 +207,67 @@ def simulate(items, nslot, tiles, seed, tail_guard=True, q_free_wait=True, s_wai
         commit(tid, mma_done[t])
         yield wait(mma_done[t], 0)
 
-    def softmax(t):
-        cb = nt = 0
+    def softmax(t, hf):
+        cb = nt = ex = 0
+        other = 1 - hf
+
+        def exchange():
+            nonlocal ex
+            b = ex & 1
+            prev = xval.get((t, b, hf))
+            if prev is not None and not prev[1]:
+                faults.append(f"tile {t} half {hf}: exchange {ex} overwrites exchange {prev[0]} "
+                              f"before the other half read it")
+            xval[(t, b, hf)] = (ex, False)
+            xchg[2 * t + b].arrive()
+            if exchange_wait:
+                yield wait(xchg[2 * t + b], ex >> 1)
+            yield ("delay", rnd.randint(0, 200))
+            got = xval.get((t, b, other))
+            if got is None or got[0] != ex:
+                faults.append(f"tile {t} half {hf}: read {got} at exchange {ex}")
+            else:
+                xval[(t, b, other)] = (got[0], True)
+            ex += 1
+
         for nch, ntiles, _ in items:
             if t >= ntiles:
                 continue
             for j in range(nch):
                 c = cb + j
                 yield wait(s_full[2 * t + (c & 1)], c >> 1)
-                yield ("delay", rnd.randint(300, 1600))
-                if j >= 1 and rnd.random() < 0.1:  # a rescale of O
+                yield ("delay", rnd.randint(100, 500))       # read this half's logits
+                s_read[(t, c, hf)] = now[0]
+                yield from exchange()                        # row maximum
+                yield ("delay", rnd.randint(150, 800))
+                if j >= 1 and rnd.random() < 0.1:  # a rescale of O (this half's columns)
                     yield wait(p_free[2 * t + ((c - 1) & 1)], (c - 1) >> 1)
                     if now[0] < pv_end.get((t, c - 1), 1 << 60):
                         faults.append(f"tile {t}: O rescaled while P V({c - 1}) still accumulates")
                     yield ("delay", 100)
-                sm_done[(t, c)] = now[0]
+                # P is written over the first half of the buffer: the other
+                # half's logits there must have been read already
+                if s_read.get((t, c, other), 1 << 60) > now[0]:
+                    faults.append(f"tile {t} chunk {c}: half {hf} writes P before half {other} "
+                                  f"read its logits")
+                sm_done[(t, c, hf)] = now[0]
                 for _ in range(4):
                     p_full[2 * t + (c & 1)].arrive()
             if nch > 0:
                 yield wait(o_last[t], nt)
+            yield from exchange()                            # row sums
             yield ("delay", rnd.randint(100, 800))
             if nch > 0:
-                o_read[(t, nt)] = now[0]
+                o_read[(t, nt, hf)] = now[0]
                 for _ in range(4):
                     o_empty[t].arrive()
                 cb += nch
                 nt += 1
 
-    roles = {"producer": producer(), "issuer0": issuer(0), "softmax0": softmax(0)}
+    roles = {"producer": producer(), "issuer0": issuer(0), "softmax0a": softmax(0, 0),
+             "softmax0b": softmax(0, 1)}
     if tiles == 2:
-        roles.update({"issuer1": issuer(1), "softmax1": softmax(1)})
+        roles.update({"issuer1": issuer(1), "softmax1a": softmax(1, 0), "softmax1b": softmax(1, 1)})
     state = {n: {"gen": g, "wait": None, "wake": 0, "done": False} for n, g in roles.items()}
     while True:
         progressed = True
@@ -281,7 +323,7 @@ def random_items(rnd, tiles):
     return items
 
 
-@pytest.mark.parametrize("nslot,tiles", [(8, 2), (6, 2), (4, 2), (4, 1)])
+@pytest.mark.parametrize("nslot,tiles", [(8, 2), (7, 2), (6, 2), (4, 2), (4, 1)])
 def test_protocol_has_no_deadlock_lap_or_overwrite(nslot, tiles):
     for trial in range(250):
         rnd = random.Random(1000 * nslot + 10 * tiles + trial)
@@ -313,3 +355,8 @@ def test_model_catches_a_missing_q_free_wait():
 def test_model_catches_an_s_mma_that_skips_the_p_free_wait():
     fault = _first_fault(s_waits_p_free=False)
     assert fault is not None and "overwrote a buffer" in fault
+
+
+def test_model_catches_halves_that_do_not_wait_for_the_exchange():
+    fault = _first_fault(exchange_wait=False)
+    assert fault is not None and ("read" in fault or "overwrites" in fault or "before half" in fault)
