@@ -530,8 +530,9 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
     int bs = r.block_size;
     void* margs[] = {&a, &bs};
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(r.num_seqs * r.num_q_heads));
-    cfg.blockDim = dim3(128);
+    const int64_t merge_rows = static_cast<int64_t>(r.num_seqs) * r.num_q_heads;
+    cfg.gridDim = dim3(static_cast<unsigned>((merge_rows + kMergeRowsPerCta - 1) / kMergeRowsPerCta));
+    cfg.blockDim = dim3(32 * kMergeRowsPerCta);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = r.stream;
     cudaLaunchAttribute attr[1];
@@ -1266,8 +1267,9 @@ pa_status_t run_prefill(const DecodeReq& r_in, const int32_t* ctx_host, const in
     int bs = r.block_size;
     void* margs[] = {&a, &bs};
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(total_q) * r.num_q_heads);
-    cfg.blockDim = dim3(128);
+    const int64_t merge_rows = static_cast<int64_t>(total_q) * r.num_q_heads;
+    cfg.gridDim = dim3(static_cast<unsigned>((merge_rows + kMergeRowsPerCta - 1) / kMergeRowsPerCta));
+    cfg.blockDim = dim3(32 * kMergeRowsPerCta);
     cfg.stream = r.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -879,77 +879,90 @@ __global__ void __launch_bounds__(Cfg::kThreads)
   }
 }
 
-// Log-sum-exp merge of partition partials. One CTA (4 warps) per (sequence,
-// query head) with more than one partition; single-partition sequences were
-// written by the decode kernel. All threads find M = max_p m_p and
-// L = sum_p l_p 2^(m_p - M); warp w accumulates partitions p = w, w+4, ...,
-// eight loads in flight per lane; the four partial sums meet in shared memory:
-//   out = sum_p acc_p 2^(m_p - M) / L.
+// Log-sum-exp merge of partition partials. One warp per (sequence, query
+// head) row with more than one partial (rows with one were written by the
+// decode kernel), four rows per CTA; no shared memory and no CTA barrier.
+// Lane i holds partition p = i (and i + 32, ...)'s m_p and l_p: the warp
+// finds M = max_p m_p and L = sum_p l_p 2^(m_p - M) by shuffles. Each lane
+// owns head_dim / 32 columns of the output and accumulates
+// out = sum_p acc_p 2^(m_p - M) / L with the weights broadcast from the
+// lanes that hold them; the partials' loads are issued eight partitions at a
+// time, so a row costs about two dependent round trips to L2.
+constexpr int kMergeRowsPerCta = 4;
+
+// VEC consecutive floats (VEC * 4 bytes aligned) in 8- or 16-byte loads.
+template <int VEC>
+__device__ __forceinline__ void load_f32s(const float* p, float (&v)[VEC]) {
+  if constexpr (VEC % 4 == 0) {
+#pragma unroll
+    for (int q = 0; q < VEC / 4; ++q) {
+      const float4 x = reinterpret_cast<const float4*>(p)[q];
+      v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+    }
+  } else {
+    static_assert(VEC == 2, "head_dim 64, 128 or 256");
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x; v[1] = x.y;
+  }
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(32 * kMergeRowsPerCta)
     lse_merge_kernel(const DecodeArgs a, int block_size) {
   constexpr int VEC = D / 32;
   constexpr int UNROLL = 8;
-  __shared__ float red[4];
-  __shared__ float accs[4][D];
   grid_dependency_wait();  // the decode grid's partials are complete and visible
-  const int row = blockIdx.x;  // s * Hq + h
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = row / a.num_q_heads;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kMergeRowsPerCta + (threadIdx.x >> 5);
+  if (row >= static_cast<int64_t>(a.num_seqs) * a.num_q_heads) return;
+  const int s = static_cast<int>(row / a.num_q_heads);
   const int base_parts = a.seq_part_base ? a.seq_part_base[s] : 0;
   const int own = a.seg_pieces != nullptr
                       ? a.seg_pieces[static_cast<int64_t>(s) * a.num_kv_heads +
-                                     (row - s * a.num_q_heads) / a.group]
+                                     (row - static_cast<int64_t>(s) * a.num_q_heads) / a.group]
                       : seq_partitions(a, s, a.max_blocks_per_seq * block_size, block_size);
   const int np = min(base_parts + own, a.max_partitions);
   if (np <= 1 && base_parts == 0) return;
-  const int64_t base = static_cast<int64_t>(row) * a.max_partitions;
+  const int64_t base = row * a.max_partitions;
   float M = -INFINITY;
-  for (int p = tid; p < np; p += 128) M = fmaxf(M, a.part_m[base + p]);
+  for (int p = lane; p < np; p += 32) M = fmaxf(M, a.part_m[base + p]);
   M = warp_max(M);
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();
   float L = 0.f;
-  for (int p = tid; p < np; p += 128) L += a.part_l[base + p] * fast_exp2(a.part_m[base + p] - M);
+  for (int p = lane; p < np; p += 32) L += a.part_l[base + p] * fast_exp2(a.part_m[base + p] - M);
   L = warp_sum(L);
-  if (lane == 0) red[warp] = L;
   float acc[VEC];
 #pragma unroll
   for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
   const float* src = a.part_acc + base * D + lane * VEC;
-  int p = warp;
-  for (; p + 4 * (UNROLL - 1) < np; p += 4 * UNROLL) {
-    float v[UNROLL][VEC];
-    float e[UNROLL];
+  for (int p0 = 0; p0 < np; p0 += 32) {
+    // this lane's weight for partition p0 + lane, broadcast below
+    const float wl = (p0 + lane < np) ? fast_exp2(a.part_m[base + p0 + lane] - M) : 0.f;
+    const int n = min(32, np - p0);
+    int k = 0;
+    for (; k + UNROLL <= n; k += UNROLL) {
+      float v[UNROLL][VEC];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int pp = p + 4 * u;
-      e[u] = a.part_m[base + pp];
+      for (int u = 0; u < UNROLL; ++u)
+        load_f32s<VEC>(src + static_cast<int64_t>(p0 + k + u) * D, v[u]);
 #pragma unroll
-      for (int j = 0; j < VEC; ++j) v[u][j] = src[static_cast<int64_t>(pp) * D + j];
+      for (int u = 0; u < UNROLL; ++u) {
+        const float w = __shfl_sync(0xffffffffu, wl, k + u);
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) acc[j] = fmaf(v[u][j], w, acc[j]);
+      }
     }
+    for (; k < n; ++k) {
+      float v[VEC];
+      load_f32s<VEC>(src + static_cast<int64_t>(p0 + k) * D, v);
+      const float w = __shfl_sync(0xffffffffu, wl, k);
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const float w = fast_exp2(e[u] - M);
-#pragma unroll
-      for (int j = 0; j < VEC; ++j) acc[j] = fmaf(v[u][j], w, acc[j]);
+      for (int j = 0; j < VEC; ++j) acc[j] = fmaf(v[j], w, acc[j]);
     }
   }
-  for (; p < np; p += 4) {
-    const float w = fast_exp2(a.part_m[base + p] - M);
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) acc[j] = fmaf(src[static_cast<int64_t>(p) * D + j], w, acc[j]);
-  }
-#pragma unroll
-  for (int j = 0; j < VEC; ++j) accs[warp][lane * VEC + j] = acc[j];
-  __syncthreads();
-  L = red[0] + red[1] + red[2] + red[3];
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
-  T* dst = reinterpret_cast<T*>(a.out) + static_cast<int64_t>(row) * D;
-  for (int d = tid; d < D; d += 128)
-    dst[d] = Elt<T>::from_f32((accs[0][d] + accs[1][d] + accs[2][d] + accs[3][d]) * inv);
+  T* dst = reinterpret_cast<T*>(a.out) + row * D + lane * VEC;
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) dst[j] = Elt<T>::from_f32(acc[j] * inv);
 }
 
 }  // namespace pagedkv
