@@ -104,14 +104,25 @@ pa_status_t pa_decode(const void* q, const void* k_pool, const void* v_pool,
                       void* stream);
 
 /* ---------------------------------------------------------------------------
- * pa_decode_split - the same result as pa_decode, computed by cutting each
- * context into partitions of partition_tokens tokens (a multiple of
- * block_size). Each (sequence, KV head, partition) produces a running max, a
- * running sum and an unnormalised accumulator; a log-sum-exp merge combines
- * the partitions. Sequences that fit in one partition are written directly.
+ * pa_decode_split - the same result as pa_decode, computed by cutting the
+ * contexts into pieces. Each (sequence, KV head, piece) produces a running
+ * max, a running sum and an unnormalised accumulator; a log-sum-exp merge
+ * combines the pieces, and a sequence held in one piece is written directly.
  * The split is a scheduling device for long and ragged contexts; it does not
  * appear on the pages, which only require that the blockwise walk reproduce
- * the contiguous result ([G] section 3).
+ * the contiguous result ([G] section 3). Two cuts, chosen by the table size:
+ *  - tables of fewer than 32768 tokens (max_blocks_per_seq * block_size):
+ *    partitions of partition_tokens tokens (a multiple of block_size),
+ *    handed to persistent CTAs as work tickets;
+ *  - longer tables: every warp of a persistent grid takes an equal run of
+ *    16-token units of one KV head's work, sequence after sequence, so the
+ *    piece boundaries follow the whole batch; partition_tokens then only
+ *    bounds the pieces: no (sequence, KV head) is cut into more than
+ *    ceil(max_blocks_per_seq / (partition_tokens / block_size)) + 1.
+ *   (PAGEDKV_SPLIT_KERNEL=ticket|stream forces one cut.) Both give the
+ *   contiguous result to rounding; with the second, the rounding of one
+ *   sequence can depend on the rest of the batch. Same inputs give the same
+ *   bits.
  *
  * workspace: caller-owned device memory of at least
  *   pa_decode_split_workspace_size(...) bytes, 256-byte aligned. It starts
@@ -121,9 +132,9 @@ pa_status_t pa_decode(const void* q, const void* k_pool, const void* v_pool,
  *   workspace serves any number of calls issued in stream order. Calls that
  *   may overlap on the GPU need separate workspaces. After a call that
  *   reported PA_DEVERR_TIMEOUT, initialise the workspace again.
- * Two kernels run: the partition kernel, then (when some sequence has more
- *   than one partition) the merge kernel, launched as a programmatic
- *   dependent so that it waits on the device rather than in the launch queue.
+ * Two kernels run: the decode kernel, then the merge kernel, launched as a
+ *   programmatic dependent so that it waits on the device rather than in the
+ *   launch queue (rows held in one piece return at once).
  * num_seqs must be <= 4096 (PA_ERR_UNSUPPORTED above that).
  * ------------------------------------------------------------------------- */
 size_t pa_decode_split_workspace_size(int num_seqs, int num_q_heads, int head_dim,
