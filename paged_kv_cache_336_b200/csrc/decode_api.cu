@@ -369,13 +369,17 @@ struct SplitExtras {
 //  * partition tickets (each CTA pulls 512-token items; the warps of a CTA
 //    split an item) stream MHA batch 64 / GQA batch 256 at 0.94 / 0.93
 //    against 0.91 / 0.90, and the shared-prefix suffix pass 10% faster.
-// So tables that can hold 32k tokens or more take the balanced kernel.
-// PAGEDKV_SPLIT_KERNEL=stream|ticket overrides the choice (tests run both).
-bool use_stream_kernel(const DecodeReq& r) {
+// So tables that can hold 32k tokens or more take the balanced kernel, and
+// so does the shared-prefix suffix pass, in a smaller CTA shape that fits
+// beside the prefix kernel's CTAs (prefix_cow call 75.7 us against 84.0 on
+// tickets). PAGEDKV_SPLIT_KERNEL=stream|ticket overrides the choice (tests
+// run both).
+bool use_stream_kernel(const DecodeReq& r, bool suffix_pass) {
   const char* e = std::getenv("PAGEDKV_SPLIT_KERNEL");
   if (e != nullptr && std::strcmp(e, "stream") == 0) return true;
   if (e != nullptr && std::strcmp(e, "ticket") == 0) return false;
-  return static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size >= kDeepContextTokens;
+  return suffix_pass ||
+         static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size >= kDeepContextTokens;
 }
 
 // clear_header: zero the workspace's control header on r.stream right before
@@ -446,7 +450,8 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
     st = device_info(&dinfo);
     if (st != PA_OK) return st;
     int occ = 0;
-    if (use_stream_kernel(r)) {
+    const bool suffix_pass = a.seq_skip_blocks != nullptr;
+    if (use_stream_kernel(r, suffix_pass)) {
       // Balanced pieces per warp (paged_decode_stream_kernel). At most this
       // many pieces per (sequence, KV head): the slots after the prefix
       // pass's (none outside shared-prefix decode).
@@ -458,15 +463,16 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
                                 ((static_cast<int64_t>(r.max_blocks_per_seq) * r.block_size + 15) / 16);
       if (units_max >= (int64_t(1) << 31))
         return fail(PA_ERR_UNSUPPORTED, "num_seqs * max context / 16 must be < 2^31");
-      kernel = inst.stream_kernel;
-      threads = inst.stream_threads;
-      smem = inst.stream_fixed_smem + (2 * r.num_seqs + 1) * 4;
+      const DecodeInstance::Stream& sk = inst.stream[suffix_pass ? 1 : 0];
+      kernel = sk.kernel;
+      threads = sk.threads;
+      smem = sk.fixed_smem + (2 * r.num_seqs + 1) * 4;
       st = prepare_kernel(kernel, smem);
       if (st != PA_OK) return st;
       st = occupancy(kernel, threads, smem, &occ);
       if (st != PA_OK) return st;
       // One warp per KV head and group of units; no more groups than units.
-      const int64_t W = inst.stream_warps;
+      const int64_t W = sk.warps;
       const int64_t need = (units_max * r.num_kv_heads + W - 1) / W;
       const int64_t at_least = (r.num_kv_heads + W - 1) / W;
       const int64_t ctas = std::max(at_least, std::min<int64_t>(need, static_cast<int64_t>(dinfo.sms) * occ));

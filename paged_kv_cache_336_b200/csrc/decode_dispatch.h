@@ -14,11 +14,15 @@ struct DecodeInstance {
   int fixed_smem = 0;            // dynamic smem bytes before the prefix array
   int stages = 0;
   const char* name = "";
-  // Split decode: paged_decode_stream_kernel<Cfg> (balanced pieces per warp).
-  const void* stream_kernel = nullptr;
-  int stream_threads = 0;
-  int stream_fixed_smem = 0;     // dynamic smem bytes before the per-sequence arrays
-  int stream_warps = 0;
+  // Split decode: paged_decode_stream_kernel<Cfg> (balanced pieces per warp),
+  // in two CTA shapes: [0] the long-context one, [1] a smaller one that
+  // shares SMs with a concurrent kernel (the shared-prefix pass).
+  struct Stream {
+    const void* kernel = nullptr;
+    int threads = 0;
+    int fixed_smem = 0;          // dynamic smem bytes before the per-sequence arrays
+    int warps = 0;
+  } stream[2];
 };
 
 // Each returns false when (head_dim, block_size, group) has no instance.

@@ -34,31 +34,48 @@ static DecodeInstance make_bf16(const char* name) {
 }
 
 template <int BS, int D, int W, int NS>
-static void add_stream(DecodeInstance* r) {
+static void add_stream(DecodeInstance* r, int which) {
   using Cfg = DecodeCfg<__nv_bfloat16, BS, D, 0, W, NS>;
-  r->stream_kernel = reinterpret_cast<const void*>(&paged_decode_stream_kernel<Cfg>);
-  r->stream_threads = Cfg::kThreads;
-  r->stream_fixed_smem = StreamCfg<Cfg>::kFixedSmem;
-  r->stream_warps = Cfg::W;
+  DecodeInstance::Stream& st = r->stream[which];
+  st.kernel = reinterpret_cast<const void*>(&paged_decode_stream_kernel<Cfg>);
+  st.threads = Cfg::kThreads;
+  st.fixed_smem = StreamCfg<Cfg>::kFixedSmem;
+  st.warps = Cfg::W;
 }
 
-// Balanced split-decode CTA shape (warps x ring stages of 16-token K+V
-// units); every shape keeps 192 KB of ring per SM at head_dim 128. Default
-// 8 x 3, one CTA per SM: its 8 warps are the 8 KV heads of one group in the
-// long-context batches, reading the same blocks together; measured on the
-// 131072-token batch at 0.988 of the HBM copy peak against 0.962-0.970 for
-// 4 x 2, 4 x 3 and 2 x 3 at the same SM clock. PAGEDKV_STREAM_SHAPE selects
-// another for measurements: "4x3", "4x2", "2x3".
+// Balanced split-decode CTA shapes (warps x ring stages of 16-token K+V
+// units); every shape keeps 192 KB of ring per SM at head_dim 128.
+//  [0] long contexts: 8 x 3, one CTA per SM: its 8 warps are the 8 KV heads
+//      of one group in the long-context batches, reading the same blocks
+//      together; measured on the 131072-token batch at 0.988 of the HBM copy
+//      peak against 0.962-0.970 for 4 x 2, 4 x 3 and 2 x 3 at the same clock.
+//  [1] the shared-prefix suffix pass, which starts beside the prefix kernel:
+//      4 x 2 (64 KB CTAs fit next to its CTAs); the whole prefix_cow call
+//      measured 75.7 us against 77.7 for 2 x 3 and 84.0 on partition tickets.
+// PAGEDKV_STREAM_SHAPE ("4x3", "4x2", "2x3", "8x3") sets both for measurements.
 template <int BS, int D>
 static void pick_stream(DecodeInstance* r) {
   const char* e = std::getenv("PAGEDKV_STREAM_SHAPE");
   if constexpr (D == 256) {
-    add_stream<BS, D, 4, 2>(r);
+    add_stream<BS, D, 4, 2>(r, 0);
+    add_stream<BS, D, 4, 2>(r, 1);
   } else {
-    if (e != nullptr && std::strcmp(e, "4x2") == 0) add_stream<BS, D, 4, 2>(r);
-    else if (e != nullptr && std::strcmp(e, "2x3") == 0) add_stream<BS, D, 2, 3>(r);
-    else if (e != nullptr && std::strcmp(e, "4x3") == 0) add_stream<BS, D, 4, 3>(r);
-    else add_stream<BS, D, 8, 3>(r);
+    if (e != nullptr && std::strcmp(e, "4x2") == 0) {
+      add_stream<BS, D, 4, 2>(r, 0);
+      add_stream<BS, D, 4, 2>(r, 1);
+    } else if (e != nullptr && std::strcmp(e, "2x3") == 0) {
+      add_stream<BS, D, 2, 3>(r, 0);
+      add_stream<BS, D, 2, 3>(r, 1);
+    } else if (e != nullptr && std::strcmp(e, "4x3") == 0) {
+      add_stream<BS, D, 4, 3>(r, 0);
+      add_stream<BS, D, 4, 3>(r, 1);
+    } else if (e != nullptr && std::strcmp(e, "8x3") == 0) {
+      add_stream<BS, D, 8, 3>(r, 0);
+      add_stream<BS, D, 8, 3>(r, 1);
+    } else {
+      add_stream<BS, D, 8, 3>(r, 0);
+      add_stream<BS, D, 4, 2>(r, 1);
+    }
   }
 }
 

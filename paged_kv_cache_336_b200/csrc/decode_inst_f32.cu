@@ -15,10 +15,12 @@ static DecodeInstance make_f32() {
   r.fixed_smem = Cfg::kFixedSmem;
   r.stages = Cfg::NS;
   r.name = "simt_f32";
-  r.stream_kernel = reinterpret_cast<const void*>(&paged_decode_stream_kernel<Cfg>);
-  r.stream_threads = Cfg::kThreads;
-  r.stream_fixed_smem = StreamCfg<Cfg>::kFixedSmem;
-  r.stream_warps = Cfg::W;
+  for (DecodeInstance::Stream& st : r.stream) {
+    st.kernel = reinterpret_cast<const void*>(&paged_decode_stream_kernel<Cfg>);
+    st.threads = Cfg::kThreads;
+    st.fixed_smem = StreamCfg<Cfg>::kFixedSmem;
+    st.warps = Cfg::W;
+  }
   return r;
 }
 

@@ -19,8 +19,8 @@
 //   for KV head h = w % Hkv, in group g = w / Hkv, on units [g*C, (g+1)*C)
 //   of h's list, with C = max(ceil(U_h / groups), ceil(U_max / (P - 1))):
 //   every warp streams the same bytes (no tickets, no tail of uneven
-//   items), and no segment of U_max units or fewer is cut into more than P
-//   pieces (the partial slots the workspace holds). The Hkv warps of a group
+//   items), and no segment (at most U_max units) is cut into more than P
+//   pieces, the partial slots the workspace holds. The Hkv warps of a group
 //   read the same blocks' tiles for different KV heads at the same time, so
 //   the DRAM pages of a block ([Hkv][block_size][head_dim] contiguous) are
 //   read together.
