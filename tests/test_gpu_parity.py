@@ -398,3 +398,56 @@ def test_host_validation_flag_rejects_bad_tables():
     assert r.returncode == 0, r.stderr[-2000:]
     assert "rejected" in r.stdout
     assert r.stdout.count("pairs rejected") == 2
+
+
+@pytest.mark.parametrize("Hq,Hkv,dtype", [(6, 3, workloads.BF16), (32, 32, workloads.BF16),
+                                          (16, 16, workloads.F32), (40, 5, workloads.BF16)])
+def test_balanced_split_kv_head_counts(Hq, Hkv, dtype):
+    """The balanced kernel's warp groups are Hkv warps wide: KV-head counts
+    that do not divide a CTA's warps (3, 5), and ones larger than a CTA (16,
+    32), against the oracle (the kernel forced for these short tables)."""
+    os.environ["PAGEDKV_SPLIT_KERNEL"] = "stream"
+    try:
+        w = workloads.random_small(120 + Hkv, num_seqs=5, num_q_heads=Hq, num_kv_heads=Hkv,
+                                   head_dim=128, block_size=16, dtype=dtype, max_ctx=900,
+                                   fixed_lens=[0, 1, 900])
+        bm, k_pool, v_pool = setup(w)
+        q = workloads.draw_queries(w, 5, device="cuda")
+        bt, ctx, tables, ctx_np = device_tables(bm, list(range(5)))
+        err = _err_word()
+        out = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=64,
+                                   dev_err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        check_close(to_f64(out), _full_oracle(q, k_pool, v_pool, tables, ctx_np, w.scale), dtype,
+                    f"Hq={Hq} Hkv={Hkv}")
+    finally:
+        os.environ.pop("PAGEDKV_SPLIT_KERNEL", None)
+
+
+def test_balanced_split_many_sequences():
+    """4096 sequences (the most pa_decode_split takes) of 0..40 tokens in
+    tables that hold 32768 tokens: the per-sequence arrays fill the balanced
+    kernel's shared memory; every output against the oracle."""
+    B, bs, mbs = 4096, 16, 2048
+    rng = np.random.default_rng(77)
+    ctx_np = rng.integers(0, 41, size=B).astype(np.int32)
+    nb = int(np.sum((ctx_np + bs - 1) // bs)) + 8
+    order = rng.permutation(nb).astype(np.int32)
+    bm = BlockManager(nb, bs, mbs, order)
+    for s in range(B):
+        bm.allocate(s, int(ctx_np[s]))
+    w = workloads.random_small(78, num_seqs=1, num_q_heads=4, num_kv_heads=2, head_dim=128,
+                               block_size=bs, dtype=workloads.BF16, max_ctx=1)
+    w.num_blocks = nb
+    k_pool, v_pool = workloads.draw_pools(w, "cuda")
+    q = workloads.draw_queries(w, B, device="cuda")
+    bt, ctx, tables, ctx2 = device_tables(bm, list(range(B)))
+    err = _err_word()
+    out = binding.decode_split(q, k_pool, v_pool, bt, ctx, w.scale, partition_tokens=512,
+                               dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    check_close(to_f64(out), _full_oracle(q, k_pool, v_pool, tables, ctx2, w.scale), w.dtype,
+                "4096 sequences")
+    assert torch.all(out[torch.from_numpy(ctx2 == 0).cuda()] == 0)
