@@ -828,7 +828,13 @@ pa_status_t run_shared_prefix(const DecodeReq& r, int partition_tokens, int num_
   // each; fewer partitions mean fewer partials for the merge. Rounding up the
   // partitions of each group can overflow the wave, so the size grows until
   // the items fit (a second, nearly empty wave costs a whole item's time).
-  const int per_sm = tc ? 2 : 3;
+  int per_sm = tc ? 2 : 3;
+  if (!tc) {
+    st = prepare_kernel(pinst.kernel, pinst.smem);
+    if (st != PA_OK) return st;
+    st = occupancy(pinst.kernel, pinst.threads, pinst.smem, &per_sm);
+    if (st != PA_OK) return st;
+  }
   const int64_t slots = static_cast<int64_t>(per_sm) * dinfo.sms;
   int pbp = static_cast<int>((total_blocks + slots - 1) / slots);
   pbp = std::max(pbp, (max_blocks + kMaxPrefixParts - 1) / kMaxPrefixParts);

@@ -101,14 +101,26 @@ bool find_decode_bf16_mma(int head_dim, int block_size, bool deep, DecodeInstanc
   return false;
 }
 
-template <int BS, int D>
-static PrefixInstance make_prefix() {
-  using Cfg = PrefixCfg<BS, D>;
+template <int BS, int D, int MINB>
+static PrefixInstance make_prefix_minb() {
+  using Cfg = PrefixCfg<BS, D, MINB>;
   PrefixInstance r;
   r.kernel = reinterpret_cast<const void*>(&prefix_decode_kernel<Cfg>);
   r.threads = Cfg::kThreads;
   r.smem = Cfg::kSmem;
   return r;
+}
+
+// The prefix kernel's registers are sized for two CTAs per SM: 168 per
+// thread and no spills at head_dim 128, against 128 and 72 bytes of spills
+// for three. Measured on the shared-prefix calls: prefix 92.3 against
+// 96.4 us, prefix_cow 74.7 against 76.1. PAGEDKV_PREFIX_MINB=3 selects the
+// three-CTA build.
+template <int BS, int D>
+static PrefixInstance make_prefix() {
+  const char* e = std::getenv("PAGEDKV_PREFIX_MINB");
+  if (e != nullptr && std::strcmp(e, "3") == 0) return make_prefix_minb<BS, D, 3>();
+  return make_prefix_minb<BS, D, 2>();
 }
 
 bool find_prefix_bf16(int head_dim, int block_size, PrefixInstance* out) {

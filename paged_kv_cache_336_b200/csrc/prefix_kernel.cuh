@@ -39,8 +39,9 @@ struct PrefixArgs {
   const int32_t* members;   // batch positions, grouped
 };
 
-template <int BS_, int D_>
+template <int BS_, int D_, int MINB_ = 2>
 struct PrefixCfg {
+  static constexpr int MINB = MINB_;  // resident CTAs per SM the registers are sized for
   using Mma = DecodeCfg<__nv_bfloat16, BS_, D_, 0, 4, 2>;  // unit geometry + per-warp math
   using Geo = typename Mma::Geo;
   static constexpr int BS = BS_;
@@ -55,7 +56,7 @@ struct PrefixCfg {
 };
 
 template <class Cfg>
-__global__ void __launch_bounds__(Cfg::kThreads, 3)
+__global__ void __launch_bounds__(Cfg::kThreads, Cfg::MINB)
     prefix_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const PrefixArgs pa) {
   using Geo = typename Cfg::Geo;
