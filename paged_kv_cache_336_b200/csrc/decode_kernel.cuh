@@ -885,9 +885,12 @@ __global__ void __launch_bounds__(Cfg::kThreads)
 // Lane i holds partition p = i (and i + 32, ...)'s m_p and l_p: the warp
 // finds M = max_p m_p and L = sum_p l_p 2^(m_p - M) by shuffles. Each lane
 // owns head_dim / 32 columns of the output and accumulates
-// out = sum_p acc_p 2^(m_p - M) / L with the weights broadcast from the
-// lanes that hold them; the partials' loads are issued eight partitions at a
-// time, so a row costs about two dependent round trips to L2.
+// out = sum_p acc_p 2^(m_p - M) / L in partition order, with the weights
+// broadcast from the lanes that hold them. The accumulators of the first
+// kMergeBatch partitions are loaded together with every m_p and l_p, before
+// M is known, and later ones kMergeBatch at a time, so a row of up to
+// kMergeBatch partials costs one dependent round trip to L2 (two up to
+// 2 * kMergeBatch).
 constexpr int kMergeRowsPerCta = 4;
 
 // VEC consecutive floats (VEC * 4 bytes aligned) in 8- or 16-byte loads.
@@ -910,7 +913,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(32 * kMergeRowsPerCta)
     lse_merge_kernel(const DecodeArgs a, int block_size) {
   constexpr int VEC = D / 32;
-  constexpr int UNROLL = 8;
+  // partitions whose accumulators are in flight at once: 64 floats per lane
+  constexpr int kMergeBatch = 64 / VEC < 32 ? 64 / VEC : 32;
   grid_dependency_wait();  // the decode grid's partials are complete and visible
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kMergeRowsPerCta + (threadIdx.x >> 5);
@@ -924,39 +928,46 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerCta)
   const int np = min(base_parts + own, a.max_partitions);
   if (np <= 1 && base_parts == 0) return;
   const int64_t base = row * a.max_partitions;
-  float M = -INFINITY;
-  for (int p = lane; p < np; p += 32) M = fmaxf(M, a.part_m[base + p]);
+  const float* src = a.part_acc + base * D + lane * VEC;
+
+  // first batch of accumulators, then every partition's m and l
+  float v[kMergeBatch][VEC];
+  const int n_first = min(kMergeBatch, np);
+#pragma unroll
+  for (int u = 0; u < kMergeBatch; ++u)
+    if (u < n_first) load_f32s<VEC>(src + static_cast<int64_t>(u) * D, v[u]);
+  const float m_lane = lane < np ? a.part_m[base + lane] : -INFINITY;
+  const float l_lane = lane < np ? a.part_l[base + lane] : 0.f;
+  float M = m_lane;
+  for (int p = lane + 32; p < np; p += 32) M = fmaxf(M, a.part_m[base + p]);
   M = warp_max(M);
-  float L = 0.f;
-  for (int p = lane; p < np; p += 32) L += a.part_l[base + p] * fast_exp2(a.part_m[base + p] - M);
+  float L = lane < np ? l_lane * fast_exp2(m_lane - M) : 0.f;
+  for (int p = lane + 32; p < np; p += 32) L += a.part_l[base + p] * fast_exp2(a.part_m[base + p] - M);
   L = warp_sum(L);
+
   float acc[VEC];
 #pragma unroll
   for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
-  const float* src = a.part_acc + base * D + lane * VEC;
   for (int p0 = 0; p0 < np; p0 += 32) {
     // this lane's weight for partition p0 + lane, broadcast below
-    const float wl = (p0 + lane < np) ? fast_exp2(a.part_m[base + p0 + lane] - M) : 0.f;
+    const float wl = p0 == 0 ? (lane < np ? fast_exp2(m_lane - M) : 0.f)
+                             : ((p0 + lane < np) ? fast_exp2(a.part_m[base + p0 + lane] - M) : 0.f);
     const int n = min(32, np - p0);
-    int k = 0;
-    for (; k + UNROLL <= n; k += UNROLL) {
-      float v[UNROLL][VEC];
+    for (int k = 0; k < n; k += kMergeBatch) {
+      const int cnt = min(kMergeBatch, n - k);
+      if (p0 + k > 0) {
 #pragma unroll
-      for (int u = 0; u < UNROLL; ++u)
-        load_f32s<VEC>(src + static_cast<int64_t>(p0 + k + u) * D, v[u]);
-#pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        const float w = __shfl_sync(0xffffffffu, wl, k + u);
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) acc[j] = fmaf(v[u][j], w, acc[j]);
+        for (int u = 0; u < kMergeBatch; ++u)
+          if (u < cnt) load_f32s<VEC>(src + static_cast<int64_t>(p0 + k + u) * D, v[u]);
       }
-    }
-    for (; k < n; ++k) {
-      float v[VEC];
-      load_f32s<VEC>(src + static_cast<int64_t>(p0 + k) * D, v);
-      const float w = __shfl_sync(0xffffffffu, wl, k);
 #pragma unroll
-      for (int j = 0; j < VEC; ++j) acc[j] = fmaf(v[j], w, acc[j]);
+      for (int u = 0; u < kMergeBatch; ++u) {
+        if (u < cnt) {
+          const float w = __shfl_sync(0xffffffffu, wl, k + u);
+#pragma unroll
+          for (int j = 0; j < VEC; ++j) acc[j] = fmaf(v[u][j], w, acc[j]);
+        }
+      }
     }
   }
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
