@@ -882,17 +882,31 @@ def run_prefill_bench(args, device_index):
     out = torch.empty_like(q)
     part = args.prefill_partition or -(-(prior + chunk) // bs) * bs
     ws = binding.prefill_workspace(B, B * chunk, Hq, Hkv, D, bs, w.max_blocks_per_seq, part, device)
-    for _ in range(args.warmup):
+    for _ in range(max(3, args.warmup)):
         binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, part, out, ws)
     torch.cuda.synchronize()
+    # Blocks of `reps` back-to-back calls, each bracketed by CUDA events, until
+    # the blocks add up to --min-seconds of device time; the median block.
+    # The kernel is tensor-bound, so its time follows the SM clock: the
+    # line carries the clocks sampled meanwhile.
     reps = max(3, min(args.steps, 200))
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(reps):
-        binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, part, out, ws)
-    t1.record()
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / reps
+    clocks = ClockSampler(device_index)
+    clocks.start()
+    per_call, total_ms = [], 0.0
+    while True:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(reps):
+            binding.prefill(q, k_pool, v_pool, bt, ctx32, qlen, w.scale, part, out, ws)
+        t1.record()
+        torch.cuda.synchronize()
+        block = t0.elapsed_time(t1)
+        per_call.append(block / reps)
+        total_ms += block
+        if total_ms >= args.min_seconds * 1e3 or len(per_call) >= 10_000:
+            break
+    clock_info = clocks.stop()
+    ms = statistics.median(per_call)
     pairs = B * int(np.sum(np.arange(prior + 1, prior + chunk + 1)))   # (query, key) pairs per head
     flops = 4.0 * D * Hq * pairs
     tflops = flops / (ms * 1e-3) / 1e12
@@ -902,8 +916,13 @@ def run_prefill_bench(args, device_index):
     except Exception:
         peak, kind = 1590.0, "fallback"
     kv_bytes = B * (prior + chunk) * Hkv * D * 2 * 2
+    q10, q90 = (float(np.percentile(per_call, x)) for x in (10, 90))
     return {"metric": "paged chunked-prefill attention TFLOP/s (causal, bf16 in, fp32 accumulate)",
             "value": round(tflops, 2), "unit": "TFLOP/s", "impl": "ours", "ms_per_call": round(ms, 4),
+            "ms_per_call_p10_p90": [round(q10, 4), round(q90, 4)], "blocks": len(per_call),
+            "calls_per_block": reps, "clocks": clock_info,
+            "tflops_per_sm_ghz": (round(tflops / (clock_info["sm_mhz"] / 1000.0), 1)
+                                  if clock_info and clock_info.get("sm_mhz") else None),
             "config": {"workload": f"prefill: batch {B}, {prior} prior + {chunk} new tokens, "
                                    f"{Hq}q/{Hkv}kv heads, head_dim {D}, bf16, block {bs}",
                        "partition_tokens": part,

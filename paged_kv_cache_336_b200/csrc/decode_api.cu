@@ -573,10 +573,46 @@ class PlanStaging {
  public:
   static constexpr int kMaxSlots = 64;
 
+  // Pieces whose device ranges lie close together (gaps of at most
+  // kMergeGap bytes, the layouts' alignment padding) go up as one copy: each
+  // cudaMemcpyAsync is a separate operation on the stream, ahead of the
+  // kernels that read the plan. The padding between merged pieces receives
+  // whatever the staging slot held there; nothing reads it.
+  static constexpr size_t kMergeGap = 4096;
+  static constexpr int kMaxPieces = 8;
+
   pa_status_t upload(const UploadPiece* pieces, int n, cudaStream_t stream) {
+    if (n > kMaxPieces) return fail(PA_ERR_INVALID_ARG, "plan upload: %d pieces (at most %d)", n, kMaxPieces);
+    UploadPiece p[kMaxPieces];
+    int m = 0;
+    for (int i = 0; i < n; ++i)
+      if (pieces[i].bytes > 0) p[m++] = pieces[i];
+    if (m == 0) return PA_OK;
+    for (int i = 1; i < m; ++i)  // by destination
+      for (int j = i; j > 0 && static_cast<uint8_t*>(p[j].dst) < static_cast<uint8_t*>(p[j - 1].dst); --j)
+        std::swap(p[j], p[j - 1]);
+    struct Run {
+      uint8_t* dst;
+      size_t bytes;
+      int first, last;  // pieces [first, last)
+    };
+    Run runs[kMaxPieces];
+    int nr = 0;
+    for (int i = 0; i < m; ++i) {
+      uint8_t* d = static_cast<uint8_t*>(p[i].dst);
+      if (nr > 0) {
+        Run& r = runs[nr - 1];
+        uint8_t* end = r.dst + r.bytes;
+        if (d >= end && static_cast<size_t>(d - end) <= kMergeGap) {
+          r.bytes = static_cast<size_t>(d + p[i].bytes - r.dst);
+          r.last = i + 1;
+          continue;
+        }
+      }
+      runs[nr++] = Run{d, p[i].bytes, i, i + 1};
+    }
     size_t total = 0;
-    for (int i = 0; i < n; ++i) total += (pieces[i].bytes + 15) & ~static_cast<size_t>(15);
-    if (total == 0) return PA_OK;
+    for (int k = 0; k < nr; ++k) total += (runs[k].bytes + 15) & ~static_cast<size_t>(15);
     std::lock_guard<std::mutex> lock(mu_);
     Slot* sl = nullptr;
     pa_status_t st = acquire(&sl);
@@ -592,13 +628,13 @@ class PlanStaging {
       sl->cap = cap;
     }
     size_t off = 0;
-    for (int i = 0; i < n; ++i) {
-      if (pieces[i].bytes == 0) continue;
-      std::memcpy(sl->host + off, pieces[i].src, pieces[i].bytes);
-      if ((err = cudaMemcpyAsync(pieces[i].dst, sl->host + off, pieces[i].bytes, cudaMemcpyHostToDevice,
-                                 stream)) != cudaSuccess)
+    for (int k = 0; k < nr; ++k) {
+      const Run& r = runs[k];
+      for (int i = r.first; i < r.last; ++i)
+        std::memcpy(sl->host + off + (static_cast<uint8_t*>(p[i].dst) - r.dst), p[i].src, p[i].bytes);
+      if ((err = cudaMemcpyAsync(r.dst, sl->host + off, r.bytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess)
         return fail(PA_ERR_CUDA, "plan upload: %s", cudaGetErrorString(err));
-      off += (pieces[i].bytes + 15) & ~static_cast<size_t>(15);
+      off += (r.bytes + 15) & ~static_cast<size_t>(15);
     }
     if ((err = cudaEventRecord(sl->done, stream)) != cudaSuccess)
       return fail(PA_ERR_CUDA, "plan staging record: %s", cudaGetErrorString(err));
