@@ -216,11 +216,15 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
  * pa_decode_split).
  *
  * Host plans (this call and pa_prefill): the plan built from the host
- * arrays is copied into a page-locked staging slot owned by the library and
- * uploaded from there on `stream`; the call returns without waiting for the
- * stream. Slots are reused once their upload has completed, so these two
- * calls must not be captured into a CUDA graph (a replay would read a slot
- * that has since been reused).
+ * arrays reaches the device on `stream` without the call waiting for the
+ * stream. A plan of up to 30 KB (a few hundred work items) travels as the
+ * parameters of a small kernel, so the call may be captured into a CUDA
+ * graph: a replay uploads the plan captured with it. A larger plan is copied
+ * into a page-locked staging slot owned by the library and uploaded from
+ * there; slots are reused once their upload has completed, so such a call
+ * is refused with PA_ERR_UNSUPPORTED while `stream` is being captured (a
+ * replay would read a slot that has since been reused), before anything is
+ * enqueued.
  * ------------------------------------------------------------------------- */
 size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                               int head_dim, int block_size,

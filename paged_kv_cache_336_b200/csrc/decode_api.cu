@@ -554,8 +554,10 @@ pa_status_t run_decode(const DecodeReq& r, bool split, int partition_tokens, voi
 
 // ---- uploads of host-built plans --------------------------------------------------------
 // pa_prefill and pa_decode_shared_prefix build small plans on the host (work
-// items, schedules, group arrays). An upload from pageable memory may make
-// the host wait for the stream, so each call copies its plan into a slot of
+// items, schedules, group arrays). Plans of up to 30 KB go up as kernel
+// parameters (upload_plan, below). For larger ones: an upload from pageable
+// memory may make the host wait for the stream, so each call copies its plan
+// into a slot of
 // a pool of page-locked buffers (one pool per device) and uploads it from
 // there with cudaMemcpyAsync, which returns at once. An event recorded after
 // the uploads marks the slot busy until the copies have read it. A call takes
@@ -694,10 +696,97 @@ class PlanStaging {
   int next_ = 0;
 };
 
-// The current device's ring (rings live until the process exits).
+// Plans of up to kParamPlanBytes travel as the parameters of a one-CTA
+// scatter kernel instead: the driver copies a launch's parameters when the
+// launch is enqueued, so the host buffer is free at once, no copy-engine
+// operation sits on the stream ahead of the plan's kernels, and the call can
+// be captured into a CUDA graph (a replay scatters the captured plan again).
+// Three parameter sizes, so that a small plan does not carry 30 KB.
+constexpr int kParamPlanPieces = 8;
+
+template <size_t N>
+struct PlanParams {
+  uint8_t* dst[kParamPlanPieces];
+  uint32_t bytes[kParamPlanPieces];
+  uint32_t off[kParamPlanPieces];  // piece i's bytes start at data + off[i] (16-byte aligned)
+  int n;
+  alignas(16) uint8_t data[N];
+};
+
+// One 16-byte chunk of the packed data per thread, 32 threads per CTA: lanes
+// reading different parameter addresses are served one address at a time, so
+// the chunks are spread over as many CTAs (and SMs) as there are 512-byte
+// slices.
+template <size_t N>
+__global__ void __launch_bounds__(32) plan_scatter_kernel(const __grid_constant__ PlanParams<N> p) {
+  const uint32_t c = blockIdx.x * 32 + threadIdx.x;
+  for (int i = 0; i < p.n; ++i) {
+    const uint32_t c0 = p.off[i] / 16, nb = p.bytes[i];
+    if (c < c0 || c >= c0 + (nb + 15) / 16) continue;
+    const uint32_t b0 = (c - c0) * 16;
+    uint8_t* d = p.dst[i] + b0;
+    const uint8_t* src = p.data + p.off[i] + b0;
+    if (b0 + 16 <= nb && (reinterpret_cast<uintptr_t>(d) & 15u) == 0) {
+      *reinterpret_cast<uint4*>(d) = *reinterpret_cast<const uint4*>(src);
+    } else {
+      for (uint32_t k = 0; k < 16 && b0 + k < nb; ++k) d[k] = src[k];
+    }
+    return;
+  }
+}
+
+template <size_t N>
+pa_status_t scatter_plan(const UploadPiece* p, int m, size_t total, cudaStream_t stream) {
+  thread_local PlanParams<N> prm;
+  size_t off = 0;
+  prm.n = m;
+  for (int i = 0; i < m; ++i) {
+    prm.dst[i] = static_cast<uint8_t*>(p[i].dst);
+    prm.bytes[i] = static_cast<uint32_t>(p[i].bytes);
+    prm.off[i] = static_cast<uint32_t>(off);
+    std::memcpy(prm.data + off, p[i].src, p[i].bytes);
+    off += (p[i].bytes + 15) & ~static_cast<size_t>(15);
+  }
+  const unsigned ctas = static_cast<unsigned>((total / 16 + 31) / 32);
+  plan_scatter_kernel<N><<<ctas, 32, 0, stream>>>(prm);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "plan scatter launch: %s", cudaGetErrorString(err));
+  return PA_OK;
+}
+
+constexpr size_t kParamPlanBytes = 30 * 1024;
+
+// Uploads a host plan on `stream`: as kernel parameters when it fits (set
+// PAGEDKV_PLAN_UPLOAD=staging to force the other path, for tests), else
+// through the current device's staging ring (rings live until the process
+// exits). A staged upload is refused while the stream is being captured.
 pa_status_t upload_plan(const UploadPiece* pieces, int n, cudaStream_t stream) {
+  UploadPiece p[kParamPlanPieces];
+  int m = 0;
+  size_t total = 0;
+  for (int i = 0; i < n; ++i) {
+    if (pieces[i].bytes == 0) continue;
+    if (m == kParamPlanPieces) return fail(PA_ERR_INVALID_ARG, "plan upload: more than %d pieces", kParamPlanPieces);
+    p[m++] = pieces[i];
+    total += (pieces[i].bytes + 15) & ~static_cast<size_t>(15);
+  }
+  if (m == 0) return PA_OK;
+  const char* mode = std::getenv("PAGEDKV_PLAN_UPLOAD");
+  const bool force_staging = mode != nullptr && std::strcmp(mode, "staging") == 0;
+  if (!force_staging && total <= kParamPlanBytes) {
+    if (total <= 2048) return scatter_plan<2048>(p, m, total, stream);
+    if (total <= 8192) return scatter_plan<8192>(p, m, total, stream);
+    return scatter_plan<kParamPlanBytes>(p, m, total, stream);
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t err = cudaStreamIsCapturing(stream, &cap);
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "cudaStreamIsCapturing: %s", cudaGetErrorString(err));
+  if (cap != cudaStreamCaptureStatusNone)
+    return fail(PA_ERR_UNSUPPORTED,
+                "a host plan of %zu bytes (more than %zu, or staging forced) is uploaded from a "
+                "reused staging slot and cannot be captured into a graph", total, kParamPlanBytes);
   int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
   static std::mutex mu;
   static std::vector<PlanStaging*> rings;
@@ -708,7 +797,7 @@ pa_status_t upload_plan(const UploadPiece* pieces, int n, cudaStream_t stream) {
     if (rings[dev] == nullptr) rings[dev] = new PlanStaging();
     ring = rings[dev];
   }
-  return ring->upload(pieces, n, stream);
+  return ring->upload(p, m, stream);
 }
 
 // ---- shared-prefix decode ------------------------------------------------------------

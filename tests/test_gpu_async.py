@@ -1,11 +1,13 @@
 """Calls that build a plan on the host (pa_prefill, pa_decode_shared_prefix)
 enqueue their work and return without waiting for the stream.
 
-Their plans are uploaded from the library's page-locked staging ring, so a
-call issued behind a long-running kernel returns while that kernel still
-runs. Back-to-back calls (more than the ring has slots) behind a ~0.5 s
-spin kernel must all return in a small fraction of it, with the stream still
-busy afterwards, and their results must still match the oracle.
+Small plans go up as the parameters of a scatter kernel; larger ones (or
+all, with PAGEDKV_PLAN_UPLOAD=staging) from the library's page-locked
+staging ring. Either way a call issued behind a long-running kernel returns
+while that kernel still runs. Back-to-back calls behind a ~0.5 s spin kernel
+must all return in a small fraction of it, with the stream still busy
+afterwards, and their results must still match the oracle. Both upload
+paths are run.
 """
 
 import time
@@ -22,7 +24,10 @@ from gpu_util import check_close, device_tables, setup, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def test_plan_uploads_do_not_wait_for_the_stream():
+@pytest.mark.parametrize("upload", ["params", "staging"])
+def test_plan_uploads_do_not_wait_for_the_stream(monkeypatch, upload):
+    if upload == "staging":
+        monkeypatch.setenv("PAGEDKV_PLAN_UPLOAD", "staging")
     w = workloads.random_small(31, num_seqs=3, num_q_heads=8, num_kv_heads=2, head_dim=128,
                                block_size=16, dtype=workloads.BF16, max_ctx=160,
                                fixed_lens=[160, 70, 20])
