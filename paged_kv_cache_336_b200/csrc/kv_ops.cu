@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // grid.y walks pairs, grid.x x blockDim.x walks the 16-byte units of a block.
+constexpr int kCopyUnroll = 4;  // 16-byte units of K and of V in flight per thread
+
 __global__ void __launch_bounds__(256)
     copy_blocks_kernel(uint4* k_pool, uint4* v_pool, const int64_t* __restrict__ pairs,
                        int num_pairs, int64_t units_per_block, int num_blocks,
@@ -73,10 +75,31 @@ __global__ void __launch_bounds__(256)
     const uint4* vs = v_pool + src * units_per_block;
     uint4* kd = k_pool + dst * units_per_block;
     uint4* vd = v_pool + dst * units_per_block;
-    for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units_per_block;
-         u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-      kd[u] = ks[u];
-      vd[u] = vs[u];
+    // Each thread loads kCopyUnroll units of K and of V before storing any:
+    // source and destination lie in the same pool, so the compiler would not
+    // move a later load above an earlier store, and a plain loop waits out a
+    // memory round trip per unit. A pair's source and destination are
+    // different blocks, and no destination is another pair's source.
+    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x * kCopyUnroll;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x * kCopyUnroll + threadIdx.x;
+         base < units_per_block; base += step) {
+      uint4 kr[kCopyUnroll], vr[kCopyUnroll];
+#pragma unroll
+      for (int i = 0; i < kCopyUnroll; ++i) {
+        const int64_t u = base + static_cast<int64_t>(i) * blockDim.x;
+        if (u < units_per_block) {
+          kr[i] = ks[u];
+          vr[i] = vs[u];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kCopyUnroll; ++i) {
+        const int64_t u = base + static_cast<int64_t>(i) * blockDim.x;
+        if (u < units_per_block) {
+          kd[u] = kr[i];
+          vd[u] = vr[i];
+        }
+      }
     }
   }
 }
@@ -228,7 +251,7 @@ pa_status_t pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* src_dst_pa
                     (long long)h[2 * i]);
   }
   const int64_t upb = static_cast<int64_t>(block_bytes / 16);
-  const int gx = static_cast<int>(std::min<int64_t>((upb + 1023) / 1024, 64));
+  const int gx = static_cast<int>(std::min<int64_t>((upb + 256 * kCopyUnroll - 1) / (256 * kCopyUnroll), 64));
   const int gy = std::min(num_pairs, 65535);
   copy_blocks_kernel<<<dim3(gx, gy), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), src_dst_pairs, num_pairs, upb,
