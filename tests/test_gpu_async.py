@@ -24,10 +24,15 @@ from gpu_util import check_close, device_tables, setup, to_f64
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("prefix_kernel", ["mma_sync", "tcgen05"])
 @pytest.mark.parametrize("upload", ["params", "staging"])
-def test_plan_uploads_do_not_wait_for_the_stream(monkeypatch, upload):
+def test_plan_uploads_do_not_wait_for_the_stream(monkeypatch, upload, prefix_kernel):
+    # staging + tcgen05: the prefix plan's pieces lie far apart in the
+    # workspace (items, then the Q-tile list), so they go up as two copies
     if upload == "staging":
         monkeypatch.setenv("PAGEDKV_PLAN_UPLOAD", "staging")
+    if prefix_kernel == "tcgen05":
+        monkeypatch.setenv("PAGEDKV_PREFIX_KERNEL", "tcgen05")
     w = workloads.random_small(31, num_seqs=3, num_q_heads=8, num_kv_heads=2, head_dim=128,
                                block_size=16, dtype=workloads.BF16, max_ctx=160,
                                fixed_lens=[160, 70, 20])
