@@ -766,11 +766,13 @@ def seq_context(w, s: int) -> int:
     return int(w.context_lens[s])
 
 
-def time_oracle(w, budget_s: float, seed: int = 0, threads: int = 1):
+def time_oracle(w, budget_s: float, seed: int = 0, threads: int = 1, per_kv_head: bool = False):
     """Times the float64 oracle on whole sequences of the workload (all query
     heads of each), with `threads` BLAS/torch threads, until ~budget_s seconds
-    of work are done. Returns (GB/s of algorithmic bytes, tokens/s,
-    description, seconds)."""
+    of work are done. With per_kv_head, the unit is one (sequence, KV head):
+    the sequence's K/V for that head and its group of query heads (a long
+    sequence is seconds of oracle work; one KV head is an eighth of it).
+    Returns (GB/s of algorithmic bytes, tokens/s, description, seconds)."""
     import torch
     from threadpoolctl import threadpool_limits
     import oracle
@@ -781,6 +783,7 @@ def time_oracle(w, budget_s: float, seed: int = 0, threads: int = 1):
     Hkv, bs, D = w.num_kv_heads, w.block_size, w.head_dim
     done_bytes = 0
     done_seqs = 0
+    done_units = 0
     elapsed = 0.0
     prev_threads = torch.get_num_threads()
     torch.set_num_threads(threads)
@@ -799,34 +802,52 @@ def time_oracle(w, budget_s: float, seed: int = 0, threads: int = 1):
                 _ORACLE_INPUT[:] = [key, (kp, vp, q)]
             kp, vp, q = _ORACLE_INPUT[1]
             table = np.arange(nb)[None, :]
-            t0 = time.perf_counter()
-            oracle.paged_decode(q, kp, vp, table, [ctx], w.scale)
-            elapsed += time.perf_counter() - t0
-            done_bytes += decode_bytes(w, np.array([ctx]))
+            G = w.num_q_heads // Hkv
+            for h in (rng.permutation(Hkv) if per_kv_head else [None]):
+                if h is None:
+                    kh, vh, qh = kp, vp, q
+                else:   # one KV head and its query heads, as contiguous arrays
+                    kh = np.ascontiguousarray(kp[:, h:h + 1])
+                    vh = np.ascontiguousarray(vp[:, h:h + 1])
+                    qh = np.ascontiguousarray(q[:, h * G:(h + 1) * G])
+                t0 = time.perf_counter()
+                oracle.paged_decode(qh, kh, vh, table, [ctx], w.scale)
+                elapsed += time.perf_counter() - t0
+                done_bytes += decode_bytes(w, np.array([ctx])) / (Hkv if h is not None else 1)
+                done_units += 1
+                if elapsed >= budget_s:   # at least one unit per call
+                    break
             done_seqs += 1
-            if elapsed >= budget_s:   # at least one whole sequence per call
+            if elapsed >= budget_s:
                 break
     torch.set_num_threads(prev_threads)
-    desc = (f"{done_seqs} of {len(w.decode_seqs)} sequences (all {w.num_q_heads} query heads each, "
-            f"the workload's context lengths and N(0,1) values) of the {w.name} workload, "
+    if per_kv_head:
+        what = (f"{done_units} (sequence, KV head) units of {len(w.decode_seqs) * Hkv} (one KV head "
+                f"and its {w.num_q_heads // Hkv} query heads each")
+        seqs_done = done_units / Hkv
+    else:
+        what = f"{done_seqs} of {len(w.decode_seqs)} sequences (all {w.num_q_heads} query heads each"
+        seqs_done = done_seqs
+    desc = (f"{what}, the workload's context lengths and N(0,1) values) of the {w.name} workload, "
             f"{elapsed:.2f} s, float64 NumPy oracle, {threads} thread{'s' if threads > 1 else ''}")
-    return done_bytes / elapsed / 1e9, done_seqs / elapsed, desc, elapsed
+    return done_bytes / elapsed / 1e9, seqs_done / elapsed, desc, elapsed
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return None
     w = make_workload(args.workload, 0, args.batch)
-    # each step: a bounded sample of the workload (at least one whole sequence),
-    # sized so that the whole run ends within a few minutes; with long
-    # sequences (seconds of oracle work each) every step times the same one
+    # each step: a bounded sample of the workload, sized so that the whole run
+    # ends within a few minutes. Long sequences (seconds of oracle work each)
+    # are sampled by (sequence, KV head) units, an eighth of a sequence at the
+    # headline, and every step starts from the same sequence
     per_step = min(10.0, 60.0 / max(1, args.steps + args.warmup))
     long_seqs = float(np.max(w.context_lens)) >= 32768
     for _ in range(args.warmup):
-        time_oracle(w, per_step / 4)
+        time_oracle(w, per_step / 4, per_kv_head=long_seqs)
     vals, tok, descs, secs = [], [], [], 0.0
     for i in range(args.steps):
-        g, t, d, el = time_oracle(w, per_step, seed=0 if long_seqs else i)
+        g, t, d, el = time_oracle(w, per_step, seed=0 if long_seqs else i, per_kv_head=long_seqs)
         vals.append(g)
         tok.append(t)
         descs.append(d)
