@@ -696,7 +696,7 @@ class PlanStaging {
   int next_ = 0;
 };
 
-// Plans of up to kParamPlanBytes travel as the parameters of a one-CTA
+// Plans of up to kParamPlanBytes travel as the parameters of a small
 // scatter kernel instead: the driver copies a launch's parameters when the
 // launch is enqueued, so the host buffer is free at once, no copy-engine
 // operation sits on the stream ahead of the plan's kernels, and the call can
