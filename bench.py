@@ -263,11 +263,14 @@ def kernel_source_hash(names=DECODE_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, kind: str = "decode", sources=None, mode: str = "split"):
+def profiled_traffic(workload: str, kind: str = "decode", sources=None, mode: str = "split",
+                     algorithmic: float | None = None):
     """DRAM bytes per call from the committed ncu summary
     profiles/<kind>_<workload>_traffic.txt (decode calls of another route:
     <route>_<workload>_traffic.txt), if it was taken on the current kernel
-    source; else None."""
+    source and (when `algorithmic` is given) on a call of the same
+    algorithmic bytes, within 1% (not, say, a smaller --batch of the same
+    workload); else None."""
     if kind == "decode" and mode != "split":
         kind = mode
     if sources is None:
@@ -282,7 +285,12 @@ def profiled_traffic(workload: str, kind: str = "decode", sources=None, mode: st
                     kv[k.strip()] = v.strip()
         if kv.get("kernel_source_sha256_16") != kernel_source_hash(sources):
             return None
-        return int(kv["dram_bytes_per_launch"])
+        dram = int(kv["dram_bytes_per_launch"])
+        if algorithmic is not None and "traffic_over_algorithmic" in kv:
+            captured = dram / float(kv["traffic_over_algorithmic"])
+            if abs(captured - algorithmic) > 0.01 * algorithmic:
+                return None
+        return dram
     except Exception:
         return None
 
@@ -529,7 +537,7 @@ def summarize(ds, reps, calls, steps, world, workload_key, mode, peak, peak_kind
         "unit": "GB/s",
         "frac": round(achieved / peak, 4),
         "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
-        "traffic": profiled_traffic(workload_key, mode=mode),
+        "traffic": profiled_traffic(workload_key, mode=mode, algorithmic=dbytes / n_calls),
         "algorithmic_bytes_per_launch": int(dbytes / n_calls),
         "avg_launch_us": round(dus / n_calls, 2),
         "launch_us_p10_p50_p90": [pct(calls, 10), pct(calls, 50), pct(calls, 90)],
