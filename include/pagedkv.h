@@ -195,6 +195,14 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
                                    int partition_tokens, void* out, uint32_t* dev_err,
                                    void* stream);
 
+/* Test aid for the contract above: sets every byte of the static scratch's
+ * control header (its first 256 bytes, the ticket counters) to `byte` on
+ * `stream`, in the current context, as a call that ended early (a device
+ * timeout) could leave it. The next pa_decode_split_static call must still
+ * be correct, since each call clears the header after its host checks.
+ * Enqueues one memset; allocates nothing. */
+pa_status_t pa_decode_split_static_fill_header(uint8_t byte, void* stream);
+
 /* ---------------------------------------------------------------------------
  * pa_decode_shared_prefix - the same result as pa_decode, reading each
  * shared prefix once. Sequences that share their first blocks (prefix

@@ -91,6 +91,7 @@ _SIGNATURES = {
                              _P, _P, _P]),
     "pa_decode_split_static": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                                     _P, _P, _P]),
+    "pa_decode_split_static_fill_header": (_I, [ctypes.c_uint8, _P]),
     "pa_decode_shared_prefix_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
     "pa_decode_shared_prefix": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                                      _I, _P, _P, _P, _P, _SZ, _P, _P, _P]),

@@ -1572,6 +1572,15 @@ pa_status_t pa_decode_split_static(const void* q, const void* k_pool, const void
                     /*clear_header=*/true);
 }
 
+pa_status_t pa_decode_split_static_fill_header(uint8_t byte, void* stream) {
+  void* scratch = nullptr;
+  pa_status_t st = static_scratch_address(&scratch);
+  if (st != PA_OK) return st;
+  const cudaError_t err = cudaMemsetAsync(scratch, byte, kWorkspaceHeader, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return fail(PA_ERR_CUDA, "filling the static header: %s", cudaGetErrorString(err));
+  return ok();
+}
+
 size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                               int head_dim, int block_size,
                                               int max_blocks_per_seq, int partition_tokens) {

@@ -7,8 +7,9 @@ tests call it through the C ABI and compare it with pa_decode_split, which
 takes a caller workspace, and with the float64 oracle, within the tolerances
 used by every decode test (fp32 max-abs 1e-5; bf16 max-abs 2e-2 and
 mean-abs 2e-3), on two calls in a row, since the array keeps the previous
-call's contents. Oversized requests, and requests refused for any other
-reason, must be turned away before anything is enqueued.
+call's contents, and after the array's header was left dirty (as a call that
+timed out could leave it). Oversized requests, and requests refused for any
+other reason, must be turned away before anything is enqueued.
 
 This file sorts last so that a run stopping at the first failure has run
 every other test first; it also passes when run alone in a fresh process.
@@ -120,3 +121,34 @@ def test_static_scratch_refuses_oversized_requests():
 
     # a call after the refusals still matches the oracle
     _static_matches(workloads.BF16, 8)
+
+
+@pytest.mark.parametrize("split_kernel", ["ticket", "stream"])
+def test_static_call_after_a_dirty_header(monkeypatch, split_kernel):
+    """A call that ended early (a device timeout) can leave the shared array's
+    ticket counters non-zero. Each static call clears the header after its
+    host checks, so a call that follows a dirty header is still correct: the
+    test fills the header with 0x5A bytes (counters 0x5A5A5A5A, far past any
+    ticket) through the library's test aid, then compares a static call with
+    the oracle. Without the clear, the ticket kernel would find no tickets
+    and leave the output unwritten."""
+    monkeypatch.setenv("PAGEDKV_SPLIT_KERNEL", split_kernel)
+    torch.cuda.set_device(0)
+    lib = binding.library()
+    w = workloads.random_small(77, num_seqs=9, num_q_heads=16, num_kv_heads=2, head_dim=128,
+                               block_size=16, dtype=workloads.BF16, max_ctx=400,
+                               fixed_lens=[0, 1, 400])
+    bm, k_pool, v_pool = setup(w)
+    q = workloads.draw_queries(w, 9, device="cuda")
+    bt, ctx, tables, ctx_np = device_tables(bm, list(range(9)))
+    want = oracle.paged_decode(to_f64(q), to_f64(k_pool), to_f64(v_pool), tables, ctx_np, w.scale)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for call in range(2):
+        assert lib.pa_decode_split_static_fill_header(0x5A, stream) == binding.PA_OK
+        out = torch.full_like(q, float("nan"))
+        status = _call_static(q, k_pool, v_pool, bt, ctx, w.scale, 48, out, err)
+        assert status == binding.PA_OK, lib.pa_last_error_string()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        check_close(to_f64(out), want, workloads.BF16, f"static call {call} after a dirty header")
