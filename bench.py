@@ -269,8 +269,9 @@ def profiled_traffic(workload: str, kind: str = "decode", sources=None, mode: st
     profiles/<kind>_<workload>_traffic.txt (decode calls of another route:
     <route>_<workload>_traffic.txt), if it was taken on the current kernel
     source and (when `algorithmic` is given) on a call of the same
-    algorithmic bytes, within 1% (not, say, a smaller --batch of the same
-    workload); else None."""
+    algorithmic bytes, within 5% (the bench cycles decode states whose
+    contexts grow a token per step; a smaller --batch of the same workload
+    differs several-fold); else None."""
     if kind == "decode" and mode != "split":
         kind = mode
     if sources is None:
@@ -288,7 +289,7 @@ def profiled_traffic(workload: str, kind: str = "decode", sources=None, mode: st
         dram = int(kv["dram_bytes_per_launch"])
         if algorithmic is not None and "traffic_over_algorithmic" in kv:
             captured = dram / float(kv["traffic_over_algorithmic"])
-            if abs(captured - algorithmic) > 0.01 * algorithmic:
+            if abs(captured - algorithmic) > 0.05 * algorithmic:
                 return None
         return dram
     except Exception:
