@@ -4,8 +4,8 @@ Forked sequences share their prompt's blocks; the shared-prefix route reads
 them once per KV head for the whole group and must still return plain decode
 attention. Small cases are compared with the full float64 oracle (several
 groups, a group wider than one CTA's rows, sequences in no group, block
-sizes 16 and 32); the full-size prefix-sharing workloads on every output
-row as well.
+sizes 16 and 32, head_dim 128 and 64); the full-size prefix-sharing
+workloads on every output row as well.
 Both prefix-pass kernels are covered: the mma.sync one (default, 64 query
 rows per CTA) and the tcgen05 one (PAGEDKV_PREFIX_KERNEL=tcgen05, 128).
 """
@@ -35,8 +35,19 @@ def kernel(request, monkeypatch):
                                            (16, 16, 20), (6, 32, 7)])
 @pytest.mark.parametrize("split_kernel", ["ticket", "stream"])
 def test_shared_prefix_small_matches_oracle(monkeypatch, kernel, split_kernel, G, bs, branches):
+    _small_case(monkeypatch, split_kernel, G, bs, branches, 128)
+
+
+@pytest.mark.parametrize("G,bs,branches", [(4, 16, 16), (8, 32, 12)])
+@pytest.mark.parametrize("split_kernel", ["ticket", "stream"])
+def test_shared_prefix_head_dim_64(monkeypatch, kernel, split_kernel, G, bs, branches):
+    """The head_dim 64 instances of both prefix kernels and both suffix kernels."""
+    _small_case(monkeypatch, split_kernel, G, bs, branches, 64)
+
+
+def _small_case(monkeypatch, split_kernel, G, bs, branches, D):
     monkeypatch.setenv("PAGEDKV_SPLIT_KERNEL", split_kernel)
-    Hkv, D = 2, 128
+    Hkv = 2
     rng = np.random.default_rng(40 + G + bs)
     NB = 400
     bm = binding.BlockManager(NB, bs, 64, rng.permutation(NB).astype(np.int32))
